@@ -1,0 +1,60 @@
+"""Plants plausible mistakes in a scratch copy of the oracle (on the CPU) and
+checks that the pin suite rejects every one of them.  The committed oracle is
+never modified; each mutant is compiled into its own temporary tree."""
+import os
+import shutil
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# (text in the oracle, its mutated form, what the mistake is)
+MUTANTS = [
+    ("double wj = a1[j] - lambda * a2[j];", "double wj = a1[j] + lambda * a2[j];", "lambda sign"),
+    ("1.0 / sqrt((double)d)", "1.0 / sqrt((double)(2 * d))", "scale over the full head width"),
+    ("diff_attention_row(qrow, qrow + d, kb, kb + d", "diff_attention_row(qrow, qrow, kb, kb + d", "branch-2 query half"),
+    ("diff_attention_row(qrow, qrow + d, kb, kb + d", "diff_attention_row(qrow, qrow + d, kb, kb", "branch-2 key half"),
+    ("int64_t n_keys = causal ? (int64_t)i + 1 : (int64_t)N;\n        const float *qrow",
+     "int64_t n_keys = causal ? (int64_t)i : (int64_t)N;\n        const float *qrow", "causal diagonal"),
+    ("int g = (2 * p) / group;", "int g = p / group;", "GQA head mapping"),
+    ("const float *qb = q + ((int64_t)b * N + i) * tok_q + (int64_t)(2 * p + 1) * d;",
+     "const float *qb = q + ((int64_t)b * N + i) * tok_q + (int64_t)(2 * p) * d;", "V2 pair member"),
+    ("const float *qa = q + ((int64_t)b * Hq + 2 * p) * d;", "const float *qa = q + ((int64_t)b * Hq + p) * d;", "decode query head"),
+    ("double inv_rms = 1.0 / sqrt(ss / (double)dv + eps);", "double inv_rms = 1.0 / sqrt(ss + eps);", "RMS mean"),
+    ("o[c] = o[c] * inv_rms * gc * (1.0 - lambda_init);", "o[c] = o[c] * inv_rms * gc * lambda_init;", "post-norm scale"),
+    ("lambda_out[h] = exp(dot1) - exp(dot2) + linit;", "lambda_out[h] = exp(dot1) + exp(dot2) + linit;", "lambda re-parameterisation sign"),
+    ("return 0.8 - 0.6 * exp(-0.3 * (double)(layer - 1));", "return 0.8 - 0.6 * exp(-0.3 * (double)(layer));", "layer base"),
+    ("x[j] = exp(x[j] - m);", "x[j] = exp(x[j]);", "softmax without the max shift"),
+    ("for (int c = 0; c < dv; ++c) o[c] += wj * (double)vj[c];", "for (int c = 0; c < dv; ++c) o[c] += a1[j] * (double)vj[c];", "second map dropped"),
+]
+
+
+def _run_mutant(tmp_root, n, before, after):
+    src = open(os.path.join(ROOT, "oracle", "diffattn_oracle.c")).read()
+    assert before in src, before
+    d = os.path.join(tmp_root, "m%d" % n)
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(d, "oracle"),
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    with open(os.path.join(d, "oracle", "diffattn_oracle.c"), "w") as f:
+        f.write(src.replace(before, after, 1))
+    os.makedirs(os.path.join(d, "tests"))
+    for name in ("conftest.py", "test_oracle_pins.py"):
+        shutil.copy(os.path.join(ROOT, "tests", name), os.path.join(d, "tests", name))
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(d, "tests", "golden"))
+    os.symlink(os.path.join(ROOT, "differential_attention_sm_b200"),
+               os.path.join(d, "differential_attention_sm_b200"))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        os.path.join("tests", "test_oracle_pins.py")],
+                       cwd=d, capture_output=True, text=True, timeout=600)
+    return r.returncode
+
+
+def test_pins_reject_every_planted_mistake(tmp_path):
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        rcs = list(ex.map(lambda a: _run_mutant(str(tmp_path), *a),
+                          [(n, b, a) for n, (b, a, _) in enumerate(MUTANTS)]))
+    missed = [MUTANTS[n][2] for n, rc in enumerate(rcs) if rc == 0]
+    assert not missed, "pins did not notice: %s" % missed

@@ -1,0 +1,326 @@
+"""Pins of the fp64 oracle against facts the pages and the mathematics fix.
+
+None of these tests re-types the oracle's formula: each checks the oracle
+against a value the pages print, a closed form, an invariant, or an
+independent library routine (torch's scaled_dot_product_attention and
+rms_norm in float64).  Together they fail on a dropped term, a flipped sign,
+a wrong scale, a swapped branch half, a wrong head/KV mapping or a wrong
+mask.
+
+Sources: "Differential Transformer" (Ultralytics glossary), section
+"Cómo funciona la atención diferencial" [G]; "Atención Diferencial (V2)"
+(ai-engineering.academy), sections "La idea diferencial", "V1 vs V2: la
+diferencia", "Implementación" and "Ejercicios" [L].
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle as O
+from differential_attention_sm_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def sdpa(q, k, v, causal=False, enable_gqa=False):
+    """torch float64 SDPA on [B, N, H, D] tensors (scale 1/sqrt(D_q))."""
+    qt, kt, vt = (x.double().permute(0, 2, 1, 3) for x in (q, k, v))
+    o = F.scaled_dot_product_attention(qt, kt, vt, is_causal=causal,
+                                       enable_gqa=enable_gqa)
+    return o.permute(0, 2, 1, 3)
+
+
+def all_rows_v1(B, N, H):
+    return np.arange(B * N * H)
+
+
+def rand(*shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(*shape, generator=g)
+
+
+# --------------------------------------------------------------------------
+# [G] worked example: seed 0, n=6, d=8, lambda 0.8 -> "0.20; 13 of 36"
+# --------------------------------------------------------------------------
+def test_worked_example_matches_printed_line():
+    gold = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
+    q1, k1, q2, k2, v = I.worked_example()
+    n = gold["n"]
+    q = torch.cat([q1, q2], -1).reshape(1, n, 1, 2 * gold["d"])
+    k = torch.cat([k1, k2], -1).reshape(1, n, 1, 2 * gold["d"])
+    vv = v.reshape(1, n, 1, gold["dv"])
+    out, w = O.v1_rows(q, k, vv, [gold["lambda"]], np.arange(n), causal=False,
+                       return_weights=True)
+    sums = w.sum(axis=1)
+    assert all("%.2f" % s == gold["printed_row_sum"] for s in sums)
+    assert int((w < 0).sum()) == gold["negative_weights"]
+    assert w.size == gold["total_weights"]
+    # the output is the weights applied to V (the page's `diff @ v`)
+    assert np.allclose(out, w @ v.double().numpy(), rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# [G]: every row of the difference map sums to 1 - lambda, for any lambda
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("lam", [0.8, -0.35, 1.7, 0.0])
+def test_row_sums_equal_one_minus_lambda(causal, lam):
+    B, N, H, d, dv = 2, 19, 3, 5, 7
+    q, k, v = rand(B, N, H, 2 * d, seed=1), rand(B, N, H, 2 * d, seed=2), rand(B, N, H, dv, seed=3)
+    lams = [lam, lam * 0.5 - 0.1, lam + 0.3]
+    _, w = O.v1_rows(q, k, v, lams, all_rows_v1(B, N, H), causal=causal,
+                     return_weights=True)
+    h = np.arange(B * N * H) % H
+    i = (np.arange(B * N * H) // H) % N
+    expect = 1.0 - np.asarray(lams)[h]
+    assert np.abs(w.sum(axis=1) - expect).max() < 1e-12
+    if causal:  # keys after the query carry no weight
+        for r in range(w.shape[0]):
+            assert np.all(w[r, i[r] + 1:] == 0.0)
+    # some weights are negative whenever lambda > 0 (softmax maps never are)
+    if lam > 0.5:
+        assert (w < 0).any()
+
+
+# --------------------------------------------------------------------------
+# [L] exercise 4: lambda = 0 is plain softmax attention of branch 1
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_lambda_zero_is_softmax_attention(causal):
+    B, N, H, d, dv = 2, 23, 3, 6, 10
+    q, k, v = rand(B, N, H, 2 * d, seed=4), rand(B, N, H, 2 * d, seed=5), rand(B, N, H, dv, seed=6)
+    out = O.v1_rows(q, k, v, [0.0] * H, all_rows_v1(B, N, H), causal=causal)
+    ref = sdpa(q[..., :d], k[..., :d], v, causal)
+    assert np.abs(out - ref.reshape(-1, dv).numpy()).max() < 1e-12
+
+
+# --------------------------------------------------------------------------
+# [G]: each map is ordinary softmax attention -> A1 V - lambda A2 V
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_v1_is_difference_of_two_attentions(causal):
+    B, N, H, d, dv = 2, 29, 4, 8, 16
+    q, k, v = rand(B, N, H, 2 * d, seed=7), rand(B, N, H, 2 * d, seed=8), rand(B, N, H, dv, seed=9)
+    lams = torch.tensor([0.8, -0.2, 1.3, 0.45], dtype=torch.float64)
+    out = O.v1_rows(q, k, v, lams, all_rows_v1(B, N, H), causal=causal)
+    a1 = sdpa(q[..., :d], k[..., :d], v, causal)
+    a2 = sdpa(q[..., d:], k[..., d:], v, causal)
+    ref = a1 - lams.view(1, 1, H, 1) * a2
+    assert np.abs(out - ref.reshape(-1, dv).numpy()).max() < 1e-12
+
+
+def test_identical_branches_scale_softmax_attention():
+    B, N, H, d, dv = 1, 31, 2, 8, 16
+    half_q, half_k = rand(B, N, H, d, seed=10), rand(B, N, H, d, seed=11)
+    q, k = torch.cat([half_q, half_q], -1), torch.cat([half_k, half_k], -1)
+    v = rand(B, N, H, dv, seed=12)
+    lam = [0.8, 0.3]
+    out = O.v1_rows(q, k, v, lam, all_rows_v1(B, N, H), causal=True)
+    ref = sdpa(half_q, half_k, v, True) * (1 - torch.tensor(lam, dtype=torch.float64)).view(1, 1, H, 1)
+    assert np.abs(out - ref.reshape(-1, dv).numpy()).max() < 1e-12
+
+
+def test_causal_first_row_closed_form():
+    B, N, H, d, dv = 2, 9, 2, 4, 8
+    q, k, v = rand(B, N, H, 2 * d, seed=13), rand(B, N, H, 2 * d, seed=14), rand(B, N, H, dv, seed=15)
+    lam = [0.8, -0.6]
+    rows = np.array([(b * N + 0) * H + h for b in range(B) for h in range(H)])
+    out = O.v1_rows(q, k, v, lam, rows, causal=True)
+    for t, r in enumerate(rows):
+        b, h = r // (N * H), r % H
+        assert np.allclose(out[t], (1 - lam[h]) * v[b, 0, h].double().numpy(), rtol=0, atol=1e-15)
+    # with the per-head norm the row becomes RMSNorm((1-lam) V0) (1 - lambda_init)
+    li = O.lambda_init(5)
+    outn = O.v1_rows(q, k, v, lam, rows, causal=True, apply_norm=True, eps=1e-5,
+                     lambda_init_value=li)
+    for t, r in enumerate(rows):
+        b, h = r // (N * H), r % H
+        pre = (1 - lam[h]) * v[b, 0, h].double()
+        ref = F.rms_norm(pre, (dv,), eps=1e-5) * (1 - li)
+        assert np.allclose(outn[t], ref.numpy(), rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# [G] per-head normalisation then (1 - lambda_init): library rms_norm pin
+# --------------------------------------------------------------------------
+def test_head_norm_matches_library_rms_norm():
+    B, N, H, d, dv = 1, 17, 3, 8, 16
+    q, k, v = rand(B, N, H, 2 * d, seed=16), rand(B, N, H, 2 * d, seed=17), rand(B, N, H, dv, seed=18)
+    g = 0.5 + rand(dv, seed=19).abs()
+    lam = [0.7, 0.2, -0.1]
+    li = O.lambda_init(12)
+    rows = all_rows_v1(B, N, H)
+    pre = O.v1_rows(q, k, v, lam, rows, causal=True)
+    post = O.v1_rows(q, k, v, lam, rows, causal=True, apply_norm=True,
+                     norm_weight=g, eps=1e-5, lambda_init_value=li)
+    ref = F.rms_norm(torch.from_numpy(pre), (dv,), weight=g.double(), eps=1e-5) * (1 - li)
+    assert np.abs(post - ref.numpy()).max() < 1e-13
+    # with unit gain every row's RMS is (1 - lambda_init) up to eps
+    post1 = O.v1_rows(q, k, v, lam, rows, causal=True, apply_norm=True, eps=0.0,
+                      lambda_init_value=li)
+    rms = np.sqrt((post1 ** 2).mean(axis=1))
+    assert np.abs(rms - (1 - li)).max() < 1e-13
+
+
+# --------------------------------------------------------------------------
+# lambda_init schedule and lambda re-parameterisation ([G], [L])
+# --------------------------------------------------------------------------
+def test_lambda_init_schedule():
+    assert O.lambda_init(1) == pytest.approx(0.2, abs=1e-15)   # exp(0) = 1
+    assert math.isnan(O.lambda_init(0))
+    vals = [O.lambda_init(l) for l in range(1, 40)]
+    assert all(b > a for a, b in zip(vals, vals[1:]))          # deeper -> closer to 0.8
+    assert O.lambda_init(2000) == pytest.approx(0.8, abs=1e-15)
+    # the gap to 0.8 shrinks by the same factor exp(-0.3) every layer
+    ratios = [(0.8 - b) / (0.8 - a) for a, b in zip(vals, vals[1:])]
+    assert max(ratios) - min(ratios) < 1e-9
+    assert ratios[0] == pytest.approx(math.exp(-0.3), rel=1e-12)
+
+
+def test_lambda_from_params_special_cases():
+    H, dim = 3, 4
+    z = np.zeros((H, dim), np.float32)
+    for layer in (1, 12, 24):
+        assert np.allclose(O.lambda_from_params(z, z, z, z, layer),
+                           O.lambda_init(layer), rtol=0, atol=1e-15)
+    # head 1: lq1 . lk1 = 1 exactly, the second dot 0 -> e - 1 + lambda_init
+    # head 2: the second dot is 2 -> 1 - e^2 + lambda_init (negative lambda)
+    lq1, lk1, lq2, lk2 = (np.zeros((H, dim), np.float32) for _ in range(4))
+    lq1[1, :2] = [0.5, 0.25]
+    lk1[1, :2] = [1.0, 2.0]
+    lq2[2, 3] = 4.0
+    lk2[2, 3] = 0.5
+    lam = O.lambda_from_params(lq1, lk1, lq2, lk2, 12)
+    li = O.lambda_init(12)
+    assert lam[0] == pytest.approx(li, abs=1e-15)
+    assert lam[1] == pytest.approx(math.e - 1 + li, abs=1e-14)
+    assert lam[2] == pytest.approx(1 - math.e ** 2 + li, abs=1e-13)
+    assert lam[2] < 0
+
+
+# --------------------------------------------------------------------------
+# V2: paired query heads sharing GQA KV heads ([L] "V1 vs V2", exercise 5)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [True, False])
+def test_v2_is_difference_of_paired_gqa_attentions(causal):
+    B, N, Hq, Hkv, d = 2, 21, 8, 2, 16
+    q, k, v = rand(B, N, Hq, d, seed=20), rand(B, N, Hkv, d, seed=21), rand(B, N, Hkv, d, seed=22)
+    lam = 0.2 + 0.6 * torch.rand(Hq // 2, generator=torch.Generator().manual_seed(23))
+    rows = np.arange(B * N * (Hq // 2))
+    out = O.v2_rows(q, k, v, lam, rows, causal=causal)
+    per_head = sdpa(q, k, v, causal, enable_gqa=True)   # head h reads kv h // (Hq/Hkv)
+    ref = per_head[:, :, 0::2] - lam.double().view(1, 1, -1, 1) * per_head[:, :, 1::2]
+    assert np.abs(out - ref.reshape(-1, d).numpy()).max() < 1e-12
+
+
+def test_v2_equals_v1_relaid_out():
+    """[L] step 2: V1 and V2 share the maths, only the bookkeeping differs."""
+    B, N, Hq, Hkv, d = 1, 13, 4, 1, 8
+    q, k, v = rand(B, N, Hq, d, seed=24), rand(B, N, Hkv, d, seed=25), rand(B, N, Hkv, d, seed=26)
+    lam = [0.8, 0.25]
+    out2 = O.v2_rows(q, k, v, lam, np.arange(B * N * 2), causal=True)
+    # as V1: head p has Q = [q_{2p} | q_{2p+1}], K = [k_g | k_g], V = v_g
+    q1 = torch.stack([torch.cat([q[:, :, 2 * p], q[:, :, 2 * p + 1]], -1) for p in range(2)], 2)
+    k1 = torch.stack([torch.cat([k[:, :, 0], k[:, :, 0]], -1) for _ in range(2)], 2)
+    v1 = torch.stack([v[:, :, 0] for _ in range(2)], 2)
+    out1 = O.v1_rows(q1, k1, v1, lam, np.arange(B * N * 2), causal=True)
+    assert np.abs(out1 - out2).max() < 1e-14
+
+
+def test_v2_gqa_cache_size_matches_baseline():
+    """[L] exercise 5: with 32 query heads and 8 KV heads the V2 cache is the
+    size of a baseline GQA cache (no doubling)."""
+    w = I.WORKLOADS["v2_decode_bf16"]
+    x = I.v2_decode_inputs(2, 8, w.Hq, w.Hkv, w.d, seed=0)
+    assert x["k_cache"].shape == (2, 8, w.Hkv, w.d)
+    assert x["k_cache"].numel() * 2 == 2 * 8 * w.Hkv * w.d * 2
+    assert x["q"].shape[1] == 2 * (w.Hq // 2)
+
+
+# --------------------------------------------------------------------------
+# decode: one query against the first len_b cache entries
+# --------------------------------------------------------------------------
+def test_v2_decode_matches_library_and_prefill_last_row():
+    B, L, Hq, Hkv, d = 3, 40, 8, 2, 16
+    x = I.v2_decode_inputs(B, L, Hq, Hkv, d, seed=27, dtype=torch.float32)
+    lens = [40, 1, 17]
+    rows = np.arange(B * Hq // 2)
+    out = O.v2_decode_rows(x["q"], x["k_cache"], x["v_cache"], x["lam"], rows, lens=lens)
+    for b in range(B):
+        n = lens[b]
+        qq = x["q"][b].reshape(1, 1, Hq, d)
+        kk = x["k_cache"][b, :n].reshape(1, n, Hkv, d)
+        vv = x["v_cache"][b, :n].reshape(1, n, Hkv, d)
+        per_head = sdpa(qq, kk, vv, False, enable_gqa=True)[0, 0]
+        ref = per_head[0::2] - x["lam"].double().view(-1, 1) * per_head[1::2]
+        got = out[b * Hq // 2:(b + 1) * Hq // 2]
+        assert np.abs(got - ref.numpy()).max() < 1e-12
+        # same as the last row of causal prefill over the cached sequence
+        qseq = torch.zeros(1, n, Hq, d)
+        qseq[0, n - 1] = x["q"][b]
+        pre = O.v2_rows(qseq, kk, vv, x["lam"], np.arange((n - 1) * Hq // 2, n * Hq // 2),
+                        causal=True)
+        assert np.abs(pre - got).max() < 1e-14
+
+
+def test_v1_decode_matches_library_with_norm():
+    B, L, H, d, dv = 2, 33, 3, 8, 16
+    x = I.v1_decode_inputs(B, L, H, d, dv, seed=28, dtype=torch.float32)
+    lam = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], 12)
+    li = O.lambda_init(12)
+    lens = [33, 5]
+    out = O.v1_decode_rows(x["q"], x["k_cache"], x["v_cache"], lam, np.arange(B * H),
+                           lens=lens, apply_norm=True, eps=1e-5, lambda_init_value=li)
+    for b in range(B):
+        n = lens[b]
+        qq = x["q"][b].reshape(1, 1, H, 2 * d)
+        kk = x["k_cache"][b, :n].reshape(1, n, H, 2 * d)
+        vv = x["v_cache"][b, :n].reshape(1, n, H, dv)
+        a1 = sdpa(qq[..., :d], kk[..., :d], vv)[0, 0]
+        a2 = sdpa(qq[..., d:], kk[..., d:], vv)[0, 0]
+        pre = a1 - torch.from_numpy(lam).view(H, 1) * a2
+        ref = F.rms_norm(pre, (dv,), eps=1e-5) * (1 - li)
+        assert np.abs(out[b * H:(b + 1) * H] - ref.numpy()).max() < 1e-13
+
+
+# --------------------------------------------------------------------------
+# planted signal of the long-context workload: branch 1 finds the needles
+# --------------------------------------------------------------------------
+def test_planted_signal_is_found_by_branch_one():
+    B, N, H, d, dv = 1, 2048, 2, 64, 128
+    x = I.v1_inputs(B, N, H, d, dv, seed=2, dtype=torch.bfloat16, planted=6)
+    rows = np.array([(N - 2) * H + h for h in range(H)] + [(N - 1) * H + h for h in range(H)])
+    _, w = O.v1_rows(x["q"], x["k"], x["v"], [0.0] * H, rows, causal=True,
+                     return_weights=True)   # lambda = 0: w is branch 1's map
+    for t, r in enumerate(rows):
+        h = r % H
+        pos = x["planted_pos"][0, h].numpy()
+        assert w[t, pos].sum() > 0.8
+
+
+def test_oracle_rejects_out_of_range_rows():
+    q = torch.zeros(1, 4, 1, 4)
+    with pytest.raises(ValueError):
+        O.v1_rows(q, q, torch.zeros(1, 4, 1, 2), [0.5], np.array([4]), causal=True)
+
+
+def test_large_logits_stay_finite_and_exact():
+    """[L] step 1 subtracts the row maximum before exponentiating, so logits
+    in the hundreds (far beyond exp's float64 range once summed) still give
+    the library's softmax attention."""
+    B, N, H, d, dv = 1, 11, 2, 8, 8
+    q = 60.0 * rand(B, N, H, 2 * d, seed=40)
+    k = 60.0 * rand(B, N, H, 2 * d, seed=41)
+    v = rand(B, N, H, dv, seed=42)
+    lam = [0.8, -0.4]
+    out = O.v1_rows(q, k, v, lam, all_rows_v1(B, N, H), causal=False)
+    assert np.isfinite(out).all()
+    a1 = sdpa(q[..., :d], k[..., :d], v)
+    a2 = sdpa(q[..., d:], k[..., d:], v)
+    ref = a1 - torch.tensor(lam, dtype=torch.float64).view(1, 1, H, 1) * a2
+    assert np.abs(out - ref.reshape(-1, dv).numpy()).max() < 1e-9
