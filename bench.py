@@ -1,0 +1,526 @@
+#!/usr/bin/env python
+"""Benchmark of the differential-attention hot path on B200.
+
+One step = one pass of the hot path over one batch: lambda from its four
+per-head vectors, then V1 causal prefill with the per-head RMS norm and the
+(1 - lambda_init) scale (batch 4, 16 heads, 4096 tokens, 64-wide branches,
+128-wide values, layer 12).  Metric: DiffAttn forward TFLOP/s, counting
+2 QK^T + 2 PV contractions per visible (query, key) pair (768 flop per pair
+for this shape, masked pairs excluded).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; each rank
+runs the same per-GPU workload (weak scaling, no collective on the data
+path), timing is taken as the max over ranks, and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DiffAttn fwd TFLOP/s (prefill), decode HBM GB/s; % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+def prefill_pairs(B, N, H, causal=True):
+    """Visible (query, key) pairs of one prefill call."""
+    return B * H * (N * (N + 1) // 2 if causal else N * N)
+
+
+def v1_flops_per_pair(d, dv):
+    return 2 * (2 * d) + 2 * (2 * dv)          # two QK^T branches + two P.V
+
+
+def v2_flops_per_pair(d):
+    return 2 * (2 * d) + 2 * (2 * d)
+
+
+def v2_decode_bytes(B, L, Hkv, d, Hq):
+    return B * L * Hkv * d * 2 * 2 + B * Hq * d * 2 + B * (Hq // 2) * d * 2
+
+
+def v1_decode_bytes(B, L, H, d, dv):
+    return B * L * H * (2 * d + dv) * 2 + B * H * 2 * d * 2 + B * H * dv * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured (MEASURED_PEAKS.json)"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("prefill_tc.cu", "ptx.cuh"):
+        with open(os.path.join(ROOT, "differential_attention_sm_b200", "csrc", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, valid only while
+    the kernel source is unchanged since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = kernel_source_hash()
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[3] == cur:
+            return float(parts[2])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read only)
+# ---------------------------------------------------------------------------
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            self.h = None
+            if uuid:
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    u = pynvml.nvmlDeviceGetUUID(hh)
+                    u = u.decode() if isinstance(u, bytes) else u
+                    if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                        self.h = hh
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.period = period_s
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in _REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU)
+# ---------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def timed_loop(fn, steps, warmup, world, stream):
+    """W untimed steps, then exactly K steps bracketed by barrier+sync;
+    returns (device ms for the K steps, max over ranks)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    return max_over_ranks(ms, world, torch.device("cuda"))
+
+
+def run_headline(args, rank, world, local_rank, peaks, peak_src):
+    import torch
+    from differential_attention_sm_b200 import binding as Bd
+    from differential_attention_sm_b200 import inputs as I
+
+    w = I.WORKLOADS["v1_prefill_bf16"]
+    dev = torch.device("cuda", local_rank)
+    x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed + 1000 * rank)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    lv = [x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")]
+    lam = torch.empty(w.H, dtype=torch.float32, device=dev)
+    out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    li = Bd.diffattn_lambda_init(w.layer)
+    stream = torch.cuda.current_stream(dev)
+    flops = prefill_pairs(w.B, w.N, w.H) * v1_flops_per_pair(w.d, w.dv)
+
+    def step():
+        Bd.lambda_from_params(*lv, w.layer, out=lam)
+        Bd.diffattn_v1_fwd(q, k, v, lam, causal=True, apply_norm=True, norm_eps=w.eps,
+                           lambda_init=li, out=out, dev_status=status)
+
+    with ClockSampler(local_rank) as clk:
+        ms = timed_loop(step, args.steps, args.warmup, world, stream)
+    # the dominant kernel alone, timed with events on its own stream
+    kms = []
+    for _ in range(max(5, min(args.steps, 50))):
+        Bd.lambda_from_params(*lv, w.layer, out=lam)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Bd.diffattn_v1_fwd(q, k, v, lam, causal=True, apply_norm=True, norm_eps=w.eps,
+                           lambda_init=li, out=out, dev_status=status)
+        b.record(stream)
+        kms.append((a, b))
+    torch.cuda.synchronize()
+    kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in kms]))
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d during the benchmark" % int(status.item()))
+
+    # end to end through the public API with pinned host buffers
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    hl = [x[n].pin_memory() for n in ("lq1", "lk1", "lq2", "lk2")]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dl = [torch.empty_like(t) for t in lv]
+
+    def e2e_step():
+        for d_, h_ in zip((dq, dk, dv_, *dl), (hq, hk, hv, *hl)):
+            d_.copy_(h_, non_blocking=True)
+        Bd.lambda_from_params(*dl, w.layer, out=lam)
+        Bd.diffattn_v1_fwd(dq, dk, dv_, lam, causal=True, apply_norm=True, norm_eps=w.eps,
+                           lambda_init=li, out=out, dev_status=status)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = timed_loop(e2e_step, e2e_steps, max(3, min(args.warmup, 5)), world, stream)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, *hl))
+    d2h = hout.numel() * hout.element_size()
+
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    traffic = recorded_traffic("diffattn_prefill_tc_kernel", "v1_prefill_bf16")
+    res = {
+        "value": world * flops * args.steps / (ms * 1e-3) / 1e12,
+        "ms_per_step": ms / args.steps,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "diffattn_prefill_tc_kernel", "kernel_ms": round(kernel_ms, 4),
+                     "peak_source": "%s dense bf16 burst" % peak_src,
+                     "work_per_launch": "%.4e flop (768 flop x %d causal pairs)" % (
+                         flops, prefill_pairs(w.B, w.N, w.H))},
+        "e2e": {"value": world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "config": {"workload": "v1_prefill_bf16: V1 causal prefill, batch 4, 16 heads, "
+                               "seq 4096, QK 64 per branch, V 128, lambda from params "
+                               "(layer 12), per-head RMSNorm eps 1e-5, x(1-lambda_init)",
+                   "batch_per_gpu": w.B, "global_batch": w.B * world, "seq_len": w.N,
+                   "heads": w.H, "d_qk": w.d, "d_v": w.dv, "causal": True,
+                   "parallelism": "dp%d (independent batches)" % world,
+                   "l2": "inputs 192 MiB per step > 126 MB L2 (no flush needed)"},
+    }
+    del q, k, v, out, dq, dk, dv_
+    torch.cuda.empty_cache()
+    return res, x
+
+
+def time_call(fn, iters, warmup, stream):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def run_extras(local_rank, peaks, peak_src):
+    """The other workloads, one GPU: V1 long-context prefill, V2 prefill,
+    V2 decode and V1 decode (same kernels the parity tests check)."""
+    import torch
+    from differential_attention_sm_b200 import binding as Bd
+    from differential_attention_sm_b200 import inputs as I
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+
+    # V2 causal prefill: B2 Hq32 Hkv8 d128 N8192
+    w = I.WORKLOADS["v2_prefill_bf16"]
+    x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
+    q, k, v, lam = (x[n].to(dev) for n in ("q", "k", "v", "lam"))
+    o = torch.empty(w.B, w.N, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
+    ms = time_call(lambda: Bd.diffattn_v2_prefill(q, k, v, lam, causal=True, out=o), 20, 3, stream)
+    fl = prefill_pairs(w.B, w.N, w.Hq // 2) * v2_flops_per_pair(w.d)
+    t = fl / (ms * 1e-3) / 1e12
+    out["v2_prefill_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
+                              "frac": round(t / peaks["bf16_tflops"], 4),
+                              "peak": peaks["bf16_tflops"], "flop": fl}
+    del q, k, v, o, x
+
+    # V1 long-context prefill: B1 H16 N32768 layer 24, planted signal
+    w = I.WORKLOADS["v1_long_bf16"]
+    x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed, planted=w.planted)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    lv = [x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")]
+    lamt = Bd.lambda_from_params(*lv, w.layer)
+    li = Bd.diffattn_lambda_init(w.layer)
+    o = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+    ms = time_call(lambda: Bd.diffattn_v1_fwd(q, k, v, lamt, causal=True, apply_norm=True,
+                                              lambda_init=li, out=o), 5, 2, stream)
+    fl = prefill_pairs(w.B, w.N, w.H) * v1_flops_per_pair(w.d, w.dv)
+    t = fl / (ms * 1e-3) / 1e12
+    out["v1_long_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
+                           "frac": round(t / peaks["bf16_tflops"], 4), "flop": fl}
+    del q, k, v, o, x
+
+    # V2 decode: B64 L32768 Hq64 Hkv8 d128
+    w = I.WORKLOADS["v2_decode_bf16"]
+    x = I.v2_decode_inputs(w.B, w.L, w.Hq, w.Hkv, w.d, w.seed, fill_caches=False)
+    kc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.Hkv, w.d, dtype=torch.bfloat16,
+                                             device=dev), 1)
+    vc = I.fill_normal_on_device(torch.empty_like(kc), 2)
+    q, lam = x["q"].to(dev), x["lam"].to(dev)
+    ws = torch.empty(Bd.diffattn_v2_decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.L),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(w.B, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
+    ms = time_call(lambda: Bd.diffattn_v2_decode(q, kc, vc, lam, workspace=ws, out=o), 20, 3,
+                   stream)
+    by = v2_decode_bytes(w.B, w.L, w.Hkv, w.d, w.Hq)
+    gbs = by / (ms * 1e-3) / 1e9
+    out["v2_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
+                             "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
+                             "bytes": by}
+    del kc, vc, ws
+    torch.cuda.empty_cache()
+
+    # V1 decode (comparison): B64 L32768 H32 d64 dv128
+    w = I.WORKLOADS["v1_decode_bf16"]
+    x = I.v1_decode_inputs(w.B, w.L, w.H, w.d, w.dv, w.seed, fill_caches=False)
+    kc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.H, 2 * w.d, dtype=torch.bfloat16,
+                                             device=dev), 3)
+    vc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.H, w.dv, dtype=torch.bfloat16,
+                                             device=dev), 4)
+    q = x["q"].to(dev)
+    lamt = Bd.lambda_from_params(*(x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")), w.layer)
+    li = Bd.diffattn_lambda_init(w.layer)
+    ws = torch.empty(Bd.diffattn_v1_decode_workspace_size(w.B, w.H, w.d, w.dv, w.L),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+    ms = time_call(lambda: Bd.diffattn_v1_decode(q, kc, vc, lamt, apply_norm=True,
+                                                 lambda_init=li, workspace=ws, out=o), 5, 2,
+                   stream)
+    by = v1_decode_bytes(w.B, w.L, w.H, w.d, w.dv)
+    gbs = by / (ms * 1e-3) / 1e9
+    out["v1_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
+                             "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": by}
+    del kc, vc, ws
+    torch.cuda.empty_cache()
+    out["peak_source"] = peak_src
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline / reference arm: the fp64 oracle on host cores
+# ---------------------------------------------------------------------------
+def oracle_sample(x, w, target_s: float, seed: int):
+    """Runs the oracle on random rows of the workload until about target_s
+    seconds of work; returns (algorithmic flop done, seconds, rows)."""
+    import oracle as O
+    lam = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+    li = O.lambda_init(w.layer)
+    rng = np.random.default_rng(seed)
+    fpp = v1_flops_per_pair(w.d, w.dv)
+    total_rows = w.B * w.N * w.H
+    n, done_fl, done_s, rows_done = 32, 0.0, 0.0, 0
+    while done_s < target_s:
+        rows = rng.integers(0, total_rows, n)
+        i = (rows // w.H) % w.N
+        t0 = time.perf_counter()
+        O.v1_rows(x["q"], x["k"], x["v"], lam, rows, causal=True, apply_norm=True,
+                  eps=w.eps, lambda_init_value=li)
+        dt = time.perf_counter() - t0
+        done_fl += float(((i + 1) * fpp).sum())
+        done_s += dt
+        rows_done += n
+        if dt < target_s / 4:
+            n *= 2
+    return done_fl, done_s, rows_done
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle as O
+    from differential_attention_sm_b200 import inputs as I
+    O.build()
+    w = I.WORKLOADS["v1_prefill_bf16"]
+    x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed)
+    for s in range(args.warmup):
+        oracle_sample(x, w, 0.5, seed=s)
+    fl, secs, rows = 0.0, 0.0, 0
+    for s in range(args.steps):
+        f, t, r = oracle_sample(x, w, 2.0, seed=1000 + s)
+        fl += f
+        secs += t
+        rows += r
+    val = fl / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "v1_prefill_bf16: V1 causal prefill, batch 4, 16 heads, seq 4096, "
+                               "QK 64 per branch, V 128, layer 12, RMSNorm",
+                   "note": "reference arm = the fp64 CPU oracle; each step is a bounded random "
+                           "sample of output rows (about 2 s of host work)"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": O.n_threads(),
+                         "kind": "oracle",
+                         "sample": "%d random output rows of the workload over %d steps" % (
+                             rows, args.steps)},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the secondary workloads (V2 prefill, long V1, decode)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="bounded host time for the oracle CPU baseline")
+    args = ap.parse_args()
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from differential_attention_sm_b200 import binding as Bd
+    Bd.load()
+    peaks, peak_src = load_peaks()
+    res, x = run_headline(args, rank, world, local_rank, peaks, peak_src)
+    extras = None
+    if world == 1 and not args.no_extras:
+        extras = run_extras(local_rank, peaks, peak_src)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    import oracle as O
+    from differential_attention_sm_b200 import inputs as I
+    cpu = None
+    if world == 1:
+        O.build()
+        w = I.WORKLOADS["v1_prefill_bf16"]
+        fl, secs, rows = oracle_sample(x, w, args.cpu_seconds, seed=7)
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": O.n_threads(),
+               "kind": "oracle",
+               "sample": "%d random output rows of the V1 prefill workload (%.1f s)" % (
+                   rows, secs)}
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), bf16-rounded)", "config": res["config"],
+        "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
+        "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+    }
+    if extras is not None:
+        line["also"] = extras
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

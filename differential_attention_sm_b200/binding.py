@@ -1,0 +1,225 @@
+"""Thin ctypes binding over libdiffattn.so (``include/diffattn.h``).
+
+Every function here has the name of the C entry point it wraps and only
+marshals arguments: torch tensors (device memory allocated by PyTorch) are
+passed as raw pointers together with their sizes, on the current CUDA
+stream.  All arithmetic happens in the library's CUDA kernels.  There is no
+fallback: if the library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdiffattn.so")
+
+DA_OK = 0
+DA_ERR_INVALID_ARG = -1
+DA_ERR_UNSUPPORTED = -2
+DA_ERR_ALIGNMENT = -3
+DA_ERR_WORKSPACE = -4
+DA_ERR_CUDA = -5
+DA_ERR_DEVICE_TIMEOUT = -6
+DA_BF16 = 0
+DA_FP32 = 1
+
+# Every symbol include/diffattn.h declares.
+EXPORTS = (
+    "diffattn_status_string",
+    "diffattn_lambda_init",
+    "lambda_from_params",
+    "diffattn_v1_fwd",
+    "diffattn_v2_prefill",
+    "diffattn_v2_decode_workspace_size",
+    "diffattn_v2_decode",
+    "diffattn_v1_decode_workspace_size",
+    "diffattn_v1_decode",
+)
+
+
+class DiffAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (fn, status_string(status), status))
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the library (once).  Raises if it is missing: there is no
+    CPU or library fallback for the operator."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError("libdiffattn.so not built (run __graft_entry__.build() or "
+                          "python -m differential_attention_sm_b200.build)")
+    lib = ctypes.CDLL(p)
+    lib.diffattn_status_string.restype = ctypes.c_char_p
+    lib.diffattn_status_string.argtypes = [_i]
+    lib.diffattn_lambda_init.restype = ctypes.c_double
+    lib.diffattn_lambda_init.argtypes = [_i]
+    lib.lambda_from_params.restype = _i
+    lib.lambda_from_params.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]
+    lib.diffattn_v1_fwd.restype = _i
+    lib.diffattn_v1_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i,
+                                    _vp, _f, _f, _vp, _vp]
+    lib.diffattn_v2_prefill.restype = _i
+    lib.diffattn_v2_prefill.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i,
+                                        _vp, _vp]
+    lib.diffattn_v2_decode_workspace_size.restype = _sz
+    lib.diffattn_v2_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+    lib.diffattn_v2_decode.restype = _i
+    lib.diffattn_v2_decode.argtypes = [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp,
+                                       _vp, _sz, _vp, _vp]
+    lib.diffattn_v1_decode_workspace_size.restype = _sz
+    lib.diffattn_v1_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+    lib.diffattn_v1_decode.restype = _i
+    lib.diffattn_v1_decode.argtypes = [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp,
+                                       _i, _vp, _f, _f, _vp, _sz, _vp, _vp]
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().diffattn_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DA_BF16
+    if t.dtype == torch.float32:
+        return DA_FP32
+    raise TypeError("unsupported dtype %s" % t.dtype)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != DA_OK:
+        raise DiffAttnError(fn, status)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not isinstance(t, int):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def diffattn_lambda_init(layer: int) -> float:
+    return float(load().diffattn_lambda_init(int(layer)))
+
+
+def lambda_from_params(lq1, lk1, lq2, lk2, layer: int, out=None, stream=None):
+    """lambda [H] (fp32, device) from four [H, dim] fp32 device vectors."""
+    _need_cuda(lq1, lk1, lq2, lk2)
+    H, dim = lq1.shape
+    if out is None:
+        out = torch.empty(H, dtype=torch.float32, device=lq1.device)
+    _check("lambda_from_params", load().lambda_from_params(
+        _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), H, dim, int(layer), _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def diffattn_v1_fwd(q, k, v, lam, *, causal=True, apply_norm=False, norm_weight=None,
+                    norm_eps=1e-5, lambda_init=0.0, out=None, dev_status=None, stream=None):
+    """V1 prefill.  q, k [B, N, H, 2d]; v [B, N, H, dv]; lam [H] fp32."""
+    _need_cuda(q, k, v, lam, norm_weight, dev_status)
+    B, N, H, d2 = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty(B, N, H, dv, dtype=q.dtype, device=q.device)
+    _check("diffattn_v1_fwd", load().diffattn_v1_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, N, H, d2 // 2, dv,
+        _ptr(lam), int(bool(causal)), int(bool(apply_norm)), _ptr(norm_weight),
+        float(norm_eps), float(lambda_init), _ptr(dev_status), _stream(stream)))
+    return out
+
+
+def diffattn_v2_prefill(q, k, v, lam, *, causal=True, out=None, dev_status=None, stream=None):
+    """V2 prefill.  q [B, N, Hq, d]; k, v [B, N, Hkv, d]; lam [Hq/2] fp32."""
+    _need_cuda(q, k, v, lam, dev_status)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty(B, N, Hq // 2, d, dtype=q.dtype, device=q.device)
+    _check("diffattn_v2_prefill", load().diffattn_v2_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, N, Hq, Hkv, d, _ptr(lam),
+        int(bool(causal)), _ptr(dev_status), _stream(stream)))
+    return out
+
+
+def diffattn_v2_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, max_len) -> int:
+    return int(load().diffattn_v2_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim,
+                                                        max_len))
+
+
+def diffattn_v2_decode(q, k_cache, v_cache, lam, *, cache_lens=None, workspace=None, out=None,
+                       dev_status=None, stream=None):
+    """V2 decode.  q [B, Hq, d]; caches [B, L, Hkv, d]; lam [Hq/2] fp32;
+    cache_lens int32 [B] or None; workspace a uint8 device tensor or None
+    (allocated here from the size query)."""
+    _need_cuda(q, k_cache, v_cache, lam, cache_lens, dev_status)
+    B, Hq, d = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    ws_need = diffattn_v2_decode_workspace_size(B, Hq, Hkv, d, L)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if out is None:
+        out = torch.empty(B, Hq // 2, d, dtype=q.dtype, device=q.device)
+    _check("diffattn_v2_decode", load().diffattn_v2_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), L, _ptr(out), _dtype_code(q),
+        B, Hq, Hkv, d, _ptr(lam), _ptr(workspace), ws_bytes, _ptr(dev_status),
+        _stream(stream)))
+    return out
+
+
+def diffattn_v1_decode_workspace_size(batch, n_heads, d_qk, d_v, max_len) -> int:
+    return int(load().diffattn_v1_decode_workspace_size(batch, n_heads, d_qk, d_v, max_len))
+
+
+def diffattn_v1_decode(q, k_cache, v_cache, lam, *, cache_lens=None, apply_norm=False,
+                       norm_weight=None, norm_eps=1e-5, lambda_init=0.0, workspace=None,
+                       out=None, dev_status=None, stream=None):
+    """V1 decode.  q [B, H, 2d]; k_cache [B, L, H, 2d]; v_cache [B, L, H, dv]."""
+    _need_cuda(q, k_cache, v_cache, lam, cache_lens, norm_weight, dev_status)
+    B, H, d2 = q.shape
+    L, dv = k_cache.shape[1], v_cache.shape[-1]
+    ws_need = diffattn_v1_decode_workspace_size(B, H, d2 // 2, dv, L)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if out is None:
+        out = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    _check("diffattn_v1_decode", load().diffattn_v1_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), L, _ptr(out), _dtype_code(q),
+        B, H, d2 // 2, dv, _ptr(lam), int(bool(apply_norm)), _ptr(norm_weight),
+        float(norm_eps), float(lambda_init), _ptr(workspace), ws_bytes, _ptr(dev_status),
+        _stream(stream)))
+    return out

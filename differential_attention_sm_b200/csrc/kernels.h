@@ -1,0 +1,92 @@
+// kernels.h — internal launch interfaces between the C-ABI layer (api.cu)
+// and the kernels.  Not installed; the public interface is diffattn.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace da {
+
+// Addressing of the generic (CUDA-core) kernel; all strides in elements.
+struct GenericProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  int batch, n_q, heads;  // output rows = batch * n_q * heads
+  int d, dv;
+  int64_t q_batch, q_tok;
+  int64_t k_batch, k_tok;
+  int k_head_stride, k2_off;
+  int64_t v_batch, v_tok;
+  int v_head_stride;
+  int kv_div;  // key/value head = output head / kv_div
+  int64_t o_batch, o_tok;
+  int n_keys;       // keys per sequence (prefill N, decode max_len)
+  int causal;       // prefill: query i sees keys <= i
+  const int* lens;  // decode: per-batch valid cache rows, or nullptr
+  const float* lambda;
+  int apply_norm;
+  const float* norm_weight;
+  float eps, post_scale;
+};
+
+cudaError_t launch_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                          int n_heads, int dim, float lambda_init, float* out,
+                          cudaStream_t stream);
+
+cudaError_t launch_generic(const GenericProblem& P, bool bf16, cudaStream_t stream);
+
+// ---- V2 split-KV decode (bf16, head_dim 128, group <= 8) ------------------
+struct V2DecodePlan {
+  int n_split;    // splits per (batch, kv head)
+  int split_len;  // tokens per split (multiple of 64)
+  int n_items;    // batch * n_kv_heads * n_split
+  int grid;       // persistent CTAs
+};
+V2DecodePlan plan_v2_decode(int batch, int n_kv_heads, int max_len, int num_sms);
+size_t v2_decode_workspace_bytes(const V2DecodePlan& plan);
+cudaError_t launch_v2_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
+                             const int* lens, int max_len, void* out, int batch, int n_q_heads,
+                             int n_kv_heads, const float* lambda, const V2DecodePlan& plan,
+                             void* workspace, int* dev_status, cudaStream_t stream);
+
+// ---- V1 split-KV decode (bf16, d_qk 64, d_v 128) --------------------------
+struct V1DecodePlan {
+  int n_split, split_len, n_items;
+};
+V1DecodePlan plan_v1_decode(int batch, int n_heads, int max_len, int num_sms);
+size_t v1_decode_workspace_bytes(const V1DecodePlan& plan);
+cudaError_t launch_v1_decode(const void* q, const void* k_cache, const void* v_cache,
+                             const int* lens, int max_len, void* out, int batch, int n_heads,
+                             const float* lambda, int apply_norm, const float* norm_weight,
+                             float eps, float post_scale, const V1DecodePlan& plan,
+                             void* workspace, cudaStream_t stream);
+
+// ---- tcgen05 prefill (bf16) -----------------------------------------------
+// Form 1 (V1): Q/K rows are 128 wide (two 64-wide branches), V 128 wide,
+//              one KV head per head, optional RMS norm.
+// Form 2 (V2): query heads 2p, 2p+1 (128 wide each) against KV head
+//              2p / group, no norm.
+struct PrefillArgs {
+  int form;  // 1 or 2
+  int batch, seqlen;
+  int heads;     // V1: heads; V2: pairs (n_q_heads / 2)
+  int kv_heads;  // V1: heads; V2: n_kv_heads
+  int pairs_per_kv;  // V2: group / 2; V1: 1
+  int causal;
+  const float* lambda;
+  int apply_norm;
+  const float* norm_weight;
+  float eps, post_scale;
+  void* out;
+  int* dev_status;
+};
+cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                              const CUtensorMap& tm_v, const PrefillArgs& a, int num_sms,
+                              cudaStream_t stream);
+
+}  // namespace da

@@ -1,0 +1,395 @@
+// prefill_tc.cu — differential-attention prefill on the 5th-generation
+// tensor cores (tcgen05 + tensor memory + TMA), both forms.
+//
+// Operator: glossary page "Differential Transformer", section "Cómo funciona
+// la atención diferencial" (two softmax maps from the two halves of each
+// head's query/key, combined as (map1 - lambda map2) V, then a per-head
+// normalisation and a (1 - lambda_init) scale); lesson "Atención
+// Diferencial (V2)", section "V1 vs V2: la diferencia" (V2: paired query
+// heads on shared GQA KV heads, full head width, no per-head norm).
+//
+// One CTA computes 128 query rows of one head (V1) or one head pair (V2).
+// Both branches see the same K and V tiles, so each 128-key tile is loaded
+// once by TMA for the pair.  Tensor memory (512 columns x 128 lanes fp32):
+//     S1 [0,128)   S2 [128,256)   O1 [256,384)   O2 [384,512)
+// P_r (bf16, 64 columns) overwrites the first half of S_r in place and
+// feeds the P.V MMA directly from tensor memory.  The two branches need
+// separate O accumulators because their running maxima and normalisers
+// differ; the subtraction happens in the epilogue:
+//     o = O1 / l1 - lambda * O2 / l2   (then, V1 only, RMS norm * g * (1 - lambda_init)).
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for branch 1 (thread = one query row = one TMEM lane)
+//   warps 4-7  softmax for branch 2
+//   warp  8    TMA producer (Q once; K and V tiles through 2-stage rings)
+//   warp  9    tcgen05.mma issuer; owns the tensor-memory allocation
+// Softmax keeps a per-row reference maximum and only rescales O (in tensor
+// memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
+// Causal masking is applied only on the diagonal tile (and the ragged tail).
+// Every wait is bounded; a timed-out wait records DA_ERR_DEVICE_TIMEOUT in
+// the caller's status word and the CTA unwinds, still freeing its TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace da {
+namespace {
+
+constexpr int kBM = 128;                 // query rows per CTA
+constexpr int kBN = 128;                 // keys per KV tile
+constexpr int kThreads = 320;
+constexpr int kBox = 128 * 64 * 2;       // one TMA box: 128 rows x 64 bf16 = 16 KB
+constexpr int kTileBytes = 2 * kBox;     // a 128 x 128 bf16 tile (two swizzle-atom columns)
+constexpr int kStages = 2;
+constexpr uint32_t kColS1 = 0, kColS2 = 128, kColO1 = 256, kColO2 = 384;
+constexpr float kLazyTau = 8.0f;         // log2 units: rescale only when max grows by > 2^8
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
+
+struct Barriers {
+  uint64_t q_full;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Params {
+  int form;
+  int batch, seqlen, heads, pairs_per_kv;
+  int n_qtiles;
+  int causal;
+  float scale_log2;
+  const float* lambda;
+  int apply_norm;
+  const float* norm_weight;
+  float eps, post_scale;
+  __nv_bfloat16* out;
+  int* dev_status;
+};
+
+__device__ __forceinline__ uint32_t q_bytes(int form) { return form == 1 ? kTileBytes : 2 * kTileBytes; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t qb = q_bytes(p.form);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + qb;                            // kStages x kTileBytes
+  uint8_t* sV = sK + kStages * kTileBytes;            // kStages x kTileBytes
+  Barriers* bars = reinterpret_cast<Barriers*>(sV + kStages * kTileBytes);
+  float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [2][128]
+  float* x_ss = x_inv_l + 2 * kBM;                       // [2][128]
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+
+  // ---- tile coordinates: heaviest (latest) query tiles first ----
+  const int bh_count = p.batch * p.heads;
+  const int mt = p.n_qtiles - 1 - (int)(blockIdx.x / bh_count);
+  const int bh = (int)(blockIdx.x % bh_count);
+  const int hh = bh % p.heads;          // V1 head or V2 pair
+  const int b = bh / p.heads;
+  const int kvh = p.form == 1 ? hh : hh / p.pairs_per_kv;
+  const int q0 = mt * kBM;
+  const int n_kv = p.causal ? mt + 1 : (p.seqlen + kBN - 1) / kBN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&bars->s_full[r], 1);
+      mbar_init(&bars->p_full[r], 128);
+      mbar_init(&bars->o_done[r], 1);
+    }
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  bool failed = false;
+
+  if (warp == 8) {
+    // ------------------------------ TMA producer ---------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&bars->q_full, qb);
+      if (p.form == 1) {
+        tma_load_4d(sQ, &tm_q, &bars->q_full, 0, hh, q0, b);
+        tma_load_4d(sQ + kBox, &tm_q, &bars->q_full, 64, hh, q0, b);
+      } else {
+        tma_load_4d(sQ, &tm_q, &bars->q_full, 0, 2 * hh, q0, b);
+        tma_load_4d(sQ + kBox, &tm_q, &bars->q_full, 64, 2 * hh, q0, b);
+        tma_load_4d(sQ + 2 * kBox, &tm_q, &bars->q_full, 0, 2 * hh + 1, q0, b);
+        tma_load_4d(sQ + 3 * kBox, &tm_q, &bars->q_full, 64, 2 * hh + 1, q0, b);
+      }
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kStages;
+        const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+        if (!mbar_wait(&bars->k_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
+        mbar_arrive_expect_tx(&bars->k_full[s], kTileBytes);
+        tma_load_4d(sK + s * kTileBytes, &tm_k, &bars->k_full[s], 0, kvh, j * kBN, b);
+        tma_load_4d(sK + s * kTileBytes + kBox, &tm_k, &bars->k_full[s], 64, kvh, j * kBN, b);
+        if (!mbar_wait(&bars->v_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
+        mbar_arrive_expect_tx(&bars->v_full[s], kTileBytes);
+        tma_load_4d(sV + s * kTileBytes, &tm_v, &bars->v_full[s], 0, kvh, j * kBN, b);
+        tma_load_4d(sV + s * kTileBytes + kBox, &tm_v, &bars->v_full[s], 64, kvh, j * kBN, b);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------ MMA issuer -----------------------------
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t k_addr = smem_u32(sK);
+      const uint32_t v_addr = smem_u32(sV);
+      const int nk = p.form == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T per branch
+      if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
+        for (int j = 0; j < n_kv; ++j) {
+          const int s = j % kStages;
+          const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+          if (!mbar_wait(&bars->k_full[s], ph, p.dev_status, &failed)) break;
+          const uint32_t kt = k_addr + s * kTileBytes;
+          for (int r = 0; r < 2; ++r) {
+            // S_r aliases P_r of the previous tile: wait until P_r(j-1).V is done
+            if (j > 0 && !mbar_wait(&bars->o_done[r], (uint32_t)(j - 1) & 1u, p.dev_status,
+                                    &failed))
+              break;
+            tc_fence_after();
+            for (int kk = 0; kk < nk; ++kk) {
+              uint32_t a, bb;
+              if (p.form == 1) {  // branch r = columns [64 r, 64 r + 64)
+                a = q_addr + r * kBox + kk * 32;
+                bb = kt + r * kBox + kk * 32;
+              } else {            // branch r = query head 2p + r, full 128 columns
+                a = q_addr + r * kTileBytes + (kk >> 2) * kBox + (kk & 3) * 32;
+                bb = kt + (kk >> 2) * kBox + (kk & 3) * 32;
+              }
+              tc_mma_ss(tmem + (r == 0 ? kColS1 : kColS2), smem_desc_sw128(a, 16, 1024),
+                        smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars->s_full[r]);
+          }
+          if (failed) break;
+          tc_commit(&bars->k_empty[s]);
+          if (!mbar_wait(&bars->v_full[s], ph, p.dev_status, &failed)) break;
+          const uint32_t vt = v_addr + s * kTileBytes;
+          for (int r = 0; r < 2; ++r) {
+            if (!mbar_wait(&bars->p_full[r], (uint32_t)j & 1u, p.dev_status, &failed)) break;
+            tc_fence_after();
+            const uint32_t pcol = tmem + (r == 0 ? kColS1 : kColS2);
+            const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              // B = V tile, MN-major: 64-column halves kBox apart, 8-key groups 1 KB apart
+              tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kBox, 1024),
+                        kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&bars->o_done[r]);
+          }
+          if (failed) break;
+          tc_commit(&bars->v_empty[s]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------ softmax warpgroups ---------------------
+    const int r = warp / 4;                  // branch
+    const int sub = warp & 3;                // TMEM lane quarter
+    const int row = sub * 32 + lane;         // query row within the tile
+    const int qrow = q0 + row;               // query row within the sequence
+    const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + (r == 0 ? kColS1 : kColS2);
+    const uint32_t t_o = tmem + lane_off + (r == 0 ? kColO1 : kColO2);
+    float m_ref = -INFINITY, l_run = 0.f;
+
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait(&bars->s_full[r], (uint32_t)j & 1u, p.dev_status, &failed)) break;
+      tc_fence_after();
+      uint32_t sr[128];  // raw S row (masked entries set to -inf)
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(t_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
+      tc_wait_ld();
+      const int k0 = j * kBN;
+      const bool need_mask = (p.causal && j == mt) || (k0 + kBN > p.seqlen);
+      const int lim = p.causal ? min(qrow + 1, p.seqlen) : p.seqlen;  // keys < lim visible
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        if (need_mask && k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
+        mx = fmaxf(mx, __uint_as_float(sr[c]));
+      }
+      mx *= p.scale_log2;  // the scale is positive, so it commutes with max
+      float alpha = 1.f;
+      bool resc = false;
+      if (j == 0) {
+        m_ref = mx;
+      } else {
+        const float m_new = fmaxf(m_ref, mx);
+        resc = m_new > m_ref + kLazyTau;
+        if (resc) {
+          alpha = ex2(m_ref - m_new);
+          m_ref = m_new;
+        }
+      }
+      const float u = m_ref == -INFINITY ? 0.f : m_ref;
+      float rowsum = 0.f;
+#pragma unroll
+      for (int qt = 0; qt < 4; ++qt) {  // 32 logits -> 16 packed bf16 pairs per store
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e]), p.scale_log2, -u));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e + 1]), p.scale_log2, -u));
+          rowsum += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(t_s + 16 * qt, pk);
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        // O_r must be quiescent (the previous tile's P.V into O_r done) before
+        // it is rescaled in place; rows that keep their reference use alpha 1.
+        if (!mbar_wait(&bars->o_done[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t ov[16];
+          tmem_ld16(t_o + 16 * c, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st16(t_o + 16 * c, ov);
+        }
+      }
+      l_run = l_run * alpha + rowsum;
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[r]);
+    }
+
+    // ---- epilogue: o = O1/l1 - lambda O2/l2 (+ V1 norm), channels [64 r, 64 r + 64) ----
+    __syncwarp();
+    if (failed) bars->abort_flag = 1;
+    const uint32_t last = (uint32_t)(n_kv - 1) & 1u;
+    mbar_wait(&bars->o_done[r], last, p.dev_status, &failed);
+    mbar_wait(&bars->o_done[r ^ 1], last, p.dev_status, &failed);
+    tc_fence_after();
+    x_inv_l[r * kBM + row] = 1.0f / l_run;
+    asm volatile("bar.sync 2, 256;" ::: "memory");
+    const float inv1 = x_inv_l[row];
+    const float inv2 = x_inv_l[kBM + row] * p.lambda[hh];
+    float o[64];
+    {
+      uint32_t a[32], c2[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(tmem + lane_off + kColO1 + 64 * r + 32 * half, a);
+        tmem_ld32(tmem + lane_off + kColO2 + 64 * r + 32 * half, c2);
+        tc_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          o[half * 32 + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
+      }
+    }
+    float mul = 1.f;
+    if (p.apply_norm) {
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) ss = fmaf(o[e], o[e], ss);
+      x_ss[r * kBM + row] = ss;
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      const float tot = x_ss[row] + x_ss[kBM + row];
+      mul = p.post_scale / sqrtf(tot * (1.0f / 128.0f) + p.eps);
+    }
+    if (qrow < p.seqlen && !bars->abort_flag) {
+      __nv_bfloat16* dst =
+          p.out + (((size_t)b * p.seqlen + qrow) * p.heads + hh) * 128 + 64 * r;
+#pragma unroll
+      for (int v8 = 0; v8 < 8; ++v8) {
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = v8 * 8 + e;
+          const float g = (p.apply_norm && p.norm_weight) ? __ldg(p.norm_weight + 64 * r + c) : 1.f;
+          y[e] = o[c] * mul * g;
+        }
+        uint4 w;
+        w.x = pack_bf16(y[0], y[1]);
+        w.y = pack_bf16(y[2], y[3]);
+        w.z = pack_bf16(y[4], y[5]);
+        w.w = pack_bf16(y[6], y[7]);
+        *reinterpret_cast<uint4*>(dst + v8 * 8) = w;
+      }
+    }
+  }
+
+  // ---- teardown: every role reaches this point, then TMEM is released ----
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                              const CUtensorMap& tm_v, const PrefillArgs& a, int num_sms,
+                              cudaStream_t stream) {
+  (void)num_sms;
+  Params p;
+  p.form = a.form;
+  p.batch = a.batch;
+  p.seqlen = a.seqlen;
+  p.heads = a.heads;
+  p.pairs_per_kv = a.pairs_per_kv;
+  p.n_qtiles = (a.seqlen + kBM - 1) / kBM;
+  p.causal = a.causal;
+  const double d = a.form == 1 ? 64.0 : 128.0;  // width of one branch's query
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(d));
+  p.lambda = a.lambda;
+  p.apply_norm = a.apply_norm;
+  p.norm_weight = a.norm_weight;
+  p.eps = a.eps;
+  p.post_scale = a.post_scale;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.dev_status = a.dev_status;
+  const int qbytes = a.form == 1 ? kTileBytes : 2 * kTileBytes;
+  const int smem = 1024 + qbytes + 2 * kStages * kTileBytes + (int)sizeof(Barriers) +
+                   4 * kBM * (int)sizeof(float) + 64;
+  cudaError_t e = cudaFuncSetAttribute(diffattn_prefill_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const long long grid = (long long)p.n_qtiles * a.batch * a.heads;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  diffattn_prefill_tc_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace da

@@ -1,0 +1,171 @@
+/*
+ * diffattn.h — C ABI of libdiffattn.so: differential attention on B200.
+ *
+ * The operator (both forms) is
+ *     DiffAttn = (softmax(Q1 K1^T / sqrt(d)) - lambda * softmax(Q2 K2^T / sqrt(d))) V
+ * as defined on the "Differential Transformer" glossary page (Ultralytics),
+ * section "Cómo funciona la atención diferencial", and in the lesson
+ * "Atención Diferencial (V2)" (ai-engineering.academy), section
+ * "La idea diferencial".  d is the width of ONE branch's query/key.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers marked "device" are caller-owned CUDA device memory; the
+ *    library never allocates, frees or keeps a pointer after returning.
+ *  - Tensors are dense, row-major (last index fastest), with the shapes
+ *    given per argument; element type is `dtype` (bf16 or fp32) for Q/K/V
+ *    and the output, fp32 for lambda and norm weights.  Q/K/V/out base
+ *    addresses must be 16-byte aligned (DA_ERR_ALIGNMENT otherwise).
+ *  - `out` must not overlap any input.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *    the legacy default stream) and returns before it completes.
+ *  - Argument errors are detected on the host before anything is enqueued
+ *    and return a negative da_status.  A launch failure returns DA_ERR_CUDA.
+ *    No C++ exception crosses this interface.
+ *  - `dev_status` (optional, device int, may be NULL): kernels that wait on
+ *    asynchronous copies bound every wait; if one ever times out the kernel
+ *    stores DA_ERR_DEVICE_TIMEOUT there (first error wins; the caller zeroes
+ *    it beforehand) and returns early, leaving the output undefined.
+ *  - Thread safety: no mutable global state; concurrent calls on different
+ *    streams are independent.
+ */
+#ifndef DIFFATTN_H_
+#define DIFFATTN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define DA_API __attribute__((visibility("default")))
+#else
+#define DA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DA_OK = 0,
+  DA_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad combination */
+  DA_ERR_UNSUPPORTED = -2,   /* valid arguments this library does not implement */
+  DA_ERR_ALIGNMENT = -3,     /* a base address is not 16-byte aligned */
+  DA_ERR_WORKSPACE = -4,     /* workspace missing or smaller than required */
+  DA_ERR_CUDA = -5,          /* a CUDA runtime/driver call or launch failed */
+  DA_ERR_DEVICE_TIMEOUT = -6 /* written to dev_status by a kernel whose wait timed out */
+} da_status;
+
+typedef enum { DA_BF16 = 0, DA_FP32 = 1 } da_dtype;
+
+/* Human-readable name of a da_status value (static string, never NULL). */
+DA_API const char* diffattn_status_string(int status);
+
+/* lambda_init(l) = 0.8 - 0.6 * exp(-0.3 * (l - 1)) for 1-based layer l
+ * (glossary page, "Cómo funciona": the per-layer starting value of lambda).
+ * Host only.  Returns NaN if layer < 1. */
+DA_API double diffattn_lambda_init(int layer);
+
+/* Per-head lambda from its four learned vectors (lesson "La idea
+ * diferencial"; glossary page: four small vectors, per-layer initial value):
+ *     lambda_h = exp(lq1_h . lk1_h) - exp(lq2_h . lk2_h) + lambda_init(layer)
+ * lq1, lk1, lq2, lk2 : device fp32 [n_heads, dim]
+ * lambda_out         : device fp32 [n_heads]
+ * Any real result is kept (lambda may be negative); no clamping.
+ * Errors: DA_ERR_INVALID_ARG for null pointers, n_heads < 1, dim < 1 or
+ * layer < 1. */
+DA_API int lambda_from_params(const float* lq1, const float* lk1, const float* lq2,
+                       const float* lk2, int n_heads, int dim, int layer,
+                       float* lambda_out, void* stream);
+
+/* V1 prefill (glossary page "Cómo funciona"; lesson "V1 vs V2").
+ * Each head's 2*d_qk-wide query/key row is split into two halves: branch 1
+ * uses columns [0, d_qk), branch 2 columns [d_qk, 2*d_qk).  V is d_v wide and
+ * shared by both branches.  Optional per-head normalisation of each output
+ * row (the page's "GroupNorm", an RMS norm over the d_v features):
+ *     y_c = o_c / sqrt(mean_c(o_c^2) + norm_eps) * g_c * (1 - lambda_init)
+ * q, k  : device [batch, seqlen, n_heads, 2*d_qk]
+ * v     : device [batch, seqlen, n_heads, d_v]
+ * out   : device [batch, seqlen, n_heads, d_v]
+ * lambda: device fp32 [n_heads]
+ * causal: nonzero -> query i sees keys j <= i (same for both branches)
+ * apply_norm: nonzero -> apply the normalisation above; norm_weight is a
+ *         device fp32 [d_v] gain or NULL for all-ones.  lambda_init is the
+ *         value that sets the post-norm scale (1 - lambda_init).
+ * Supported: fp32 with any d_qk <= 128, d_v <= 256 (CUDA-core kernel); bf16
+ * with d_qk = 64, d_v = 128 on the tcgen05 tensor-core kernel, other bf16
+ * widths up to the same limits on the CUDA-core kernel. */
+DA_API int diffattn_v1_fwd(const void* q, const void* k, const void* v, void* out,
+                    da_dtype dtype, int batch, int seqlen, int n_heads, int d_qk,
+                    int d_v, const float* lambda, int causal, int apply_norm,
+                    const float* norm_weight, float norm_eps, float lambda_init,
+                    int* dev_status, void* stream);
+
+/* V2 prefill (lesson "V1 vs V2": query heads doubled, KV heads kept, head
+ * width kept, no per-head norm; "Ejercicios" 5: GQA).
+ * Query heads come in subtracted pairs p = (2p, 2p+1), head 2p positive;
+ * query head h reads KV head h / (n_q_heads / n_kv_heads), so both heads of a
+ * pair share one KV head (n_q_heads / n_kv_heads must be even).
+ * q     : device [batch, seqlen, n_q_heads, head_dim]
+ * k, v  : device [batch, seqlen, n_kv_heads, head_dim]
+ * out   : device [batch, seqlen, n_q_heads / 2, head_dim]
+ * lambda: device fp32 [n_q_heads / 2]
+ * Supported: bf16 head_dim = 128 on the tcgen05 kernel; fp32 (and other bf16
+ * widths) with head_dim <= 128 on the CUDA-core kernel. */
+DA_API int diffattn_v2_prefill(const void* q, const void* k, const void* v, void* out,
+                        da_dtype dtype, int batch, int seqlen, int n_q_heads,
+                        int n_kv_heads, int head_dim, const float* lambda,
+                        int causal, int* dev_status, void* stream);
+
+/* Bytes of device workspace diffattn_v2_decode needs for these sizes
+ * (0 if it needs none).  Host only; never fails (returns 0 for bad sizes,
+ * which the decode call then rejects). */
+DA_API size_t diffattn_v2_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads,
+                                         int head_dim, int max_cache_len);
+
+/* V2 single-token decode against a KV cache (lesson "V1 vs V2": the cache is
+ * read once per step for both heads of every pair).  The new token's K/V
+ * must already be in the cache: batch entry b attends cache rows
+ * 0 .. cache_lens[b]-1.
+ * q        : device [batch, n_q_heads, head_dim]
+ * k_cache, v_cache : device [batch, max_len, n_kv_heads, head_dim]
+ * cache_lens: device int32 [batch] with 1 <= cache_lens[b] <= max_len, or
+ *            NULL (every entry uses max_len).  Values are not checked on the
+ *            host; an out-of-range length is clamped on the device.
+ * out      : device [batch, n_q_heads / 2, head_dim]
+ * lambda   : device fp32 [n_q_heads / 2]
+ * workspace: device, at least diffattn_v2_decode_workspace_size(...) bytes,
+ *            16-byte aligned, caller-owned scratch (contents undefined
+ *            after the call); NULL allowed only when that size is 0.
+ * Supported: bf16 head_dim = 128 with (n_q_heads / n_kv_heads) in {2, 4, 6, 8}
+ * on the split-KV tensor-core kernel; other shapes (and fp32) with
+ * head_dim <= 128 on the CUDA-core kernel. */
+DA_API int diffattn_v2_decode(const void* q, const void* k_cache, const void* v_cache,
+                       const int* cache_lens, int max_len, void* out, da_dtype dtype,
+                       int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                       const float* lambda, void* workspace, size_t workspace_bytes,
+                       int* dev_status, void* stream);
+
+/* Bytes of device workspace diffattn_v1_decode needs (0 if none). */
+DA_API size_t diffattn_v1_decode_workspace_size(int batch, int n_heads, int d_qk, int d_v,
+                                         int max_cache_len);
+
+/* V1 single-token decode against a multi-head cache (lesson "V1 vs V2").
+ * Both branches read each cached value row once here.
+ * q       : device [batch, n_heads, 2*d_qk]
+ * k_cache : device [batch, max_len, n_heads, 2*d_qk]
+ * v_cache : device [batch, max_len, n_heads, d_v]
+ * out     : device [batch, n_heads, d_v]
+ * Other arguments as for diffattn_v1_fwd and diffattn_v2_decode.
+ * Supported: bf16 d_qk = 64, d_v = 128 on the split-KV kernel; other
+ * widths (and fp32) with d_qk <= 128, d_v <= 256 on the CUDA-core kernel. */
+DA_API int diffattn_v1_decode(const void* q, const void* k_cache, const void* v_cache,
+                       const int* cache_lens, int max_len, void* out, da_dtype dtype,
+                       int batch, int n_heads, int d_qk, int d_v, const float* lambda,
+                       int apply_norm, const float* norm_weight, float norm_eps,
+                       float lambda_init, void* workspace, size_t workspace_bytes,
+                       int* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIFFATTN_H_ */

@@ -1,0 +1,135 @@
+"""The C-ABI library builds, loads without a GPU, exports every symbol the
+public header declares, and rejects bad arguments on the host before any
+CUDA call (so these run on a machine with no device)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "diffattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from differential_attention_sm_b200 import build as B
+    B.build()
+    from differential_attention_sm_b200 import binding
+    return binding.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return set(re.findall(r"DA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for name in ("diffattn_v1_fwd", "diffattn_v2_prefill", "diffattn_v2_decode",
+                 "lambda_from_params"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from differential_attention_sm_b200 import binding
+    syms = declared_symbols()
+    assert syms == set(binding.EXPORTS)
+    for name in syms:
+        assert hasattr(lib, name), name
+
+
+def test_lambda_init_and_status_strings(lib):
+    from differential_attention_sm_b200 import binding as b
+    assert b.diffattn_lambda_init(1) == pytest.approx(0.2, abs=1e-15)
+    assert math.isnan(b.diffattn_lambda_init(0))
+    import oracle
+    for l in (1, 2, 12, 24, 100):
+        assert b.diffattn_lambda_init(l) == pytest.approx(oracle.lambda_init(l), abs=1e-15)
+    assert b.status_string(b.DA_OK) == "DA_OK"
+    assert b.status_string(b.DA_ERR_DEVICE_TIMEOUT) == "DA_ERR_DEVICE_TIMEOUT"
+    assert b.status_string(12345) == "DA_ERR_UNKNOWN"
+
+
+# Fake device addresses: validation must reject before dereferencing anything.
+A = 0x10000   # 16-byte aligned
+U = 0x10008   # misaligned
+
+
+def test_v1_fwd_host_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    f = lib.diffattn_v1_fwd
+    ok = (A, A, A, A, b.DA_BF16, 1, 128, 1, 64, 128, A, 1, 1, None, 1e-5, 0.2, None, None)
+    bad = list(ok); bad[0] = None
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[4] = 7
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[6] = 0
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[8] = 129
+    assert f(*bad) == b.DA_ERR_UNSUPPORTED
+    bad = list(ok); bad[1] = U
+    assert f(*bad) == b.DA_ERR_ALIGNMENT
+    bad = list(ok); bad[14] = -1.0
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+
+
+def test_v2_prefill_host_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    f = lib.diffattn_v2_prefill
+    ok = [A, A, A, A, b.DA_BF16, 2, 256, 32, 8, 128, A, 1, None, None]
+    bad = list(ok); bad[7] = 31          # odd query heads
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[7], bad[8] = 8, 8  # group 1: a pair would span two KV heads
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[3] = U
+    assert f(*bad) == b.DA_ERR_ALIGNMENT
+    bad = list(ok); bad[10] = None
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+
+
+def test_decode_workspace_and_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    ws = b.diffattn_v2_decode_workspace_size(64, 64, 8, 128, 32768)
+    assert ws > 0 and ws % 16 == 0
+    assert b.diffattn_v2_decode_workspace_size(64, 64, 8, 64, 32768) == 0   # generic path
+    assert b.diffattn_v2_decode_workspace_size(0, 64, 8, 128, 32768) == 0
+    assert b.diffattn_v1_decode_workspace_size(64, 32, 64, 128, 32768) > 0
+    f = lib.diffattn_v2_decode
+    args = [A, A, A, None, 32768, A, b.DA_BF16, 64, 64, 8, 128, A, A, ws - 16, None, None]
+    assert f(*args) == b.DA_ERR_WORKSPACE
+    args[12] = None
+    args[13] = ws
+    assert f(*args) == b.DA_ERR_WORKSPACE
+    args[12] = U
+    assert f(*args) == b.DA_ERR_ALIGNMENT
+    args[12] = A
+    args[4] = 0
+    assert f(*args) == b.DA_ERR_INVALID_ARG
+    g = lib.diffattn_v1_decode
+    wsv1 = b.diffattn_v1_decode_workspace_size(2, 4, 64, 128, 1000)
+    args = [A, A, A, None, 1000, A, b.DA_BF16, 2, 4, 64, 128, A, 1, None, 1e-5, 0.2, A,
+            wsv1 - 1, None, None]
+    assert g(*args) == b.DA_ERR_WORKSPACE
+    args[1] = U
+    assert g(*args) == b.DA_ERR_ALIGNMENT
+
+
+def test_lambda_from_params_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    f = lib.lambda_from_params
+    assert f(A, A, A, A, 4, 64, 0, A, None) == b.DA_ERR_INVALID_ARG
+    assert f(A, None, A, A, 4, 64, 1, A, None) == b.DA_ERR_INVALID_ARG
+    assert f(A, A, A, A, 0, 64, 1, A, None) == b.DA_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The library and its binding never load the oracle."""
+    pkg = os.path.join(ROOT, "differential_attention_sm_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text, fn
+                assert "diffattn_oracle" not in text, fn

@@ -1,0 +1,201 @@
+"""GPU parity of the prefill path (C ABI via the binding) against the fp64
+oracle: the tiny fp32 workload, small ragged bf16 cases on the tensor-core
+kernel and the generic kernel, and the full-size bf16 workloads on sampled
+rows (same launch configuration as the benchmark)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from differential_attention_sm_b200 import inputs as I
+from parity import (assert_bf16_close, assert_fp32_close, assert_status_ok, status_word)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    from differential_attention_sm_b200 import binding
+    binding.load()
+    return binding
+
+
+def cuda(t):
+    return t.cuda().contiguous()
+
+
+# ---------------------------------------------------------------------------
+# tiny fp32 workload: B1 H1 N128 d8 dv16, lambda 0.8 or from params (layer 1)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("lam_mode", ["fixed", "params"])
+def test_tiny_v1_fp32(B, causal, lam_mode):
+    w = I.WORKLOADS["tiny_v1_fp32"]
+    x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed, dtype=torch.float32)
+    if lam_mode == "fixed":
+        lam_host = np.array([w.fixed_lambda])
+        lam_dev = torch.tensor([w.fixed_lambda], dtype=torch.float32, device="cuda")
+    else:
+        lam_host = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+        lam_dev = B.lambda_from_params(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")),
+                                       w.layer)
+    st = status_word()
+    out = B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), lam_dev, causal=causal,
+                            dev_status=st)
+    assert_status_ok(st)
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam_host, np.arange(w.B * w.N * w.H), causal=causal)
+    assert_fp32_close(out.reshape(-1, w.dv), ref, "tiny fp32")
+
+
+def test_worked_example_on_gpu(B):
+    q1, k1, q2, k2, v = I.worked_example()
+    q = torch.cat([q1, q2], -1).reshape(1, 6, 1, 16)
+    k = torch.cat([k1, k2], -1).reshape(1, 6, 1, 16)
+    vv = v.reshape(1, 6, 1, 16)
+    lam = torch.tensor([0.8], device="cuda")
+    out = B.diffattn_v1_fwd(cuda(q), cuda(k), cuda(vv), lam, causal=False)
+    ref = O.v1_rows(q, k, vv, [0.8], np.arange(6), causal=False)
+    assert_fp32_close(out.reshape(6, 16), ref, "worked example")
+
+
+def test_lambda_from_params_matches_oracle(B):
+    g = torch.Generator().manual_seed(5)
+    vecs = [0.3 * torch.randn(16, 64, generator=g) for _ in range(4)]
+    for layer in (1, 12, 24):
+        got = B.lambda_from_params(*(cuda(t) for t in vecs), layer).cpu().double().numpy()
+        ref = O.lambda_from_params(*vecs, layer)
+        assert np.abs(got - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
+
+
+# ---------------------------------------------------------------------------
+# V1 bf16, small and ragged (tcgen05 kernel: d_qk 64, d_v 128)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("Bn,N,H,causal", [
+    (2, 300, 3, True),    # two full tiles + a ragged tail
+    (1, 128, 2, True),    # exactly one tile
+    (1, 1, 2, True),      # single token
+    (2, 129, 1, True),    # one row past a tile edge
+    (1, 200, 2, False),   # non-causal, ragged key tail
+    (1, 640, 1, True),    # five tiles: exercises the 2-stage rings' reuse
+])
+def test_v1_bf16_small(B, Bn, N, H, causal):
+    d, dv, layer = 64, 128, 12
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=100 + N, dtype=torch.bfloat16)
+    lam_dev = B.lambda_from_params(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")), layer)
+    lam_host = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], layer)
+    li = O.lambda_init(layer)
+    st = status_word()
+    out = B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), lam_dev, causal=causal,
+                            apply_norm=True, norm_eps=1e-5, lambda_init=li, dev_status=st)
+    assert_status_ok(st)
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam_host, np.arange(Bn * N * H), causal=causal,
+                    apply_norm=True, eps=1e-5, lambda_init_value=li)
+    assert_bf16_close(out.reshape(-1, dv), ref, False, "v1 bf16 N=%d" % N)
+
+
+def test_v1_bf16_no_norm_and_gain(B):
+    Bn, N, H, d, dv = 1, 257, 2, 64, 128
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=7, dtype=torch.bfloat16)
+    lam = torch.tensor([0.8, -0.3], dtype=torch.float32)
+    out = B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(lam), causal=True)
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam.double().numpy(), np.arange(Bn * N * H),
+                    causal=True)
+    assert_bf16_close(out.reshape(-1, dv), ref, True, "v1 bf16 no norm")
+    g = 0.5 + torch.rand(dv, generator=torch.Generator().manual_seed(3))
+    li = O.lambda_init(3)
+    out = B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(lam), causal=True,
+                            apply_norm=True, norm_weight=cuda(g), lambda_init=li)
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam.double().numpy(), np.arange(Bn * N * H),
+                    causal=True, apply_norm=True, norm_weight=g, lambda_init_value=li)
+    assert_bf16_close(out.reshape(-1, dv), ref, False, "v1 bf16 gain")
+
+
+def test_v1_bf16_generic_widths(B):
+    """Widths outside the tensor-core kernel run on the CUDA-core kernel."""
+    Bn, N, H, d, dv = 1, 150, 2, 32, 64
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=8, dtype=torch.bfloat16)
+    lam = torch.tensor([0.6, 0.9], dtype=torch.float32)
+    out = B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(lam), causal=True,
+                            apply_norm=True, lambda_init=0.2)
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam.double().numpy(), np.arange(Bn * N * H),
+                    causal=True, apply_norm=True, lambda_init_value=0.2)
+    assert_bf16_close(out.reshape(-1, dv), ref, False, "v1 generic")
+
+
+# ---------------------------------------------------------------------------
+# V2 bf16, small and ragged (tcgen05 kernel: head_dim 128)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("Bn,N,Hq,Hkv,causal", [
+    (2, 333, 8, 2, True),
+    (1, 256, 4, 2, True),    # group of 2: one pair per KV head
+    (1, 1, 4, 1, True),
+    (1, 190, 8, 1, False),
+])
+def test_v2_bf16_small(B, Bn, N, Hq, Hkv, causal):
+    d = 128
+    x = I.v2_inputs(Bn, N, Hq, Hkv, d, seed=200 + N)
+    st = status_word()
+    out = B.diffattn_v2_prefill(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(x["lam"]),
+                                causal=causal, dev_status=st)
+    assert_status_ok(st)
+    ref = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], np.arange(Bn * N * Hq // 2),
+                    causal=causal)
+    assert_bf16_close(out.reshape(-1, d), ref, True, "v2 bf16 N=%d" % N)
+
+
+def test_v2_fp32_generic(B):
+    Bn, N, Hq, Hkv, d = 1, 70, 4, 2, 16
+    x = I.v2_inputs(Bn, N, Hq, Hkv, d, seed=9, dtype=torch.float32)
+    out = B.diffattn_v2_prefill(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(x["lam"]),
+                                causal=True)
+    ref = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], np.arange(Bn * N * Hq // 2), causal=True)
+    assert_fp32_close(out.reshape(-1, d), ref, "v2 fp32")
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled rows
+# ---------------------------------------------------------------------------
+def sample_rows(Bn, N, H, n_random, seed):
+    """Rows (b*N + i)*H + h: tile edges, first/last rows and random ones."""
+    rng = np.random.default_rng(seed)
+    picks = set()
+    for i in {0, 1, 127, 128, 129, N // 2, N - 129, N - 128, N - 2, N - 1}:
+        if 0 <= i < N:
+            for _ in range(2):
+                picks.add((int(rng.integers(Bn)) * N + i) * H + int(rng.integers(H)))
+    picks.update(int(r) for r in rng.integers(0, Bn * N * H, n_random))
+    return np.array(sorted(picks))
+
+
+@pytest.mark.parametrize("name", ["v1_prefill_bf16", "v1_long_bf16"])
+def test_v1_full_size_sampled(B, name):
+    w = I.WORKLOADS[name]
+    x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed, planted=w.planted)
+    lam_dev = B.lambda_from_params(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")), w.layer)
+    lam_host = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+    li = O.lambda_init(w.layer)
+    st = status_word()
+    out = B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), lam_dev, causal=True,
+                            apply_norm=True, norm_eps=w.eps, lambda_init=li, dev_status=st)
+    assert_status_ok(st)
+    rows = sample_rows(w.B, w.N, w.H, 48 if w.N > 8192 else 160, seed=w.seed)
+    if w.planted:  # the two rows the needles were planted for, every head
+        extra = [((0 * w.N + i) * w.H + h) for i in (w.N - 2, w.N - 1) for h in range(w.H)]
+        rows = np.unique(np.concatenate([rows, np.array(extra)]))
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam_host, rows, causal=True, apply_norm=True,
+                    eps=w.eps, lambda_init_value=li)
+    got = out.reshape(-1, w.dv)[torch.from_numpy(rows).cuda()]
+    assert_bf16_close(got, ref, False, name)
+
+
+def test_v2_full_size_sampled(B):
+    w = I.WORKLOADS["v2_prefill_bf16"]
+    x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
+    st = status_word()
+    out = B.diffattn_v2_prefill(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(x["lam"]),
+                                causal=True, dev_status=st)
+    assert_status_ok(st)
+    rows = sample_rows(w.B, w.N, w.Hq // 2, 160, seed=w.seed)
+    ref = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], rows, causal=True)
+    got = out.reshape(-1, w.d)[torch.from_numpy(rows).cuda()]
+    assert_bf16_close(got, ref, True, "v2 full")
