@@ -35,6 +35,7 @@ EXPORTS = (
     "diffattn_v2_prefill",
     "diffattn_v2_decode_workspace_size",
     "diffattn_v2_decode",
+    "diffattn_v2_decode_noalloc",
     "diffattn_v1_decode_workspace_size",
     "diffattn_v1_decode",
 )
@@ -81,6 +82,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.diffattn_v2_decode.restype = _i
     lib.diffattn_v2_decode.argtypes = [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp,
                                        _vp, _sz, _vp, _vp]
+    lib.diffattn_v2_decode_noalloc.restype = _i
+    lib.diffattn_v2_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp,
+                                               _vp, _vp]
     lib.diffattn_v1_decode_workspace_size.restype = _sz
     lib.diffattn_v1_decode_workspace_size.argtypes = [_i, _i, _i, _i, _i]
     lib.diffattn_v1_decode.restype = _i
@@ -197,6 +201,24 @@ def diffattn_v2_decode(q, k_cache, v_cache, lam, *, cache_lens=None, workspace=N
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), L, _ptr(out), _dtype_code(q),
         B, Hq, Hkv, d, _ptr(lam), _ptr(workspace), ws_bytes, _ptr(dev_status),
         _stream(stream)))
+    return out
+
+
+def diffattn_v2_decode_noalloc(q, k_cache, v_cache, lam, *, cache_lens=None, out=None,
+                               dev_status=None, stream=None):
+    """V2 decode without a workspace (bf16, head_dim 128): for callers that
+    cannot allocate device memory.  The split-KV partials live in the
+    library's fixed 8 MiB device array; calls that overlap on the GPU race
+    on it.  Note that this wrapper still allocates `out` through PyTorch when
+    it is not given."""
+    _need_cuda(q, k_cache, v_cache, lam, cache_lens, dev_status)
+    B, Hq, d = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty(B, Hq // 2, d, dtype=q.dtype, device=q.device)
+    _check("diffattn_v2_decode_noalloc", load().diffattn_v2_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), L, _ptr(out), B, Hq, Hkv,
+        _ptr(lam), _ptr(dev_status), _stream(stream)))
     return out
 
 

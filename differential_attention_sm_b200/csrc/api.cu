@@ -82,6 +82,13 @@ bool fits_int(long long x) { return x > 0 && x < (1LL << 31); }
 
 }  // namespace
 
+namespace da {
+int make_tmap_bf16_4d(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  return make_tmap_4d(tm, base, d0, d1, d2, d3, b0, b1, b2, b3);
+}
+}  // namespace da
+
 extern "C" {
 
 const char* diffattn_status_string(int status) {

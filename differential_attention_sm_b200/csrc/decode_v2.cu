@@ -352,6 +352,30 @@ V2DecodePlan plan_v2_decode(int batch, int n_kv_heads, int max_len, int num_sms)
   return best;
 }
 
+V2DecodePlan plan_v2_decode_capped(int batch, int n_kv_heads, int max_len, int num_sms,
+                                   size_t max_bytes) {
+  const long units = (long)batch * n_kv_heads;
+  const int max_split = (max_len + kChunk - 1) / kChunk;
+  const size_t per_item = (size_t)kHeads * (kD + 2) * sizeof(float);
+  V2DecodePlan best{0, 0, 0, 0};
+  double best_cost = 1e300;
+  for (int ns = 1; ns <= max_split && ns <= 256; ++ns) {
+    int sl = (max_len + ns - 1) / ns;
+    sl = (sl + kChunk - 1) / kChunk * kChunk;
+    const int ns_eff = (max_len + sl - 1) / sl;
+    const long items = units * ns_eff;
+    if ((size_t)items * per_item > max_bytes) break;  // more splits only grow the workspace
+    const long grid = items < num_sms ? items : num_sms;
+    const long per_cta = (items + grid - 1) / grid;
+    const double cost = (double)per_cta * (sl + kChunk);
+    if (cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = {ns_eff, sl, (int)items, (int)grid};
+    }
+  }
+  return best;
+}
+
 size_t v2_decode_workspace_bytes(const V2DecodePlan& plan) {
   return (size_t)plan.n_items * kHeads * (kD + 2) * sizeof(float);
 }

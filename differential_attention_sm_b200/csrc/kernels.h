@@ -48,6 +48,10 @@ struct V2DecodePlan {
   int grid;       // persistent CTAs
 };
 V2DecodePlan plan_v2_decode(int batch, int n_kv_heads, int max_len, int num_sms);
+// Same search restricted to plans whose workspace fits in max_bytes; returns
+// a plan with n_items == 0 if none does.
+V2DecodePlan plan_v2_decode_capped(int batch, int n_kv_heads, int max_len, int num_sms,
+                                   size_t max_bytes);
 size_t v2_decode_workspace_bytes(const V2DecodePlan& plan);
 cudaError_t launch_v2_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
                              const int* lens, int max_len, void* out, int batch, int n_q_heads,
@@ -65,6 +69,11 @@ cudaError_t launch_v1_decode(const void* q, const void* k_cache, const void* v_c
                              const float* lambda, int apply_norm, const float* norm_weight,
                              float eps, float post_scale, const V1DecodePlan& plan,
                              void* workspace, cudaStream_t stream);
+
+// 4-D bf16 tensor map (128-byte swizzle, zero fill) over a dense
+// [d3][d2][d1][d0] array; returns a da_status.  Implemented in api.cu.
+int make_tmap_bf16_4d(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3);
 
 // ---- tcgen05 prefill (bf16) -----------------------------------------------
 // Form 1 (V1): Q/K rows are 128 wide (two 64-wide branches), V 128 wide,

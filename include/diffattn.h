@@ -144,6 +144,39 @@ DA_API int diffattn_v2_decode(const void* q, const void* k_cache, const void* v_
                        const float* lambda, void* workspace, size_t workspace_bytes,
                        int* dev_status, void* stream);
 
+/* Size of the fixed device scratch array behind diffattn_v2_decode_noalloc:
+ * 8 MiB.  Every GPU on which that entry point runs keeps this array until the
+ * process exits. */
+#define DA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* diffattn_v2_decode for callers that cannot allocate device memory.
+ * The source pages have no counterpart to this entry point; it exists for
+ * callers that are not able to hand over a workspace, e.g. code that must
+ * never call cudaMalloc (an allocation can synchronise the device and stall
+ * a serving loop), a plug-in whose host framework owns every device buffer,
+ * or a runtime whose device-memory budget is fixed at start-up.
+ * Same operator, arguments and layouts as diffattn_v2_decode with
+ * dtype = DA_BF16 and head_dim = 128, minus the workspace: the split-KV
+ * partial results go to a statically allocated device array of
+ * DA_NOALLOC_SCRATCH_BYTES, and the call allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine).
+ *  - Supported: n_q_heads / n_kv_heads in {2, 4, 6, 8}; otherwise
+ *    DA_ERR_UNSUPPORTED.  Sizes whose partial results cannot fit in the
+ *    scratch (batch * n_kv_heads above 2016) return DA_ERR_UNSUPPORTED
+ *    before anything is enqueued.
+ *  - Set-up: the first call on a device, with that device current, looks up
+ *    the array's device address (cudaGetSymbolAddress) and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last
+ *    call's contents; nothing in it needs to start at zero.  Calls whose
+ *    execution overlaps on the GPU (other streams, other host threads) race
+ *    on the array: the caller must serialise them. */
+DA_API int diffattn_v2_decode_noalloc(const void* q, const void* k_cache,
+                                      const void* v_cache, const int* cache_lens,
+                                      int max_len, void* out, int batch, int n_q_heads,
+                                      int n_kv_heads, const float* lambda,
+                                      int* dev_status, void* stream);
+
 /* Bytes of device workspace diffattn_v1_decode needs (0 if none). */
 DA_API size_t diffattn_v1_decode_workspace_size(int batch, int n_heads, int d_qk, int d_v,
                                          int max_cache_len);
