@@ -312,9 +312,13 @@ def time_call(fn, iters, warmup, stream):
     return a.elapsed_time(b) / iters
 
 
-def run_extras(local_rank, peaks, peak_src):
-    """The other workloads, one GPU: V1 long-context prefill, V2 prefill,
-    V2 decode and V1 decode (same kernels the parity tests check)."""
+def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
+    """The other workloads, one GPU: V2 prefill, V1 long-context prefill,
+    V2 decode and V1 decode (same kernels the parity tests check).
+    `only` restricts the run to one of them and `decode_batch` shrinks the
+    decode batch (used for small profiling runs)."""
+    import dataclasses
+
     import torch
     from differential_attention_sm_b200 import binding as Bd
     from differential_attention_sm_b200 import inputs as I
@@ -322,77 +326,89 @@ def run_extras(local_rank, peaks, peak_src):
     stream = torch.cuda.current_stream(dev)
     out = {}
 
-    # V2 causal prefill: B2 Hq32 Hkv8 d128 N8192
-    w = I.WORKLOADS["v2_prefill_bf16"]
-    x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
-    q, k, v, lam = (x[n].to(dev) for n in ("q", "k", "v", "lam"))
-    o = torch.empty(w.B, w.N, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
-    ms = time_call(lambda: Bd.diffattn_v2_prefill(q, k, v, lam, causal=True, out=o), 20, 3, stream)
-    fl = prefill_pairs(w.B, w.N, w.Hq // 2) * v2_flops_per_pair(w.d)
-    t = fl / (ms * 1e-3) / 1e12
-    out["v2_prefill_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
-                              "frac": round(t / peaks["bf16_tflops"], 4),
-                              "peak": peaks["bf16_tflops"], "flop": fl}
-    del q, k, v, o, x
+    def want(name):
+        return only is None or only == name
 
-    # V1 long-context prefill: B1 H16 N32768 layer 24, planted signal
-    w = I.WORKLOADS["v1_long_bf16"]
-    x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed, planted=w.planted)
-    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
-    lv = [x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")]
-    lamt = Bd.lambda_from_params(*lv, w.layer)
-    li = Bd.diffattn_lambda_init(w.layer)
-    o = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=dev)
-    ms = time_call(lambda: Bd.diffattn_v1_fwd(q, k, v, lamt, causal=True, apply_norm=True,
-                                              lambda_init=li, out=o), 5, 2, stream)
-    fl = prefill_pairs(w.B, w.N, w.H) * v1_flops_per_pair(w.d, w.dv)
-    t = fl / (ms * 1e-3) / 1e12
-    out["v1_long_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
-                           "frac": round(t / peaks["bf16_tflops"], 4), "flop": fl}
-    del q, k, v, o, x
+    def wl(name):
+        w = I.WORKLOADS[name]
+        if decode_batch and w.kind.endswith("decode"):
+            w = dataclasses.replace(w, B=decode_batch)
+        return w
 
-    # V2 decode: B64 L32768 Hq64 Hkv8 d128
-    w = I.WORKLOADS["v2_decode_bf16"]
-    x = I.v2_decode_inputs(w.B, w.L, w.Hq, w.Hkv, w.d, w.seed, fill_caches=False)
-    kc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.Hkv, w.d, dtype=torch.bfloat16,
-                                             device=dev), 1)
-    vc = I.fill_normal_on_device(torch.empty_like(kc), 2)
-    q, lam = x["q"].to(dev), x["lam"].to(dev)
-    ws = torch.empty(Bd.diffattn_v2_decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.L),
-                     dtype=torch.uint8, device=dev)
-    o = torch.empty(w.B, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
-    ms = time_call(lambda: Bd.diffattn_v2_decode(q, kc, vc, lam, workspace=ws, out=o), 20, 3,
-                   stream)
-    by = v2_decode_bytes(w.B, w.L, w.Hkv, w.d, w.Hq)
-    gbs = by / (ms * 1e-3) / 1e9
-    out["v2_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
-                             "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"],
-                             "bytes": by}
-    del kc, vc, ws
-    torch.cuda.empty_cache()
+    if want("v2_prefill_bf16"):  # B2 Hq32 Hkv8 d128 N8192
+        w = wl("v2_prefill_bf16")
+        x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
+        q, k, v, lam = (x[n].to(dev) for n in ("q", "k", "v", "lam"))
+        o = torch.empty(w.B, w.N, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v2_prefill(q, k, v, lam, causal=True, out=o), 20, 3,
+                       stream)
+        fl = prefill_pairs(w.B, w.N, w.Hq // 2) * v2_flops_per_pair(w.d)
+        t = fl / (ms * 1e-3) / 1e12
+        out["v2_prefill_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
+                                  "frac": round(t / peaks["bf16_tflops"], 4),
+                                  "peak": peaks["bf16_tflops"], "flop": fl}
+        del q, k, v, o, x
 
-    # V1 decode (comparison): B64 L32768 H32 d64 dv128
-    w = I.WORKLOADS["v1_decode_bf16"]
-    x = I.v1_decode_inputs(w.B, w.L, w.H, w.d, w.dv, w.seed, fill_caches=False)
-    kc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.H, 2 * w.d, dtype=torch.bfloat16,
-                                             device=dev), 3)
-    vc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.H, w.dv, dtype=torch.bfloat16,
-                                             device=dev), 4)
-    q = x["q"].to(dev)
-    lamt = Bd.lambda_from_params(*(x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")), w.layer)
-    li = Bd.diffattn_lambda_init(w.layer)
-    ws = torch.empty(Bd.diffattn_v1_decode_workspace_size(w.B, w.H, w.d, w.dv, w.L),
-                     dtype=torch.uint8, device=dev)
-    o = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=dev)
-    ms = time_call(lambda: Bd.diffattn_v1_decode(q, kc, vc, lamt, apply_norm=True,
-                                                 lambda_init=li, workspace=ws, out=o), 5, 2,
-                   stream)
-    by = v1_decode_bytes(w.B, w.L, w.H, w.d, w.dv)
-    gbs = by / (ms * 1e-3) / 1e9
-    out["v1_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
-                             "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": by}
-    del kc, vc, ws
-    torch.cuda.empty_cache()
+    if want("v1_long_bf16"):  # B1 H16 N32768, layer 24, planted signal
+        w = wl("v1_long_bf16")
+        x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed, planted=w.planted)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        lamt = Bd.lambda_from_params(*(x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")),
+                                     w.layer)
+        li = Bd.diffattn_lambda_init(w.layer)
+        o = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v1_fwd(q, k, v, lamt, causal=True, apply_norm=True,
+                                                  lambda_init=li, out=o), 5, 2, stream)
+        fl = prefill_pairs(w.B, w.N, w.H) * v1_flops_per_pair(w.d, w.dv)
+        t = fl / (ms * 1e-3) / 1e12
+        out["v1_long_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
+                               "frac": round(t / peaks["bf16_tflops"], 4), "flop": fl}
+        del q, k, v, o, x
+
+    if want("v2_decode_bf16"):  # B64 L32768 Hq64 Hkv8 d128
+        w = wl("v2_decode_bf16")
+        x = I.v2_decode_inputs(w.B, w.L, w.Hq, w.Hkv, w.d, w.seed, fill_caches=False)
+        kc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.Hkv, w.d, dtype=torch.bfloat16,
+                                                 device=dev), 1)
+        vc = I.fill_normal_on_device(torch.empty_like(kc), 2)
+        q, lam = x["q"].to(dev), x["lam"].to(dev)
+        ws = torch.empty(Bd.diffattn_v2_decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, w.L),
+                         dtype=torch.uint8, device=dev)
+        o = torch.empty(w.B, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v2_decode(q, kc, vc, lam, workspace=ws, out=o), 20, 3,
+                       stream)
+        by = v2_decode_bytes(w.B, w.L, w.Hkv, w.d, w.Hq)
+        gbs = by / (ms * 1e-3) / 1e9
+        out["v2_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
+                                 "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                 "peak": peaks["hbm_gbs"], "bytes": by, "batch": w.B}
+        del kc, vc, ws
+        torch.cuda.empty_cache()
+
+    if want("v1_decode_bf16"):  # B64 L32768 H32 d64 dv128 (comparison)
+        w = wl("v1_decode_bf16")
+        x = I.v1_decode_inputs(w.B, w.L, w.H, w.d, w.dv, w.seed, fill_caches=False)
+        kc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.H, 2 * w.d, dtype=torch.bfloat16,
+                                                 device=dev), 3)
+        vc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.H, w.dv, dtype=torch.bfloat16,
+                                                 device=dev), 4)
+        q = x["q"].to(dev)
+        lamt = Bd.lambda_from_params(*(x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")),
+                                     w.layer)
+        li = Bd.diffattn_lambda_init(w.layer)
+        ws = torch.empty(Bd.diffattn_v1_decode_workspace_size(w.B, w.H, w.d, w.dv, w.L),
+                         dtype=torch.uint8, device=dev)
+        o = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v1_decode(q, kc, vc, lamt, apply_norm=True,
+                                                     lambda_init=li, workspace=ws, out=o), 5, 2,
+                       stream)
+        by = v1_decode_bytes(w.B, w.L, w.H, w.d, w.dv)
+        gbs = by / (ms * 1e-3) / 1e9
+        out["v1_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
+                                 "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": by,
+                                 "batch": w.B}
+        del kc, vc, ws
+        torch.cuda.empty_cache()
     out["peak_source"] = peak_src
     return out
 
@@ -472,10 +488,23 @@ def main():
                     help="skip the secondary workloads (V2 prefill, long V1, decode)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded host time for the oracle CPU baseline")
+    ap.add_argument("--only", default=None,
+                    choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
+                             "v1_decode_bf16"],
+                    help="run just this secondary workload (one GPU) and print its numbers")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="with --only: smaller decode batch (profiling runs)")
     args = ap.parse_args()
     rank, world, local_rank = dist_env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.only:
+        import torch
+        torch.cuda.set_device(local_rank)
+        peaks, peak_src = load_peaks()
+        print(json.dumps(run_extras(local_rank, peaks, peak_src, args.only, args.decode_batch)),
+              flush=True)
+        return 0
 
     import torch
     torch.cuda.set_device(local_rank)
