@@ -138,9 +138,10 @@ int diffattn_v1_fwd(const void* q, const void* k, const void* v, void* out, da_d
     if (sms < 1) return DA_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     // [B][N][H][128] viewed as 4-D (c, h, n, b); 64-column boxes of 128 rows
+    // Q: 128-row boxes (one query tile); K, V: 64-row boxes (one key tile)
     if (make_tmap_4d(&tq, q, 128, n_heads, seqlen, batch, 64, 1, 128, 1) ||
-        make_tmap_4d(&tk, k, 128, n_heads, seqlen, batch, 64, 1, 128, 1) ||
-        make_tmap_4d(&tv, v, 128, n_heads, seqlen, batch, 64, 1, 128, 1))
+        make_tmap_4d(&tk, k, 128, n_heads, seqlen, batch, 64, 1, 64, 1) ||
+        make_tmap_4d(&tv, v, 128, n_heads, seqlen, batch, 64, 1, 64, 1))
       return DA_ERR_CUDA;
     da::PrefillArgs a{};
     a.form = 1;
@@ -214,8 +215,8 @@ int diffattn_v2_prefill(const void* q, const void* k, const void* v, void* out, 
     if (sms < 1) return DA_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     if (make_tmap_4d(&tq, q, 128, n_q_heads, seqlen, batch, 64, 1, 128, 1) ||
-        make_tmap_4d(&tk, k, 128, n_kv_heads, seqlen, batch, 64, 1, 128, 1) ||
-        make_tmap_4d(&tv, v, 128, n_kv_heads, seqlen, batch, 64, 1, 128, 1))
+        make_tmap_4d(&tk, k, 128, n_kv_heads, seqlen, batch, 64, 1, 64, 1) ||
+        make_tmap_4d(&tv, v, 128, n_kv_heads, seqlen, batch, 64, 1, 64, 1))
       return DA_ERR_CUDA;
     da::PrefillArgs a{};
     a.form = 2;

@@ -9,25 +9,33 @@
 // heads on shared GQA KV heads, full head width, no per-head norm).
 //
 // One CTA computes 128 query rows of one head (V1) or one head pair (V2).
-// Both branches see the same K and V tiles, so each 128-key tile is loaded
+// Both branches see the same K and V tiles, so each 64-key tile is loaded
 // once by TMA for the pair.  Tensor memory (512 columns x 128 lanes fp32):
-//     S1 [0,128)   S2 [128,256)   O1 [256,384)   O2 [384,512)
-// P_r (bf16, 64 columns) overwrites the first half of S_r in place and
-// feeds the P.V MMA directly from tensor memory.  The two branches need
-// separate O accumulators because their running maxima and normalisers
-// differ; the subtraction happens in the epilogue:
+//     S1 [0,64) [64,128)   S2 [128,192) [192,256)   O1 [256,384)   O2 [384,512)
+// Each branch's score tile is double-buffered: while the softmax warps of
+// branch r turn S_r(j) into P_r(j) (bf16, written in place over the first
+// 32 columns of that buffer and fed to the P.V MMA straight from tensor
+// memory), the tensor core already computes S_r(j+1) into the other buffer.
+// The two branches need separate O accumulators because their running
+// maxima and normalisers differ; the subtraction happens in the epilogue:
 //     o = O1 / l1 - lambda * O2 / l2   (then, V1 only, RMS norm * g * (1 - lambda_init)).
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3  softmax for branch 1 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax for branch 2
-//   warp  8    TMA producer (Q once; K and V tiles through 2-stage rings)
-//   warp  9    tcgen05.mma issuer; owns the tensor-memory allocation
+//   warp  8    TMA producer (Q once; K and V tiles through 4-stage rings)
+//   warp  9    issues the Q.K^T MMAs; owns the tensor-memory allocation
+//   warp 10    issues the P.V MMAs
+// Two issuing warps keep the P.V of tile j from queueing behind the wait
+// that guards score buffer reuse (S_r(j+2) may only overwrite the buffer
+// after P_r(j).V has completed).
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
-// Causal masking is applied only on the diagonal tile (and the ragged tail).
-// Every wait is bounded; a timed-out wait records DA_ERR_DEVICE_TIMEOUT in
-// the caller's status word and the CTA unwinds, still freeing its TMEM.
+// Causal masking is applied only on the tiles that cross the diagonal (and
+// the ragged tail).  CTAs are ordered by groups of heads whose K/V fit in L2,
+// heaviest query tiles first within a group.  Every wait is bounded; a
+// timed-out wait records DA_ERR_DEVICE_TIMEOUT in the caller's status word
+// and the CTA unwinds, still freeing its tensor memory.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -41,23 +49,26 @@
 namespace da {
 namespace {
 
-constexpr int kBM = 128;                 // query rows per CTA
-constexpr int kBN = 128;                 // keys per KV tile
-constexpr int kThreads = 320;
-constexpr int kBox = 128 * 64 * 2;       // one TMA box: 128 rows x 64 bf16 = 16 KB
-constexpr int kTileBytes = 2 * kBox;     // a 128 x 128 bf16 tile (two swizzle-atom columns)
-constexpr int kStages = 2;
+constexpr int kBM = 128;                   // query rows per CTA
+constexpr int kBN = 64;                    // keys per KV tile
+constexpr int kThreads = 352;
+constexpr int kQBox = kBM * 64 * 2;        // TMA box of Q: 128 rows x 64 bf16 = 16 KB
+constexpr int kQTile = 2 * kQBox;          // one 128 x 128 query tile
+constexpr int kKVBox = kBN * 64 * 2;       // TMA box of K/V: 64 rows x 64 bf16 = 8 KB
+constexpr int kKVTile = 2 * kKVBox;        // one 64 x 128 key or value tile
+constexpr int kStages = 4;
 constexpr uint32_t kColS1 = 0, kColS2 = 128, kColO1 = 256, kColO2 = 384;
-constexpr float kLazyTau = 8.0f;         // log2 units: rescale only when max grows by > 2^8
+constexpr float kLazyTau = 8.0f;           // log2 units: rescale only when max grows by > 2^8
 
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBN, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
 
 struct Barriers {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t s_full[2][2], p_full[2][2];   // [branch][buffer]
+  uint64_t o_done[2][2];                  // [branch][buffer]: P_r(j).V complete
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -66,6 +77,7 @@ struct Params {
   int form;
   int batch, seqlen, heads, pairs_per_kv;
   int n_qtiles;
+  int group;        // heads (V1) / pairs (V2) scheduled together for L2 reuse
   int causal;
   float scale_log2;
   const float* lambda;
@@ -76,7 +88,9 @@ struct Params {
   int* dev_status;
 };
 
-__device__ __forceinline__ uint32_t q_bytes(int form) { return form == 1 ? kTileBytes : 2 * kTileBytes; }
+__device__ __forceinline__ uint32_t s_col(int r, int buf) {
+  return (r == 0 ? kColS1 : kColS2) + 64u * (uint32_t)buf;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -85,26 +99,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t qb = q_bytes(p.form);
+  const uint32_t qbytes = p.form == 1 ? kQTile : 2 * kQTile;
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + qb;                            // kStages x kTileBytes
-  uint8_t* sV = sK + kStages * kTileBytes;            // kStages x kTileBytes
-  Barriers* bars = reinterpret_cast<Barriers*>(sV + kStages * kTileBytes);
+  uint8_t* sK = smem + qbytes;                         // kStages x kKVTile
+  uint8_t* sV = sK + kStages * kKVTile;                // kStages x kKVTile
+  Barriers* bars = reinterpret_cast<Barriers*>(sV + kStages * kKVTile);
   float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [2][128]
   float* x_ss = x_inv_l + 2 * kBM;                       // [2][128]
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
 
-  // ---- tile coordinates: heaviest (latest) query tiles first ----
+  // ---- tile coordinates: groups of heads, heaviest query tiles first ----
   const int bh_count = p.batch * p.heads;
-  const int mt = p.n_qtiles - 1 - (int)(blockIdx.x / bh_count);
-  const int bh = (int)(blockIdx.x % bh_count);
+  const int per_group = p.group * p.n_qtiles;
+  const int g = (int)(blockIdx.x / per_group);
+  const int rr = (int)(blockIdx.x % per_group);
+  const int g_size = min(p.group, bh_count - g * p.group);
+  const int mt = p.n_qtiles - 1 - rr / g_size;
+  const int bh = g * p.group + rr % g_size;
   const int hh = bh % p.heads;          // V1 head or V2 pair
   const int b = bh / p.heads;
   const int kvh = p.form == 1 ? hh : hh / p.pairs_per_kv;
   const int q0 = mt * kBM;
-  const int n_kv = p.causal ? mt + 1 : (p.seqlen + kBN - 1) / kBN;
+  const int key_end = p.causal ? min(q0 + kBM, p.seqlen) : p.seqlen;  // keys this tile needs
+  const int n_kv = (key_end + kBN - 1) / kBN;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -115,9 +134,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_empty[s], 1);
     }
     for (int r = 0; r < 2; ++r) {
-      mbar_init(&bars->s_full[r], 1);
-      mbar_init(&bars->p_full[r], 128);
-      mbar_init(&bars->o_done[r], 1);
+      for (int u = 0; u < 2; ++u) {
+        mbar_init(&bars->s_full[r][u], 1);
+        mbar_init(&bars->p_full[r][u], 128);
+        mbar_init(&bars->o_done[r][u], 1);
+      }
     }
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -138,81 +159,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, qb);
+      mbar_arrive_expect_tx(&bars->q_full, qbytes);
       if (p.form == 1) {
         tma_load_4d(sQ, &tm_q, &bars->q_full, 0, hh, q0, b);
-        tma_load_4d(sQ + kBox, &tm_q, &bars->q_full, 64, hh, q0, b);
+        tma_load_4d(sQ + kQBox, &tm_q, &bars->q_full, 64, hh, q0, b);
       } else {
         tma_load_4d(sQ, &tm_q, &bars->q_full, 0, 2 * hh, q0, b);
-        tma_load_4d(sQ + kBox, &tm_q, &bars->q_full, 64, 2 * hh, q0, b);
-        tma_load_4d(sQ + 2 * kBox, &tm_q, &bars->q_full, 0, 2 * hh + 1, q0, b);
-        tma_load_4d(sQ + 3 * kBox, &tm_q, &bars->q_full, 64, 2 * hh + 1, q0, b);
+        tma_load_4d(sQ + kQBox, &tm_q, &bars->q_full, 64, 2 * hh, q0, b);
+        tma_load_4d(sQ + 2 * kQBox, &tm_q, &bars->q_full, 0, 2 * hh + 1, q0, b);
+        tma_load_4d(sQ + 3 * kQBox, &tm_q, &bars->q_full, 64, 2 * hh + 1, q0, b);
       }
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kStages;
         const uint32_t ph = (uint32_t)(j / kStages) & 1u;
         if (!mbar_wait(&bars->k_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
-        mbar_arrive_expect_tx(&bars->k_full[s], kTileBytes);
-        tma_load_4d(sK + s * kTileBytes, &tm_k, &bars->k_full[s], 0, kvh, j * kBN, b);
-        tma_load_4d(sK + s * kTileBytes + kBox, &tm_k, &bars->k_full[s], 64, kvh, j * kBN, b);
+        mbar_arrive_expect_tx(&bars->k_full[s], kKVTile);
+        tma_load_4d(sK + s * kKVTile, &tm_k, &bars->k_full[s], 0, kvh, j * kBN, b);
+        tma_load_4d(sK + s * kKVTile + kKVBox, &tm_k, &bars->k_full[s], 64, kvh, j * kBN, b);
         if (!mbar_wait(&bars->v_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
-        mbar_arrive_expect_tx(&bars->v_full[s], kTileBytes);
-        tma_load_4d(sV + s * kTileBytes, &tm_v, &bars->v_full[s], 0, kvh, j * kBN, b);
-        tma_load_4d(sV + s * kTileBytes + kBox, &tm_v, &bars->v_full[s], 64, kvh, j * kBN, b);
+        mbar_arrive_expect_tx(&bars->v_full[s], kKVTile);
+        tma_load_4d(sV + s * kKVTile, &tm_v, &bars->v_full[s], 0, kvh, j * kBN, b);
+        tma_load_4d(sV + s * kKVTile + kKVBox, &tm_v, &bars->v_full[s], 64, kvh, j * kBN, b);
       }
     }
   } else if (warp == 9) {
-    // ------------------------------ MMA issuer -----------------------------
+    // ------------------------- Q.K^T issuer ---------------------------------
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
-      const uint32_t v_addr = smem_u32(sV);
       const int nk = p.form == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T per branch
       if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
-        for (int j = 0; j < n_kv; ++j) {
+        for (int j = 0; j < n_kv && !failed; ++j) {
           const int s = j % kStages;
-          const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-          if (!mbar_wait(&bars->k_full[s], ph, p.dev_status, &failed)) break;
-          const uint32_t kt = k_addr + s * kTileBytes;
+          if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status,
+                         &failed))
+            break;
+          const uint32_t kt = k_addr + s * kKVTile;
           for (int r = 0; r < 2; ++r) {
-            // S_r aliases P_r of the previous tile: wait until P_r(j-1).V is done
-            if (j > 0 && !mbar_wait(&bars->o_done[r], (uint32_t)(j - 1) & 1u, p.dev_status,
-                                    &failed))
+            // buffer j % 2 last held P_r(j-2): its P.V must have completed
+            if (j >= 2 && !mbar_wait(&bars->o_done[r][j & 1], (uint32_t)((j - 2) >> 1) & 1u,
+                                     p.dev_status, &failed))
               break;
             tc_fence_after();
             for (int kk = 0; kk < nk; ++kk) {
               uint32_t a, bb;
               if (p.form == 1) {  // branch r = columns [64 r, 64 r + 64)
-                a = q_addr + r * kBox + kk * 32;
-                bb = kt + r * kBox + kk * 32;
+                a = q_addr + r * kQBox + kk * 32;
+                bb = kt + r * kKVBox + kk * 32;
               } else {            // branch r = query head 2p + r, full 128 columns
-                a = q_addr + r * kTileBytes + (kk >> 2) * kBox + (kk & 3) * 32;
-                bb = kt + (kk >> 2) * kBox + (kk & 3) * 32;
+                a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
+                bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
               }
-              tc_mma_ss(tmem + (r == 0 ? kColS1 : kColS2), smem_desc_sw128(a, 16, 1024),
+              tc_mma_ss(tmem + s_col(r, j & 1), smem_desc_sw128(a, 16, 1024),
                         smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
             }
-            tc_commit(&bars->s_full[r]);
+            tc_commit(&bars->s_full[r][j & 1]);
           }
           if (failed) break;
           tc_commit(&bars->k_empty[s]);
-          if (!mbar_wait(&bars->v_full[s], ph, p.dev_status, &failed)) break;
-          const uint32_t vt = v_addr + s * kTileBytes;
-          for (int r = 0; r < 2; ++r) {
-            if (!mbar_wait(&bars->p_full[r], (uint32_t)j & 1u, p.dev_status, &failed)) break;
-            tc_fence_after();
-            const uint32_t pcol = tmem + (r == 0 ? kColS1 : kColS2);
-            const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              // B = V tile, MN-major: 64-column halves kBox apart, 8-key groups 1 KB apart
-              tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kBox, 1024),
-                        kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc_commit(&bars->o_done[r]);
-          }
-          if (failed) break;
-          tc_commit(&bars->v_empty[s]);
         }
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------- P.V issuer -----------------------------------
+    if (lane == 0) {
+      const uint32_t v_addr = smem_u32(sV);
+      for (int j = 0; j < n_kv && !failed; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait(&bars->v_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
+          break;
+        const uint32_t vt = v_addr + s * kKVTile;
+        for (int r = 0; r < 2; ++r) {
+          if (!mbar_wait(&bars->p_full[r][j & 1], (uint32_t)(j >> 1) & 1u, p.dev_status,
+                         &failed))
+            break;
+          tc_fence_after();
+          const uint32_t pcol = tmem + s_col(r, j & 1);
+          const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
+            tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
+                      kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&bars->o_done[r][j & 1]);
+        }
+        if (failed) break;
+        tc_commit(&bars->v_empty[s]);
       }
     }
   } else {
@@ -222,28 +254,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = sub * 32 + lane;         // query row within the tile
     const int qrow = q0 + row;               // query row within the sequence
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + (r == 0 ? kColS1 : kColS2);
     const uint32_t t_o = tmem + lane_off + (r == 0 ? kColO1 : kColO2);
+    const int lim = p.causal ? min(qrow + 1, p.seqlen) : p.seqlen;  // keys < lim visible
+    const float sc = p.scale_log2;
     float m_ref = -INFINITY, l_run = 0.f;
 
     for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait(&bars->s_full[r], (uint32_t)j & 1u, p.dev_status, &failed)) break;
+      const int buf = j & 1;
+      if (!mbar_wait(&bars->s_full[r][buf], (uint32_t)(j >> 1) & 1u, p.dev_status, &failed))
+        break;
       tc_fence_after();
-      uint32_t sr[128];  // raw S row (masked entries set to -inf)
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(t_s + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
+      const uint32_t t_s = tmem + lane_off + s_col(r, buf);
+      uint32_t sr[64];  // raw S row of this tile (masked entries set to -inf)
+      tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
       tc_wait_ld();
       const int k0 = j * kBN;
-      const bool need_mask = (p.causal && j == mt) || (k0 + kBN > p.seqlen);
-      const int lim = p.causal ? min(qrow + 1, p.seqlen) : p.seqlen;  // keys < lim visible
-      float mx = -INFINITY;
+      if (k0 + kBN > lim) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        if (need_mask && k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
-        mx = fmaxf(mx, __uint_as_float(sr[c]));
+        for (int c = 0; c < 64; ++c)
+          if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
       }
-      mx *= p.scale_log2;  // the scale is positive, so it commutes with max
+      float m8[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) m8[c] = __uint_as_float(sr[c]);
+#pragma unroll
+      for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sr[c]));
+      const float mx =
+          fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sc;  // sc > 0 commutes
       float alpha = 1.f;
       bool resc = false;
       if (j == 0) {
@@ -257,15 +296,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const float u = m_ref == -INFINITY ? 0.f : m_ref;
-      float rowsum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int qt = 0; qt < 4; ++qt) {  // 32 logits -> 16 packed bf16 pairs per store
+      for (int qt = 0; qt < 2; ++qt) {  // 32 logits -> 16 packed bf16 pairs per store
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e]), p.scale_log2, -u));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e + 1]), p.scale_log2, -u));
-          rowsum += p0 + p1;
+          const float p0 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e]), sc, -u));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e + 1]), sc, -u));
+          ps[e & 3] += p0 + p1;
           pk[e] = pack_bf16(p0, p1);
         }
         tmem_st16(t_s + 16 * qt, pk);
@@ -273,7 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__any_sync(0xffffffffu, resc)) {
         // O_r must be quiescent (the previous tile's P.V into O_r done) before
         // it is rescaled in place; rows that keep their reference use alpha 1.
-        if (!mbar_wait(&bars->o_done[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed)) break;
+        if (!mbar_wait(&bars->o_done[r][(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u,
+                       p.dev_status, &failed))
+          break;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -285,21 +326,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(t_o + 16 * c, ov);
         }
       }
-      l_run = l_run * alpha + rowsum;
+      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[r]);
+      mbar_arrive(&bars->p_full[r][buf]);
     }
 
     // ---- epilogue: o = O1/l1 - lambda O2/l2 (+ V1 norm), channels [64 r, 64 r + 64) ----
     __syncwarp();
     if (failed) bars->abort_flag = 1;
-    const uint32_t last = (uint32_t)(n_kv - 1) & 1u;
-    mbar_wait(&bars->o_done[r], last, p.dev_status, &failed);
-    mbar_wait(&bars->o_done[r ^ 1], last, p.dev_status, &failed);
+    // own branch's last P.V done; the named barrier then orders both branches
+    mbar_wait(&bars->o_done[r][(n_kv - 1) & 1], (uint32_t)((n_kv - 1) >> 1) & 1u, p.dev_status,
+              &failed);
     tc_fence_after();
     x_inv_l[r * kBM + row] = 1.0f / l_run;
     asm volatile("bar.sync 2, 256;" ::: "memory");
+    tc_fence_after();
     const float inv1 = x_inv_l[row];
     const float inv2 = x_inv_l[kBM + row] * p.lambda[hh];
     float o[64];
@@ -317,10 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float mul = 1.f;
     if (p.apply_norm) {
-      float ss = 0.f;
+      float ss4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < 64; ++e) ss = fmaf(o[e], o[e], ss);
-      x_ss[r * kBM + row] = ss;
+      for (int e = 0; e < 64; ++e) ss4[e & 3] = fmaf(o[e], o[e], ss4[e & 3]);
+      x_ss[r * kBM + row] = (ss4[0] + ss4[1]) + (ss4[2] + ss4[3]);
       asm volatile("bar.sync 2, 256;" ::: "memory");
       const float tot = x_ss[row] + x_ss[kBM + row];
       mul = p.post_scale / sqrtf(tot * (1.0f / 128.0f) + p.eps);
@@ -334,8 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int c = v8 * 8 + e;
-          const float g = (p.apply_norm && p.norm_weight) ? __ldg(p.norm_weight + 64 * r + c) : 1.f;
-          y[e] = o[c] * mul * g;
+          const float gm = (p.apply_norm && p.norm_weight) ? __ldg(p.norm_weight + 64 * r + c)
+                                                           : 1.f;
+          y[e] = o[c] * mul * gm;
         }
         uint4 w;
         w.x = pack_bf16(y[0], y[1]);
@@ -370,6 +413,13 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.heads = a.heads;
   p.pairs_per_kv = a.pairs_per_kv;
   p.n_qtiles = (a.seqlen + kBM - 1) / kBM;
+  // Heads (V1) or pairs (V2) scheduled together: as many as keep their K and
+  // V (2 x seqlen x 128 bf16 per KV head) within about half of the L2.
+  const double kv_bytes = 2.0 * a.seqlen * 128 * 2;
+  const int bh_count = a.batch * a.heads;
+  int grp = (int)((64.0 * 1024 * 1024) / kv_bytes) * a.pairs_per_kv;
+  grp = grp < a.pairs_per_kv ? a.pairs_per_kv : grp;
+  p.group = grp > bh_count ? bh_count : grp;
   p.causal = a.causal;
   const double d = a.form == 1 ? 64.0 : 128.0;  // width of one branch's query
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(d));
@@ -380,13 +430,13 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.post_scale = a.post_scale;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.dev_status = a.dev_status;
-  const int qbytes = a.form == 1 ? kTileBytes : 2 * kTileBytes;
-  const int smem = 1024 + qbytes + 2 * kStages * kTileBytes + (int)sizeof(Barriers) +
+  const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
+  const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +
                    4 * kBM * (int)sizeof(float) + 64;
   cudaError_t e = cudaFuncSetAttribute(diffattn_prefill_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const long long grid = (long long)p.n_qtiles * a.batch * a.heads;
+  const long long grid = (long long)p.n_qtiles * bh_count;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   diffattn_prefill_tc_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
   return cudaGetLastError();
