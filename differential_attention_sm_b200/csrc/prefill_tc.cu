@@ -24,11 +24,12 @@
 //   warps 0-3  softmax for branch 1 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax for branch 2
 //   warp  8    TMA producer (Q once; K and V tiles through 4-stage rings)
-//   warp  9    issues the Q.K^T MMAs; owns the tensor-memory allocation
-//   warp 10    issues the P.V MMAs
-// Two issuing warps keep the P.V of tile j from queueing behind the wait
-// that guards score buffer reuse (S_r(j+2) may only overwrite the buffer
-// after P_r(j).V has completed).
+//   warp  9    issues branch 1's MMAs (Q1.K^T, P1.V); owns the tensor memory
+//   warp 10    issues branch 2's MMAs (Q2.K^T, P2.V)
+// tcgen05.mma issue runs at the tensor pipe's pace, so one issuing warp per
+// branch keeps each branch's chain (P_r(j).V, then S_r(j+2) into the buffer
+// it frees) from waiting behind the other branch's order of work.
+// Per branch the issue order is S_r(j+1), then P_r(j).V.
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
 // Causal masking is applied only on the tiles that cross the diagonal (and
@@ -129,9 +130,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->k_empty[s], 2);   // released by both branches' MMAs
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 2);
     }
     for (int r = 0; r < 2; ++r) {
       for (int u = 0; u < 2; ++u) {
@@ -182,69 +183,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sV + s * kKVTile + kKVBox, &tm_v, &bars->v_full[s], 64, kvh, j * kBN, b);
       }
     }
-  } else if (warp == 9) {
-    // ------------------------- Q.K^T issuer ---------------------------------
+  } else if (warp == 9 || warp == 10) {
+    // ------------------- MMA issuer of branch r = warp - 9 -------------------
     if (lane == 0) {
+      const int r = warp - 9;
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
-      const int nk = p.form == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T per branch
-      if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
-        for (int j = 0; j < n_kv && !failed; ++j) {
+      const uint32_t v_addr = smem_u32(sV);
+      const int nk = p.form == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T
+      // S_r(j) = Q_r . K(j)^T into buffer j % 2 of branch r.
+      auto issue_scores = [&](int j) -> bool {
+        const int s = j % kStages;
+        if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
+          return false;
+        // buffer j % 2 last held P_r(j-2): its P.V must have completed
+        if (j >= 2 && !mbar_wait(&bars->o_done[r][j & 1], (uint32_t)((j - 2) >> 1) & 1u,
+                                 p.dev_status, &failed))
+          return false;
+        tc_fence_after();
+        const uint32_t kt = k_addr + s * kKVTile;
+        for (int kk = 0; kk < nk; ++kk) {
+          uint32_t a, bb;
+          if (p.form == 1) {  // branch r = columns [64 r, 64 r + 64)
+            a = q_addr + r * kQBox + kk * 32;
+            bb = kt + r * kKVBox + kk * 32;
+          } else {            // branch r = query head 2p + r, full 128 columns
+            a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
+            bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
+          }
+          tc_mma_ss(tmem + s_col(r, j & 1), smem_desc_sw128(a, 16, 1024),
+                    smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars->s_full[r][j & 1]);
+        tc_commit(&bars->k_empty[s]);
+        return true;
+      };
+      if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed) && issue_scores(0)) {
+        const uint32_t pcol0 = tmem + s_col(r, 0);
+        const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
+        for (int j = 0; j < n_kv; ++j) {
+          if (j + 1 < n_kv && !issue_scores(j + 1)) break;
           const int s = j % kStages;
-          if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status,
+          if (!mbar_wait(&bars->v_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status,
                          &failed))
             break;
-          const uint32_t kt = k_addr + s * kKVTile;
-          for (int r = 0; r < 2; ++r) {
-            // buffer j % 2 last held P_r(j-2): its P.V must have completed
-            if (j >= 2 && !mbar_wait(&bars->o_done[r][j & 1], (uint32_t)((j - 2) >> 1) & 1u,
-                                     p.dev_status, &failed))
-              break;
-            tc_fence_after();
-            for (int kk = 0; kk < nk; ++kk) {
-              uint32_t a, bb;
-              if (p.form == 1) {  // branch r = columns [64 r, 64 r + 64)
-                a = q_addr + r * kQBox + kk * 32;
-                bb = kt + r * kKVBox + kk * 32;
-              } else {            // branch r = query head 2p + r, full 128 columns
-                a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
-                bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
-              }
-              tc_mma_ss(tmem + s_col(r, j & 1), smem_desc_sw128(a, 16, 1024),
-                        smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(&bars->s_full[r][j & 1]);
-          }
-          if (failed) break;
-          tc_commit(&bars->k_empty[s]);
-        }
-      }
-    }
-  } else if (warp == 10) {
-    // ------------------------- P.V issuer -----------------------------------
-    if (lane == 0) {
-      const uint32_t v_addr = smem_u32(sV);
-      for (int j = 0; j < n_kv && !failed; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(&bars->v_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
-          break;
-        const uint32_t vt = v_addr + s * kKVTile;
-        for (int r = 0; r < 2; ++r) {
           if (!mbar_wait(&bars->p_full[r][j & 1], (uint32_t)(j >> 1) & 1u, p.dev_status,
                          &failed))
             break;
           tc_fence_after();
-          const uint32_t pcol = tmem + s_col(r, j & 1);
-          const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
+          const uint32_t vt = v_addr + s * kKVTile;
+          const uint32_t pcol = pcol0 + 64u * (uint32_t)(j & 1);
           for (int kk = 0; kk < kBN / 16; ++kk) {
             // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
             tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
                       kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&bars->o_done[r][j & 1]);
+          tc_commit(&bars->v_empty[s]);
         }
-        if (failed) break;
-        tc_commit(&bars->v_empty[s]);
       }
     }
   } else {
@@ -275,14 +271,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 64; ++c)
           if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
       }
+      // row maximum: 3-input max over 8 independent chains
       float m8[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) m8[c] = __uint_as_float(sr[c]);
-#pragma unroll
-      for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sr[c]));
-      const float mx =
-          fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sc;  // sc > 0 commutes
+      for (int i = 0; i < 8; ++i) {
+        float m = max3(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]),
+                       __uint_as_float(sr[16 + i]));
+        m = max3(m, __uint_as_float(sr[24 + i]), __uint_as_float(sr[32 + i]));
+        m = max3(m, __uint_as_float(sr[40 + i]), __uint_as_float(sr[48 + i]));
+        m8[i] = fmaxf(m, __uint_as_float(sr[56 + i]));
+      }
+      const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
+                            fmaxf(m8[6], m8[7])) * sc;  // sc > 0 commutes with max
       float alpha = 1.f;
       bool resc = false;
       if (j == 0) {
@@ -296,19 +296,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const float u = m_ref == -INFINITY ? 0.f : m_ref;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      // p = 2^(s*sc - u): pairs on the f32x2 pipe; one pair in four takes the
+      // polynomial 2^x, the rest the multi-function unit.
+      const uint64_t sc2 = f2pack(sc, sc), nu2 = f2pack(-u, -u);
+      uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int qt = 0; qt < 2; ++qt) {  // 32 logits -> 16 packed bf16 pairs per store
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e]), sc, -u));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[qt * 32 + 2 * e + 1]), sc, -u));
-          ps[e & 3] += p0 + p1;
+          const int c = qt * 32 + 2 * e;
+          const uint64_t x2 = fma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                   sc2, nu2);
+          float x0, x1, p0, p1;
+          f2unpack(x2, x0, x1);
+          if ((e & 3) == 3) {
+            exp2_poly2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          ps2[e & 3] = add2(ps2[e & 3], f2pack(p0, p1));
           pk[e] = pack_bf16(p0, p1);
         }
         tmem_st16(t_s + 16 * qt, pk);
       }
+      float psum, psum_hi;
+      f2unpack(add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3])), psum, psum_hi);
+      psum += psum_hi;
       if (__any_sync(0xffffffffu, resc)) {
         // O_r must be quiescent (the previous tile's P.V into O_r done) before
         // it is rescaled in place; rows that keep their reference use alpha 1.
@@ -326,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(t_o + 16 * c, ov);
         }
       }
-      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      l_run = l_run * alpha + psum;
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[r][buf]);

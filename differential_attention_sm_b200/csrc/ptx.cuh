@@ -50,6 +50,59 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// 3-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pairs (.b64 register holding {lo, hi}) for the f32x2 pipe ops.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair on the FMA/ALU pipes instead of the multi-function unit:
+// n = round(x) via the 1.5*2^23 shifter, f = x - n in [-1/2, 1/2], 2^f from a
+// relative-minimax cubic (coefficients fitted by csrc/exp2_poly.py, max
+// relative error 7.5e-5), 2^n added into the exponent field.  x is clamped at
+// -126 (results below 2^-126 are negligible next to the row's terms).
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t xv = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = add2(xv, f2pack(kShift, kShift));
+  const uint64_t r = add2(t, f2pack(-kShift, -kShift));                // round(x)
+  const uint64_t f = fma2(r, f2pack(-1.0f, -1.0f), xv);                // x - round(x)
+  uint64_t q = fma2(f2pack(kExp2C3, kExp2C3), f, f2pack(kExp2C2, kExp2C2));
+  q = fma2(q, f, f2pack(kExp2C1, kExp2C1));
+  q = fma2(q, f, f2pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  // (bits(t) - bits(1.5*2^23)) << 23 == bits(t) << 23 modulo 2^32
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 // Record a device-side failure (first writer wins) if a status word exists.
 __device__ __forceinline__ void report(int* dev_status, int code) {
   if (dev_status) atomicCAS(dev_status, 0, code);
