@@ -20,16 +20,19 @@
 // maxima and normalisers differ; the subtraction happens in the epilogue:
 //     o = O1 / l1 - lambda * O2 / l2   (then, V1 only, RMS norm * g * (1 - lambda_init)).
 //
-// Warp roles (352 threads):
+// Warp roles (416 threads):
 //   warps 0-3  softmax for branch 1 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax for branch 2
 //   warp  8    TMA producer (Q once; K and V tiles through 4-stage rings)
-//   warp  9    issues branch 1's MMAs (Q1.K^T, P1.V); owns the tensor memory
-//   warp 10    issues branch 2's MMAs (Q2.K^T, P2.V)
-// tcgen05.mma issue runs at the tensor pipe's pace, so one issuing warp per
-// branch keeps each branch's chain (P_r(j).V, then S_r(j+2) into the buffer
-// it frees) from waiting behind the other branch's order of work.
-// Per branch the issue order is S_r(j+1), then P_r(j).V.
+//   warp  9    issues branch 1's score MMAs (Q1.K^T); owns the tensor memory
+//   warp 10    issues branch 2's score MMAs (Q2.K^T)
+//   warp 11    issues branch 1's P1.V MMAs
+//   warp 12    issues branch 2's P2.V MMAs
+// tcgen05.mma issue runs at the tensor pipe's pace and every commit and
+// barrier poll costs the issuing thread time, so each of the four MMA
+// streams has its own thread: P_r(j).V goes out as soon as P_r(j) is ready,
+// and S_r(j+2) as soon as that P.V has freed its buffer, without either
+// waiting behind the other's bookkeeping.
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
 // Causal masking is applied only on the tiles that cross the diagonal (and
@@ -52,7 +55,7 @@ namespace {
 
 constexpr int kBM = 128;                   // query rows per CTA
 constexpr int kBN = 64;                    // keys per KV tile
-constexpr int kThreads = 352;
+constexpr int kThreads = 416;
 constexpr int kQBox = kBM * 64 * 2;        // TMA box of Q: 128 rows x 64 bf16 = 16 KB
 constexpr int kQTile = 2 * kQBox;          // one 128 x 128 query tile
 constexpr int kKVBox = kBN * 64 * 2;       // TMA box of K/V: 64 rows x 64 bf16 = 8 KB
@@ -184,63 +187,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 9 || warp == 10) {
-    // ------------------- MMA issuer of branch r = warp - 9 -------------------
+    // ------------- score MMA issuer of branch r = warp - 9: S_r(j) = Q_r . K(j)^T -------------
     if (lane == 0) {
       const int r = warp - 9;
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
-      const uint32_t v_addr = smem_u32(sV);
       const int nk = p.form == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T
-      // S_r(j) = Q_r . K(j)^T into buffer j % 2 of branch r.
-      auto issue_scores = [&](int j) -> bool {
-        const int s = j % kStages;
-        if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
-          return false;
-        // buffer j % 2 last held P_r(j-2): its P.V must have completed
-        if (j >= 2 && !mbar_wait(&bars->o_done[r][j & 1], (uint32_t)((j - 2) >> 1) & 1u,
-                                 p.dev_status, &failed))
-          return false;
-        tc_fence_after();
-        const uint32_t kt = k_addr + s * kKVTile;
-        for (int kk = 0; kk < nk; ++kk) {
-          uint32_t a, bb;
-          if (p.form == 1) {  // branch r = columns [64 r, 64 r + 64)
-            a = q_addr + r * kQBox + kk * 32;
-            bb = kt + r * kKVBox + kk * 32;
-          } else {            // branch r = query head 2p + r, full 128 columns
-            a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
-            bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
-          }
-          tc_mma_ss(tmem + s_col(r, j & 1), smem_desc_sw128(a, 16, 1024),
-                    smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars->s_full[r][j & 1]);
-        tc_commit(&bars->k_empty[s]);
-        return true;
-      };
-      if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed) && issue_scores(0)) {
-        const uint32_t pcol0 = tmem + s_col(r, 0);
-        const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
+      if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
         for (int j = 0; j < n_kv; ++j) {
-          if (j + 1 < n_kv && !issue_scores(j + 1)) break;
           const int s = j % kStages;
-          if (!mbar_wait(&bars->v_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status,
-                         &failed))
+          if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
             break;
-          if (!mbar_wait(&bars->p_full[r][j & 1], (uint32_t)(j >> 1) & 1u, p.dev_status,
-                         &failed))
+          // buffer j % 2 last held P_r(j-2): its P.V must have completed
+          if (j >= 2 && !mbar_wait(&bars->o_done[r][j & 1], (uint32_t)((j - 2) >> 1) & 1u,
+                                   p.dev_status, &failed))
             break;
           tc_fence_after();
-          const uint32_t vt = v_addr + s * kKVTile;
-          const uint32_t pcol = pcol0 + 64u * (uint32_t)(j & 1);
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
-            tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
-                      kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t kt = k_addr + s * kKVTile;
+          for (int kk = 0; kk < nk; ++kk) {
+            uint32_t a, bb;
+            if (p.form == 1) {  // branch r = columns [64 r, 64 r + 64)
+              a = q_addr + r * kQBox + kk * 32;
+              bb = kt + r * kKVBox + kk * 32;
+            } else {            // branch r = query head 2p + r, full 128 columns
+              a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
+              bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
+            }
+            tc_mma_ss(tmem + s_col(r, j & 1), smem_desc_sw128(a, 16, 1024),
+                      smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
           }
-          tc_commit(&bars->o_done[r][j & 1]);
-          tc_commit(&bars->v_empty[s]);
+          tc_commit(&bars->s_full[r][j & 1]);
+          tc_commit(&bars->k_empty[s]);
         }
+      }
+    }
+  } else if (warp == 11 || warp == 12) {
+    // ------------- P.V MMA issuer of branch r = warp - 11: O_r += P_r(j) . V(j) -------------
+    if (lane == 0) {
+      const int r = warp - 11;
+      const uint32_t v_addr = smem_u32(sV);
+      const uint32_t pcol0 = tmem + s_col(r, 0);
+      const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait(&bars->v_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
+          break;
+        if (!mbar_wait(&bars->p_full[r][j & 1], (uint32_t)(j >> 1) & 1u, p.dev_status,
+                       &failed))
+          break;
+        tc_fence_after();
+        const uint32_t vt = v_addr + s * kKVTile;
+        const uint32_t pcol = pcol0 + 64u * (uint32_t)(j & 1);
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
+          tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
+                    kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars->o_done[r][j & 1]);
+        tc_commit(&bars->v_empty[s]);
       }
     }
   } else {

@@ -156,3 +156,16 @@ def test_v1_decode_full_size_sampled(B):
         assert_bf16_close(out[b], ref, False, "v1 decode full b=%d" % b)
     del kc, vc
     torch.cuda.empty_cache()
+
+
+def test_v2_decode_large_logits_and_negative_lambda(B):
+    Bn, L, Hq, Hkv, d = 2, 3000, 16, 2, 128
+    x = I.v2_decode_inputs(Bn, L, Hq, Hkv, d, seed=35, dtype=torch.float32)
+    ramp = torch.linspace(0.1, 1.0, L).view(1, L, 1, 1)
+    q = (5.0 * x["q"]).to(torch.bfloat16)
+    kc = (x["k_cache"] * ramp).to(torch.bfloat16)
+    vc = x["v_cache"].to(torch.bfloat16)
+    lam = torch.linspace(-1.0, 1.5, Hq // 2)
+    out = B.diffattn_v2_decode(cuda(q), cuda(kc), cuda(vc), cuda(lam))
+    ref = O.v2_decode_rows(q, kc, vc, lam.double().numpy(), np.arange(Bn * Hq // 2))
+    assert_bf16_close(out.reshape(-1, d), ref, True, "v2 decode large logits")

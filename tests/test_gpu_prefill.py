@@ -76,7 +76,7 @@ def test_lambda_from_params_matches_oracle(B):
     (1, 1, 2, True),      # single token
     (2, 129, 1, True),    # one row past a tile edge
     (1, 200, 2, False),   # non-causal, ragged key tail
-    (1, 640, 1, True),    # five tiles: exercises the 2-stage rings' reuse
+    (1, 640, 1, True),    # ten key tiles: every K/V ring stage is reused
 ])
 def test_v1_bf16_small(B, Bn, N, H, causal):
     d, dv, layer = 64, 128, 12
@@ -199,3 +199,53 @@ def test_v2_full_size_sampled(B):
     ref = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], rows, causal=True)
     got = out.reshape(-1, w.d)[torch.from_numpy(rows).cuda()]
     assert_bf16_close(got, ref, True, "v2 full")
+
+
+# ---------------------------------------------------------------------------
+# harder numerics: lambda outside [0, 1], large logits (many lazy rescales)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("lam_values", [(-0.6, 1.4, 0.0), (2.5, -1.2, 0.9)])
+def test_v1_bf16_extreme_lambda(B, lam_values):
+    Bn, N, H, d, dv = 1, 384, 3, 64, 128
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=31, dtype=torch.bfloat16)
+    lam = torch.tensor(lam_values, dtype=torch.float32)
+    out = B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(lam), causal=True,
+                            apply_norm=True, lambda_init=0.3)
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam.double().numpy(), np.arange(Bn * N * H),
+                    causal=True, apply_norm=True, lambda_init_value=0.3)
+    assert_bf16_close(out.reshape(-1, dv), ref, False, "v1 extreme lambda")
+
+
+def test_v2_bf16_extreme_lambda(B):
+    Bn, N, Hq, Hkv, d = 1, 300, 4, 1, 128
+    x = I.v2_inputs(Bn, N, Hq, Hkv, d, seed=32)
+    lam = torch.tensor([-0.75, 1.6], dtype=torch.float32)
+    out = B.diffattn_v2_prefill(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(lam), causal=True)
+    ref = O.v2_rows(x["q"], x["k"], x["v"], lam.double().numpy(), np.arange(Bn * N * 2),
+                    causal=True)
+    assert_bf16_close(out.reshape(-1, d), ref, True, "v2 extreme lambda")
+
+
+@pytest.mark.parametrize("scale", [3.0, 6.0])
+def test_large_logits_rescale_paths(B, scale):
+    """Queries scaled up so that row maxima jump by far more than the lazy
+    rescale threshold across key tiles (and exponents span a wide range)."""
+    Bn, N, H, d, dv = 1, 700, 2, 64, 128
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=33, dtype=torch.float32)
+    ramp = torch.linspace(0.2, 1.0, N).view(1, N, 1, 1)   # later keys grow: maxima keep rising
+    q = (scale * x["q"]).to(torch.bfloat16)
+    k = (x["k"] * ramp).to(torch.bfloat16)
+    v = x["v"].to(torch.bfloat16)
+    lam = torch.tensor([0.7, 0.4], dtype=torch.float32)
+    out = B.diffattn_v1_fwd(cuda(q), cuda(k), cuda(v), cuda(lam), causal=True, apply_norm=True,
+                            lambda_init=0.2)
+    ref = O.v1_rows(q, k, v, lam.double().numpy(), np.arange(Bn * N * H), causal=True,
+                    apply_norm=True, lambda_init_value=0.2)
+    assert_bf16_close(out.reshape(-1, dv), ref, False, "v1 large logits x%g" % scale)
+    x2 = I.v2_inputs(1, N, 4, 2, 128, seed=34, dtype=torch.float32)
+    q2 = (scale * x2["q"]).to(torch.bfloat16)
+    k2 = (x2["k"] * ramp).to(torch.bfloat16)
+    v2 = x2["v"].to(torch.bfloat16)
+    out2 = B.diffattn_v2_prefill(cuda(q2), cuda(k2), cuda(v2), cuda(x2["lam"]), causal=True)
+    ref2 = O.v2_rows(q2, k2, v2, x2["lam"], np.arange(N * 2), causal=True)
+    assert_bf16_close(out2.reshape(-1, 128), ref2, True, "v2 large logits x%g" % scale)
