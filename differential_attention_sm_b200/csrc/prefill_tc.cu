@@ -96,6 +96,8 @@ __device__ __forceinline__ uint32_t s_col(int r, int buf) {
   return (r == 0 ? kColS1 : kColS2) + 64u * (uint32_t)buf;
 }
 
+// kForm: 1 = V1 (d_qk 64 per branch, one head), 2 = V2 (d 128 per branch, a head pair).
+template <int kForm>
 __global__ void __launch_bounds__(kThreads, 1)
     diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t qbytes = p.form == 1 ? kQTile : 2 * kQTile;
+  const uint32_t qbytes = kForm == 1 ? kQTile : 2 * kQTile;
   uint8_t* sQ = smem;
   uint8_t* sK = smem + qbytes;                         // kStages x kKVTile
   uint8_t* sV = sK + kStages * kKVTile;                // kStages x kKVTile
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = g * p.group + rr % g_size;
   const int hh = bh % p.heads;          // V1 head or V2 pair
   const int b = bh / p.heads;
-  const int kvh = p.form == 1 ? hh : hh / p.pairs_per_kv;
+  const int kvh = kForm == 1 ? hh : hh / p.pairs_per_kv;
   const int q0 = mt * kBM;
   const int key_end = p.causal ? min(q0 + kBM, p.seqlen) : p.seqlen;  // keys this tile needs
   const int n_kv = (key_end + kBN - 1) / kBN;
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(&bars->q_full, qbytes);
-      if (p.form == 1) {
+      if (kForm == 1) {
         tma_load_4d(sQ, &tm_q, &bars->q_full, 0, hh, q0, b);
         tma_load_4d(sQ + kQBox, &tm_q, &bars->q_full, 64, hh, q0, b);
       } else {
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = warp - 9;
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
-      const int nk = p.form == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T
+      const int nk = kForm == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T
       if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
         for (int j = 0; j < n_kv; ++j) {
           const int s = j % kStages;
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t kt = k_addr + s * kKVTile;
           for (int kk = 0; kk < nk; ++kk) {
             uint32_t a, bb;
-            if (p.form == 1) {  // branch r = columns [64 r, 64 r + 64)
+            if (kForm == 1) {  // branch r = columns [64 r, 64 r + 64)
               a = q_addr + r * kQBox + kk * 32;
               bb = kt + r * kKVBox + kk * 32;
             } else {            // branch r = query head 2p + r, full 128 columns
@@ -261,8 +263,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int j = 0; j < n_kv; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(&bars->s_full[r][buf], (uint32_t)(j >> 1) & 1u, p.dev_status, &failed))
+      // Tensor-memory loads and stores below are warp-collective, so a failed
+      // wait in any lane ends the loop for the whole warp.
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&bars->s_full[r][buf], (uint32_t)(j >> 1) & 1u, p.dev_status,
+                                &failed))) {
+        failed = true;
         break;
+      }
       tc_fence_after();
       const uint32_t t_s = tmem + lane_off + s_col(r, buf);
       uint32_t sr[64];  // raw S row of this tile (masked entries set to -inf)
@@ -314,7 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    sc2, nu2);
           float x0, x1, p0, p1;
           f2unpack(x2, x0, x1);
-          if ((e & 3) == 3) {
+          // Share of exponentials on the polynomial: V1's shorter Q.K^T leaves
+          // the softmax the critical path, so it offloads more (measured).
+          if (kForm == 1 ? (e & 3) == 3 : (e & 7) == 7) {
             exp2_poly2(x0, x1, p0, p1);
           } else {
             p0 = ex2(x0);
@@ -331,9 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__any_sync(0xffffffffu, resc)) {
         // O_r must be quiescent (the previous tile's P.V into O_r done) before
         // it is rescaled in place; rows that keep their reference use alpha 1.
-        if (!mbar_wait(&bars->o_done[r][(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u,
-                       p.dev_status, &failed))
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[r][(j - 1) & 1],
+                                                (uint32_t)((j - 1) >> 1) & 1u, p.dev_status,
+                                                &failed))) {
+          failed = true;
           break;
+        }
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -452,12 +465,13 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
   const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +
                    4 * kBM * (int)sizeof(float) + 64;
-  cudaError_t e = cudaFuncSetAttribute(diffattn_prefill_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = a.form == 1 ? diffattn_prefill_tc_kernel<1> : diffattn_prefill_tc_kernel<2>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long grid = (long long)p.n_qtiles * bh_count;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-  diffattn_prefill_tc_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
+  kern<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
   return cudaGetLastError();
 }
 
