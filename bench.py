@@ -420,6 +420,34 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
                                  "batch": w.B}
         del kc, vc, ws
         torch.cuda.empty_cache()
+
+    if want("snr_v1_decode"):  # noise-cancellation sweep, 6 configs x 11 lambdas, L 1024
+        from differential_attention_sm_b200 import snr as S
+        w = wl("snr_v1_decode")
+        x = I.snr_inputs(w.seed, w.L, w.d, w.dv, **{k: w.extra[k] for k in
+                                                     ("sigmas", "rhos", "alpha", "pos")})
+        res = S.run_sweep(x, device=str(dev))
+        q, kc, vc, lamt = (x[n].to(dev) for n in ("q", "k_cache", "v_cache", "lam"))
+        B_, H_ = q.shape[0], q.shape[1]
+        ws = torch.empty(Bd.diffattn_v1_decode_workspace_size(B_, H_, w.d, w.dv, w.L),
+                         dtype=torch.uint8, device=dev)
+        o = torch.empty(B_, H_, w.dv, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v1_decode(q, kc, vc, lamt, workspace=ws, out=o),
+                       20, 3, stream)
+        by = v1_decode_bytes(B_, w.L, H_, w.d, w.dv)
+        gbs = by / (ms * 1e-3) / 1e9
+        summary = []
+        for c, (sigma, rho) in enumerate(res["configs"]):
+            r = res["snr"][c]
+            i = int(np.nanargmax(r))
+            summary.append({"sigma": sigma, "rho": rho, "snr_softmax": round(float(r[0]), 3),
+                            "snr_best": round(float(r[i]), 3),
+                            "best_lambda": round(float(res["lam"][i]), 2)})
+        out["snr_v1_decode"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
+                                "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": by,
+                                "batch": B_, "sweep": summary}
+        del kc, vc, ws
+        torch.cuda.empty_cache()
     out["peak_source"] = peak_src
     return out
 
@@ -498,12 +526,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the secondary workloads (V2 prefill, long V1, decode)")
+                    help="skip the secondary workloads (V2 prefill, long V1, decode, SNR sweep)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded host time for the oracle CPU baseline")
     ap.add_argument("--only", default=None,
                     choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
-                             "v1_decode_bf16"],
+                             "v1_decode_bf16", "snr_v1_decode"],
                     help="run just this secondary workload (one GPU) and print its numbers")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="with --only: smaller decode batch (profiling runs)")

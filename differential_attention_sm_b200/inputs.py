@@ -19,6 +19,9 @@ Recipe (shared by every test and the benchmark):
     K[p] is set to 4 * (Q1[N-2] + Q1[N-1]) / 2 in float32 before rounding.
     This mimics the six-needle retrieval setting of the "Differential
     Transformer" glossary page ("Ventajas comunicadas").
+  * noise-cancellation query (``snr_inputs``): one query against 1024 keys,
+    following step 4 of the lesson "Atencion Diferencial (V2)" (a signal
+    token at a known position, noise everywhere else).  See that function.
 """
 from __future__ import annotations
 
@@ -69,6 +72,12 @@ WORKLOADS = {
                                L=32768, Hq=64, Hkv=8, d=128),
     "v1_decode_bf16": Workload("v1_decode_bf16", "v1_decode", BF16, 4, B=64,
                                L=32768, H=32, d=64, dv=128, layer=12),
+    # noise-cancellation sweep: 3 noise amplitudes x 2 branch-noise correlations,
+    # lambda 0, 0.1, ..., 1.0 as 11 heads, run through the V1 decode kernel
+    "snr_v1_decode": Workload("snr_v1_decode", "snr", BF16, 5, B=48, L=1024, H=11,
+                              d=64, dv=128,
+                              extra={"sigmas": (1.0, 2.0, 3.0), "rhos": (1.0, 0.9),
+                                     "alpha": 6.0, "pos": 517}),
 }
 
 
@@ -188,3 +197,70 @@ def fill_normal_on_device(t: torch.Tensor, seed: int) -> torch.Tensor:
         flat[lo:hi] = torch.randn(hi - lo, generator=g, device=t.device,
                                   dtype=torch.float32).to(t.dtype)
     return t
+
+
+def snr_inputs(seed: int = 5, L: int = 1024, d: int = 64, dv: int = 128,
+               sigmas=(1.0, 2.0, 3.0), rhos=(1.0, 0.9), alpha: float = 6.0,
+               pos: int = 517, lam_grid=None):
+    """Signal-plus-noise query for the noise-cancellation sweep.
+
+    Step 4 of the lesson "Atencion Diferencial (V2)" (section "Paso 4:
+    medicion de la cancelacion de ruido") puts a signal token at a known
+    position of a length-1024 sequence and fills the rest with noise;
+    exercise 4 sweeps lambda from 0 to 1 and exercise 1 varies the noise
+    amplitude.  Reading used here (the pages fix no construction):
+
+      * one configuration per (noise amplitude sigma, branch correlation rho);
+        u is a seeded random unit vector in R^d and both branches query with
+        q1 = q2 = sqrt(d) u, so a key k scores u . k in either branch;
+      * noise keys: branch 1 draws n ~ N(0, sigma^2 I); branch 2 uses
+        rho n + sqrt(1 - rho^2) n' (n' independent), i.e. the noise both maps
+        see is shared to the degree rho;
+      * the signal key at ``pos``: branch 1 holds alpha u (score alpha),
+        branch 2 an ordinary noise draw (the branches differ on the signal);
+      * lambda is swept over ``lam_grid`` (default 0, 0.1, ..., 1.0), one
+        value per head, all heads holding the same query and keys.
+
+    To read the per-key differential weights w_j through the decode kernel,
+    each configuration is repeated over L / dv batch entries that differ only
+    in V: entry g of a configuration has V[j, c] = 1 when j = g * dv + c and
+    0 otherwise, so its output row is w restricted to keys [g dv, (g+1) dv).
+
+    Returns q [B, H, 2d], k_cache [B, L, H, 2d], v_cache [B, L, H, dv]
+    (bf16), lam [H] (float32), and per configuration the (bf16-rounded)
+    query ``q_cfg`` [C, 2d] and keys ``k_cfg`` [C, L, 2d] as float32, with
+    ``configs`` [(sigma, rho)], ``groups`` = L / dv and ``pos``.
+    """
+    if L % dv:
+        raise ValueError("L must be a multiple of dv")
+    if lam_grid is None:
+        lam_grid = [i / 10.0 for i in range(11)]
+    H = len(lam_grid)
+    configs = [(float(s_), float(r_)) for s_ in sigmas for r_ in rhos]
+    C, G = len(configs), L // dv
+    g = _gen(seed)
+    q_cfg = torch.empty(C, 2 * d)
+    k_cfg = torch.empty(C, L, 2 * d)
+    for c, (sigma, rho) in enumerate(configs):
+        u = torch.randn(d, generator=g)
+        u = u / u.norm()
+        n1 = sigma * torch.randn(L, d, generator=g)
+        n2 = sigma * torch.randn(L, d, generator=g)
+        q_cfg[c, :d] = (d ** 0.5) * u
+        q_cfg[c, d:] = (d ** 0.5) * u
+        k_cfg[c, :, :d] = n1
+        k_cfg[c, :, d:] = rho * n1 + (1.0 - rho * rho) ** 0.5 * n2
+        k_cfg[c, pos, :d] = alpha * u
+    q_cfg = q_cfg.to(BF16).float()
+    k_cfg = k_cfg.to(BF16).float()
+    B = C * G
+    q = q_cfg.repeat_interleave(G, dim=0)[:, None, :].expand(B, H, 2 * d)
+    k = k_cfg.repeat_interleave(G, dim=0)[:, :, None, :].expand(B, L, H, 2 * d)
+    onehot = torch.zeros(G, L, dv)
+    for gi in range(G):
+        onehot[gi, gi * dv:(gi + 1) * dv, :] = torch.eye(dv)
+    v = onehot.repeat(C, 1, 1)[:, :, None, :].expand(B, L, H, dv)
+    return {"q": q.to(BF16).contiguous(), "k_cache": k.to(BF16).contiguous(),
+            "v_cache": v.to(BF16).contiguous(),
+            "lam": torch.tensor(lam_grid, dtype=FP32), "q_cfg": q_cfg, "k_cfg": k_cfg,
+            "configs": configs, "groups": G, "pos": pos}

@@ -13,4 +13,6 @@ from .oracle import (  # noqa: F401
     v2_decode_rows,
     v1_decode_rows,
     n_threads,
+    v1_query_weights,
+    snr,
 )

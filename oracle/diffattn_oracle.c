@@ -17,7 +17,8 @@
  *        edition, "Diferansiyel Dikkat Nasıl Çalışır").
  *   [L]  "Atención Diferencial (V2)", ai-engineering.academy lesson:
  *        "El piso de ruido de softmax", "La idea diferencial",
- *        "V1 vs V2: la diferencia", "Implementación" steps 1-3.
+ *        "V1 vs V2: la diferencia", "Implementación" steps 1-3, and
+ *        step 4 "medición de la cancelación de ruido" (signal-to-noise).
  *
  * Readings of points the pages leave open (each one is listed with its
  * reason in the design notes):
@@ -74,6 +75,17 @@ int oracle_lambda_from_params(const float *lq1, const float *lk1,
         lambda_out[h] = exp(dot1) - exp(dot2) + linit;
     }
     return ORACLE_OK;
+}
+
+/* Sliding window: of the n visible keys 0..n-1 (causal prefix or cache
+ * entries), only the last `window` stay visible; window <= 0 keeps all.
+ * [L] "Úselo" names hybrids of differential and sliding-window attention;
+ * the reading is that query i then sees keys j with i - window < j <= i in
+ * both branches, and a decode query the last `window` cache entries.
+ * Returns the first visible key. */
+static int64_t window_start(int64_t n, int window)
+{
+    return (window > 0 && n > (int64_t)window) ? n - (int64_t)window : 0;
 }
 
 /* softmax of one row with the row maximum subtracted first
@@ -158,7 +170,7 @@ static void head_rms_norm(double *o, int dv, const float *g, double eps,
  */
 int oracle_v1_rows(const float *q, const float *k, const float *v,
                    int B, int N, int H, int d, int dv,
-                   const double *lambda, int causal,
+                   const double *lambda, int causal, int window,
                    int apply_norm, const float *norm_weight, double eps,
                    double lambda_init,
                    const int64_t *rows, int64_t n_rows,
@@ -187,8 +199,12 @@ int oracle_v1_rows(const float *q, const float *k, const float *v,
         double *w = weights ? weights + t * (int64_t)N : NULL;
         if (w) for (int64_t j = 0; j < N; ++j) w[j] = 0.0;
         double *o = out + t * (int64_t)dv;
+        const int64_t first = window_start(n_keys, window);
+        kb += first * tok_qk;
+        vb += first * tok_v;
+        if (w) w += first;
         diff_attention_row(qrow, qrow + d, kb, kb + d, tok_qk, vb, tok_v,
-                           n_keys, d, dv, lambda[h], a1, a2, w, o);
+                           n_keys - first, d, dv, lambda[h], a1, a2, w, o);
         if (apply_norm) head_rms_norm(o, dv, norm_weight, eps, lambda_init);
     }
     free(a1);
@@ -206,7 +222,7 @@ int oracle_v1_rows(const float *q, const float *k, const float *v,
  */
 int oracle_v2_rows(const float *q, const float *k, const float *v,
                    int B, int N, int Hq, int Hkv, int d,
-                   const double *lambda, int causal,
+                   const double *lambda, int causal, int window,
                    const int64_t *rows, int64_t n_rows,
                    double *out, double *weights)
 {
@@ -234,7 +250,11 @@ int oracle_v2_rows(const float *q, const float *k, const float *v,
         const float *vb = v + (int64_t)b * N * tok_kv + (int64_t)g * d;
         double *w = weights ? weights + t * (int64_t)N : NULL;
         if (w) for (int64_t j = 0; j < N; ++j) w[j] = 0.0;
-        diff_attention_row(qa, qb, kb, kb, tok_kv, vb, tok_kv, n_keys, d, d,
+        const int64_t first = window_start(n_keys, window);
+        kb += first * tok_kv;
+        vb += first * tok_kv;
+        if (w) w += first;
+        diff_attention_row(qa, qb, kb, kb, tok_kv, vb, tok_kv, n_keys - first, d, d,
                            lambda[p], a1, a2, w, out + t * (int64_t)d);
     }
     free(a1);
@@ -251,7 +271,7 @@ int oracle_v2_rows(const float *q, const float *k, const float *v,
  * appended).  [L] "V1 vs V2" (KV cache read once per decode step in V2).
  */
 int oracle_v2_decode_rows(const float *q, const float *k_cache, const float *v_cache,
-                          const int *lens, int max_len,
+                          const int *lens, int max_len, int window,
                           int B, int Hq, int Hkv, int d, const double *lambda,
                           const int64_t *rows, int64_t n_rows, double *out)
 {
@@ -273,7 +293,10 @@ int oracle_v2_decode_rows(const float *q, const float *k_cache, const float *v_c
         const float *qa = q + ((int64_t)b * Hq + 2 * p) * d;
         const float *kb = k_cache + (int64_t)b * max_len * tok_kv + (int64_t)g * d;
         const float *vb = v_cache + (int64_t)b * max_len * tok_kv + (int64_t)g * d;
-        diff_attention_row(qa, qa + d, kb, kb, tok_kv, vb, tok_kv, len, d, d,
+        const int64_t first = window_start(len, window);
+        kb += first * tok_kv;
+        vb += first * tok_kv;
+        diff_attention_row(qa, qa + d, kb, kb, tok_kv, vb, tok_kv, len - first, d, d,
                            lambda[p], a1, a2, NULL, out + t * (int64_t)d);
     }
     free(a1);
@@ -287,7 +310,7 @@ int oracle_v2_decode_rows(const float *q, const float *k_cache, const float *v_c
  *   rows : r = b*H + h;  out : [n_rows, dv]; optional per-head norm as in V1.
  */
 int oracle_v1_decode_rows(const float *q, const float *k_cache, const float *v_cache,
-                          const int *lens, int max_len,
+                          const int *lens, int max_len, int window,
                           int B, int H, int d, int dv, const double *lambda,
                           int apply_norm, const float *norm_weight, double eps,
                           double lambda_init,
@@ -310,11 +333,33 @@ int oracle_v1_decode_rows(const float *q, const float *k_cache, const float *v_c
         const float *kb = k_cache + (int64_t)b * max_len * tok_k + (int64_t)h * 2 * d;
         const float *vb = v_cache + (int64_t)b * max_len * tok_v + (int64_t)h * dv;
         double *o = out + t * (int64_t)dv;
-        diff_attention_row(qr, qr + d, kb, kb + d, tok_k, vb, tok_v, len, d, dv,
+        const int64_t first = window_start(len, window);
+        kb += first * tok_k;
+        vb += first * tok_v;
+        diff_attention_row(qr, qr + d, kb, kb + d, tok_k, vb, tok_v, len - first, d, dv,
                            lambda[h], a1, a2, NULL, o);
         if (apply_norm) head_rms_norm(o, dv, norm_weight, eps, lambda_init);
     }
     free(a1);
     free(a2);
     return rc;
+}
+
+/*
+ * Signal-to-noise ratio of one attention-weight row ([L] step 4 asks for the
+ * ratio at a signal position in a signal-plus-noise query but fixes no
+ * formula).  Reading: the weight at the signal position divided by the
+ * root-mean-square weight over every other position,
+ *     snr = w[pos] / sqrt( (1/(n-1)) * sum_{j != pos} w[j]^2 ),
+ * so a map that puts no weight off the signal has infinite ratio.
+ */
+int oracle_snr(const double *w, int64_t n, int64_t pos, double *out)
+{
+    if (!w || !out || n < 2 || pos < 0 || pos >= n) return ORACLE_ERR_ARG;
+    double ss = 0.0;
+    for (int64_t j = 0; j < n; ++j)
+        if (j != pos) ss += w[j] * w[j];
+    const double rms = sqrt(ss / (double)(n - 1));
+    *out = rms > 0.0 ? w[pos] / rms : (w[pos] > 0.0 ? INFINITY : (w[pos] < 0.0 ? -INFINITY : NAN));
+    return ORACLE_OK;
 }

@@ -58,20 +58,22 @@ def _load():
         lib.oracle_v1_rows.restype = ctypes.c_int
         lib.oracle_v1_rows.argtypes = [
             _f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_int, ctypes.c_int, _f64p, ctypes.c_int, ctypes.c_int, _f32p,
+            ctypes.c_int, ctypes.c_int, _f64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p,
             ctypes.c_double, ctypes.c_double, _i64p, ctypes.c_int64, _f64p, _f64p]
         lib.oracle_v2_rows.restype = ctypes.c_int
         lib.oracle_v2_rows.argtypes = [
             _f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_int, ctypes.c_int, _f64p, ctypes.c_int, _i64p, ctypes.c_int64,
+            ctypes.c_int, ctypes.c_int, _f64p, ctypes.c_int, ctypes.c_int, _i64p, ctypes.c_int64,
             _f64p, _f64p]
         lib.oracle_v2_decode_rows.restype = ctypes.c_int
         lib.oracle_v2_decode_rows.argtypes = [
-            _f32p, _f32p, _f32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            _f32p, _f32p, _f32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, _f64p, _i64p, ctypes.c_int64, _f64p]
+        lib.oracle_snr.restype = ctypes.c_int
+        lib.oracle_snr.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64, _f64p]
         lib.oracle_v1_decode_rows.restype = ctypes.c_int
         lib.oracle_v1_decode_rows.argtypes = [
-            _f32p, _f32p, _f32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            _f32p, _f32p, _f32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, _f64p, ctypes.c_int, _f32p, ctypes.c_double,
             ctypes.c_double, _i64p, ctypes.c_int64, _f64p]
         _lib = lib
@@ -146,9 +148,10 @@ def lambda_from_params(lq1, lk1, lq2, lk2, layer: int) -> np.ndarray:
 
 def v1_rows(q, k, v, lam, rows, *, causal: bool, apply_norm: bool = False,
             norm_weight=None, eps: float = 1e-5, lambda_init_value: float = 0.0,
-            return_weights: bool = False, threads: int | None = None):
+            return_weights: bool = False, window: int = 0, threads: int | None = None):
     """V1 rows r = (b*N + i)*H + h of out [B, N, H, dv] (double).
-    q, k: [B, N, H, 2d]; v: [B, N, H, dv]; lam: [H]."""
+    q, k: [B, N, H, 2d]; v: [B, N, H, dv]; lam: [H].  window > 0 keeps only
+    the last ``window`` visible keys of each row (sliding window)."""
     qf, kf, vf = _f32(q), _f32(k), _f32(v)
     B, N, H, d2 = qf.shape
     dv = vf.shape[-1]
@@ -159,7 +162,7 @@ def v1_rows(q, k, v, lam, rows, *, causal: bool, apply_norm: bool = False,
     def call(r, o, w):
         return lib.oracle_v1_rows(
             _ptr(qf, _f32p), _ptr(kf, _f32p), _ptr(vf, _f32p), B, N, H, d2 // 2, dv,
-            _ptr(lamd, _f64p), int(causal), int(apply_norm), _ptr(g, _f32p),
+            _ptr(lamd, _f64p), int(causal), int(window), int(apply_norm), _ptr(g, _f32p),
             float(eps), float(lambda_init_value), _ptr(r, _i64p), r.size,
             _ptr(o, _f64p), _ptr(w, _f64p))
 
@@ -167,7 +170,7 @@ def v1_rows(q, k, v, lam, rows, *, causal: bool, apply_norm: bool = False,
 
 
 def v2_rows(q, k, v, lam, rows, *, causal: bool, return_weights: bool = False,
-            threads: int | None = None):
+            window: int = 0, threads: int | None = None):
     """V2 rows r = (b*N + i)*(Hq/2) + p of out [B, N, Hq/2, d] (double).
     q: [B, N, Hq, d]; k, v: [B, N, Hkv, d]; lam: [Hq/2]."""
     qf, kf, vf = _f32(q), _f32(k), _f32(v)
@@ -179,13 +182,13 @@ def v2_rows(q, k, v, lam, rows, *, causal: bool, return_weights: bool = False,
     def call(r, o, w):
         return lib.oracle_v2_rows(
             _ptr(qf, _f32p), _ptr(kf, _f32p), _ptr(vf, _f32p), B, N, Hq, Hkv, d,
-            _ptr(lamd, _f64p), int(causal), _ptr(r, _i64p), r.size,
+            _ptr(lamd, _f64p), int(causal), int(window), _ptr(r, _i64p), r.size,
             _ptr(o, _f64p), _ptr(w, _f64p))
 
     return _run_rows(call, rows, d, N if return_weights else None, threads)
 
 
-def v2_decode_rows(q, k_cache, v_cache, lam, rows, *, lens=None,
+def v2_decode_rows(q, k_cache, v_cache, lam, rows, *, lens=None, window: int = 0,
                    threads: int | None = None):
     """V2 decode rows r = b*(Hq/2) + p of out [B, Hq/2, d] (double).
     q: [B, Hq, d]; caches: [B, max_len, Hkv, d]; lens: [B] or None."""
@@ -200,7 +203,7 @@ def v2_decode_rows(q, k_cache, v_cache, lam, rows, *, lens=None,
     def call(r, o, w):
         return lib.oracle_v2_decode_rows(
             _ptr(qf, _f32p), _ptr(kf, _f32p), _ptr(vf, _f32p), _ptr(ln, _i32p),
-            max_len, B, Hq, Hkv, d, _ptr(lamd, _f64p), _ptr(r, _i64p), r.size,
+            max_len, int(window), B, Hq, Hkv, d, _ptr(lamd, _f64p), _ptr(r, _i64p), r.size,
             _ptr(o, _f64p))
 
     return _run_rows(call, rows, d, None, threads)
@@ -208,7 +211,8 @@ def v2_decode_rows(q, k_cache, v_cache, lam, rows, *, lens=None,
 
 def v1_decode_rows(q, k_cache, v_cache, lam, rows, *, lens=None,
                    apply_norm: bool = False, norm_weight=None, eps: float = 1e-5,
-                   lambda_init_value: float = 0.0, threads: int | None = None):
+                   lambda_init_value: float = 0.0, window: int = 0,
+                   threads: int | None = None):
     """V1 decode rows r = b*H + h of out [B, H, dv] (double).
     q: [B, H, 2d]; k_cache: [B, max_len, H, 2d]; v_cache: [B, max_len, H, dv]."""
     qf, kf, vf = _f32(q), _f32(k_cache), _f32(v_cache)
@@ -223,8 +227,42 @@ def v1_decode_rows(q, k_cache, v_cache, lam, rows, *, lens=None,
     def call(r, o, w):
         return lib.oracle_v1_decode_rows(
             _ptr(qf, _f32p), _ptr(kf, _f32p), _ptr(vf, _f32p), _ptr(ln, _i32p),
-            max_len, B, H, d2 // 2, dv, _ptr(lamd, _f64p), int(apply_norm),
+            max_len, int(window), B, H, d2 // 2, dv, _ptr(lamd, _f64p), int(apply_norm),
             _ptr(g, _f32p), float(eps), float(lambda_init_value), _ptr(r, _i64p),
             r.size, _ptr(o, _f64p))
 
     return _run_rows(call, rows, dv, None, threads)
+
+
+def v1_query_weights(q_row, keys, lam):
+    """Differential weights w_j = a1_j - lam_h * a2_j of ONE V1 query row
+    against L keys, for every lambda in ``lam``: returns [len(lam), L]
+    (double).  q_row: [2d]; keys: [L, 2d].  Computed by the oracle's V1
+    row routine (non-causal, query placed at row 0 of an L-row block)."""
+    q_row = np.asarray(q_row, dtype=np.float32).reshape(-1)
+    keys = np.asarray(keys, dtype=np.float32)
+    L, d2 = keys.shape
+    H = int(np.asarray(lam).size)
+    q = np.zeros((1, L, H, d2), dtype=np.float32)
+    q[0, 0, :, :] = q_row
+    k = np.ascontiguousarray(np.broadcast_to(keys[None, :, None, :], (1, L, H, d2)))
+    v = np.zeros((1, L, H, 1), dtype=np.float32)
+    _, w = v1_rows(q, k, v, lam, np.arange(H), causal=False, return_weights=True)
+    return w
+
+
+def snr(weights, pos: int):
+    """Signal-to-noise ratio of each weight row (last axis): the weight at
+    ``pos`` over the RMS weight elsewhere (``oracle_snr``)."""
+    w = np.ascontiguousarray(np.asarray(weights, dtype=np.float64))
+    flat = w.reshape(-1, w.shape[-1])
+    out = np.empty(flat.shape[0])
+    lib = _load()
+    one = np.zeros(1)
+    for i in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[i])
+        rc = lib.oracle_snr(_ptr(row, _f64p), row.size, int(pos), _ptr(one, _f64p))
+        if rc != 0:
+            raise ValueError("oracle_snr status %d" % rc)
+        out[i] = one[0]
+    return out.reshape(w.shape[:-1])

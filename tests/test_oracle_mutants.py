@@ -29,6 +29,13 @@ MUTANTS = [
     ("return 0.8 - 0.6 * exp(-0.3 * (double)(layer - 1));", "return 0.8 - 0.6 * exp(-0.3 * (double)(layer));", "layer base"),
     ("x[j] = exp(x[j] - m);", "x[j] = exp(x[j]);", "softmax without the max shift"),
     ("for (int c = 0; c < dv; ++c) o[c] += wj * (double)vj[c];", "for (int c = 0; c < dv; ++c) o[c] += a1[j] * (double)vj[c];", "second map dropped"),
+    ("if (j != pos) ss += w[j] * w[j];", "ss += w[j] * w[j];", "signal counted as noise in the ratio"),
+    ("sqrt(ss / (double)(n - 1))", "sqrt(ss / (double)n)", "noise mean over every position"),
+    ("? n - (int64_t)window : 0;", "? n - (int64_t)window + 1 : 0;", "window one key short"),
+    ("        vb += first * tok_v;\n        if (w) w += first;\n        diff_attention_row(qrow",
+     "        if (w) w += first;\n        diff_attention_row(qrow", "window not applied to values (V1)"),
+    ("        const int64_t first = window_start(len, window);\n        kb += first * tok_kv;",
+     "        const int64_t first = 0;\n        kb += first * tok_kv;", "window ignored in V2 decode"),
 ]
 
 

@@ -324,3 +324,145 @@ def test_large_logits_stay_finite_and_exact():
     a2 = sdpa(q[..., d:], k[..., d:], v)
     ref = a1 - torch.tensor(lam, dtype=torch.float64).view(1, 1, H, 1) * a2
     assert np.abs(out - ref.reshape(-1, dv).numpy()).max() < 1e-9
+
+
+# --------------------------------------------------------------------------
+# [L] step 4 / exercises 1 and 4: noise cancellation on a signal-plus-noise
+# query.  The ratio is the signal weight over the RMS of the other weights.
+# --------------------------------------------------------------------------
+def test_snr_statistic_on_hand_built_rows():
+    w = np.full(101, 0.01)
+    w[1::2] = -0.01
+    w[40] = 0.5
+    assert O.snr(w, 40) == pytest.approx(50.0, rel=1e-14)
+    w2 = np.zeros(7)
+    w2[3] = 0.25
+    assert O.snr(w2, 3) == math.inf
+    w3 = np.array([3.0, 1.0, 1.0, 1.0, 4.0])   # noise rms = sqrt((9+1+1+16)/4) at pos 1
+    assert O.snr(w3, 1) == pytest.approx(1.0 / math.sqrt(27.0 / 4.0), rel=1e-14)
+
+
+def _snr_scores(x, c):
+    """fp64 scores of the sweep query against its keys, per branch."""
+    q = x["q_cfg"][c].double()
+    k = x["k_cfg"][c].double()
+    d = q.numel() // 2
+    return (k[:, :d] @ q[:d]) / math.sqrt(d), (k[:, d:] @ q[d:]) / math.sqrt(d)
+
+
+def test_snr_sweep_lambda_zero_is_softmax_and_rows_sum_to_one_minus_lambda():
+    x = I.snr_inputs()
+    lam = x["lam"].double().numpy()
+    for c in range(len(x["configs"])):
+        w = O.v1_query_weights(x["q_cfg"][c], x["k_cfg"][c], lam)
+        s1, _ = _snr_scores(x, c)
+        assert np.abs(w[0] - torch.softmax(s1, 0).numpy()).max() < 1e-15
+        assert np.abs(w.sum(1) - (1.0 - lam)).max() < 1e-12
+
+
+def test_snr_shared_noise_cancels_exactly_at_partition_ratio():
+    """With q1 = q2 and the same noise keys in both branches, every noise
+    weight is e^{s_j} (1/Z1 - lambda/Z2): all of them vanish together at
+    lambda* = Z2 / Z1, where only the signal weight is left."""
+    x = I.snr_inputs(sigmas=(1.5,), rhos=(1.0,))
+    s1, s2 = _snr_scores(x, 0)
+    pos = x["pos"]
+    mask = torch.ones_like(s1, dtype=torch.bool)
+    mask[pos] = False
+    assert torch.equal(s1[mask], s2[mask])
+    lam_star = float(torch.exp(torch.logsumexp(s2, 0) - torch.logsumexp(s1, 0)))
+    w = O.v1_query_weights(x["q_cfg"][0], x["k_cfg"][0], [lam_star, 0.5])
+    noise = np.delete(w[0], pos)
+    assert np.abs(noise).max() < 1e-15 * np.abs(w[0]).max() + 1e-300
+    sig = float(torch.softmax(s1, 0)[pos] - lam_star * torch.softmax(s2, 0)[pos])
+    assert w[0, pos] == pytest.approx(sig, rel=1e-12)
+    assert O.snr(w[1:], pos)[0] < O.snr(w[:1], pos)[0]
+
+
+def test_snr_identical_branches_do_not_depend_on_lambda():
+    """K2 = K1 everywhere (the signal included): w = (1 - lambda) softmax, so
+    the ratio is the same for every lambda < 1."""
+    x = I.snr_inputs(sigmas=(1.0,), rhos=(1.0,))
+    k = x["k_cfg"][0].clone()
+    d = k.shape[1] // 2
+    k[:, d:] = k[:, :d]
+    lam = np.array([0.0, 0.3, 0.6, 0.9])
+    r = O.snr(O.v1_query_weights(x["q_cfg"][0], k, lam), x["pos"])
+    assert np.abs(r / r[0] - 1.0).max() < 1e-12
+
+
+# --------------------------------------------------------------------------
+# [L] "Úselo": differential attention combined with sliding-window attention.
+# Reading: query i sees keys j with i - W < j <= i, in both branches.
+# --------------------------------------------------------------------------
+def _band_mask(N, W):
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    return (j <= i) & (j > i - W)
+
+
+@pytest.mark.parametrize("W", [1, 5, 16, 40])
+def test_window_is_difference_of_band_masked_attentions(W):
+    B, N, H, d, dv = 2, 37, 3, 8, 16
+    q, k, v = rand(B, N, H, 2 * d, seed=70), rand(B, N, H, 2 * d, seed=71), rand(B, N, H, dv, seed=72)
+    lams = torch.tensor([0.8, -0.3, 1.2], dtype=torch.float64)
+    out = O.v1_rows(q, k, v, lams, all_rows_v1(B, N, H), causal=True, window=W)
+    m = _band_mask(N, W)
+
+    def att(qh, kh):
+        qt, kt, vt = (x.double().permute(0, 2, 1, 3) for x in (qh, kh, v))
+        return F.scaled_dot_product_attention(qt, kt, vt, attn_mask=m).permute(0, 2, 1, 3)
+
+    ref = att(q[..., :d], k[..., :d]) - lams.view(1, 1, H, 1) * att(q[..., d:], k[..., d:])
+    assert np.abs(out - ref.reshape(-1, dv).numpy()).max() < 1e-12
+
+
+def test_window_one_keeps_only_the_diagonal_and_wide_window_is_causal():
+    B, N, H, d, dv = 1, 19, 2, 8, 16
+    q, k, v = rand(B, N, H, 2 * d, seed=73), rand(B, N, H, 2 * d, seed=74), rand(B, N, H, dv, seed=75)
+    lam = [0.6, 1.4]
+    out = O.v1_rows(q, k, v, lam, all_rows_v1(B, N, H), causal=True, window=1)
+    ref = (1.0 - torch.tensor(lam, dtype=torch.float64)).view(1, 1, H, 1) * v.double()
+    assert np.abs(out - ref.reshape(-1, dv).numpy()).max() < 1e-15
+    full = O.v1_rows(q, k, v, lam, all_rows_v1(B, N, H), causal=True)
+    wide = O.v1_rows(q, k, v, lam, all_rows_v1(B, N, H), causal=True, window=N)
+    assert np.array_equal(full, wide)
+
+
+def test_window_row_equals_last_row_of_the_sliced_sequence():
+    """Row i under window W is causal attention over tokens i-W+1..i alone."""
+    B, N, Hq, Hkv, d, W = 1, 41, 4, 2, 16, 9
+    x = I.v2_inputs(B, N, Hq, Hkv, d, seed=76, dtype=torch.float32)
+    P = Hq // 2
+    out = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], np.arange(B * N * P), causal=True,
+                    window=W).reshape(N, P, d)
+    for i in (0, 5, W - 1, W, 23, N - 1):
+        a = max(0, i - W + 1)
+        sl = O.v2_rows(x["q"][:, a:i + 1], x["k"][:, a:i + 1], x["v"][:, a:i + 1], x["lam"],
+                       np.arange((i - a) * P, (i - a + 1) * P), causal=True).reshape(P, d)
+        assert np.abs(out[i] - sl).max() < 1e-13
+
+
+def test_window_decode_equals_decode_over_the_last_entries():
+    Bn, L, Hq, Hkv, d, W = 2, 70, 8, 2, 16, 13
+    x = I.v2_decode_inputs(Bn, L, Hq, Hkv, d, seed=77, dtype=torch.float32)
+    lens = [70, 31]
+    rows = np.arange(Bn * Hq // 2)
+    out = O.v2_decode_rows(x["q"], x["k_cache"], x["v_cache"], x["lam"], rows, lens=lens,
+                           window=W).reshape(Bn, Hq // 2, d)
+    for b, n in enumerate(lens):
+        kc = x["k_cache"][b:b + 1, n - W:n]
+        vc = x["v_cache"][b:b + 1, n - W:n]
+        ref = O.v2_decode_rows(x["q"][b:b + 1], kc, vc, x["lam"], np.arange(Hq // 2))
+        assert np.abs(out[b] - ref).max() < 1e-13
+    # V1 decode: the window applies before the norm
+    x1 = I.v1_decode_inputs(Bn, L, 3, 8, 16, seed=78)
+    lam1 = np.array([0.7, 0.2, -0.4])
+    o1 = O.v1_decode_rows(x1["q"], x1["k_cache"], x1["v_cache"], lam1, np.arange(Bn * 3),
+                          lens=lens, apply_norm=True, lambda_init_value=0.5,
+                          window=W).reshape(Bn, 3, 16)
+    for b, n in enumerate(lens):
+        r1 = O.v1_decode_rows(x1["q"][b:b + 1], x1["k_cache"][b:b + 1, n - W:n],
+                              x1["v_cache"][b:b + 1, n - W:n], lam1, np.arange(3),
+                              apply_norm=True, lambda_init_value=0.5)
+        assert np.abs(o1[b] - r1).max() < 1e-13
