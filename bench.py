@@ -53,6 +53,13 @@ def v2_decode_bytes(B, L, Hkv, d, Hq):
     return B * L * Hkv * d * 2 * 2 + B * Hq * d * 2 + B * (Hq // 2) * d * 2
 
 
+def window_pairs(B, N, H, W):
+    """Visible (query, key) pairs of causal prefill with a sliding window W:
+    row i sees min(i + 1, W) keys."""
+    full = min(N, W)
+    return B * H * (full * (full + 1) // 2 + (N - full) * W)
+
+
 def v1_decode_bytes(B, L, H, d, dv):
     return B * L * H * (2 * d + dv) * 2 + B * H * 2 * d * 2 + B * H * dv * 2
 
@@ -421,6 +428,48 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         del kc, vc, ws
         torch.cuda.empty_cache()
 
+    if want("v2_prefill_window_bf16"):  # V2 prefill with a 1024-key sliding window
+        w = wl("v2_prefill_window_bf16")
+        W = w.extra["window"]
+        x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
+        q, k, v, lamt = (x[n].to(dev) for n in ("q", "k", "v", "lam"))
+        o = torch.empty(w.B, w.N, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v2_prefill_window(q, k, v, lamt, W, out=o), 20, 3,
+                       stream)
+        pairs = window_pairs(w.B, w.N, w.Hq // 2, W)
+        flop = pairs * v2_flops_per_pair(w.d)
+        t = flop / (ms * 1e-3) / 1e12
+        out["v2_prefill_window_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s",
+                                         "ms": round(ms, 4),
+                                         "frac": round(t / peaks["bf16_tflops"], 4),
+                                         "flop": flop, "window": W}
+        del q, k, v, o
+        torch.cuda.empty_cache()
+
+    if want("v2_decode_window_bf16"):  # V2 decode reading the last 4096 of 32768 entries
+        w = wl("v2_decode_window_bf16")
+        W = w.extra["window"]
+        x = I.v2_decode_inputs(w.B, w.L, w.Hq, w.Hkv, w.d, w.seed, fill_caches=False)
+        kc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.Hkv, w.d, dtype=torch.bfloat16,
+                                                 device=dev), 5)
+        vc = I.fill_normal_on_device(torch.empty(w.B, w.L, w.Hkv, w.d, dtype=torch.bfloat16,
+                                                 device=dev), 6)
+        q, lamt = x["q"].to(dev), x["lam"].to(dev)
+        span = min(W, w.L)
+        ws = torch.empty(Bd.diffattn_v2_decode_workspace_size(w.B, w.Hq, w.Hkv, w.d, span),
+                         dtype=torch.uint8, device=dev)
+        o = torch.empty(w.B, w.Hq // 2, w.d, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v2_decode_window(q, kc, vc, lamt, W, workspace=ws,
+                                                            out=o), 20, 3, stream)
+        by = v2_decode_bytes(w.B, span, w.Hkv, w.d, w.Hq)
+        gbs = by / (ms * 1e-3) / 1e9
+        out["v2_decode_window_bf16"] = {"value": round(gbs, 1), "unit": "GB/s",
+                                        "ms": round(ms, 4),
+                                        "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": by,
+                                        "batch": w.B, "window": W}
+        del kc, vc, ws
+        torch.cuda.empty_cache()
+
     if want("snr_v1_decode"):  # noise-cancellation sweep, 6 configs x 11 lambdas, L 1024
         from differential_attention_sm_b200 import snr as S
         w = wl("snr_v1_decode")
@@ -531,7 +580,8 @@ def main():
                     help="bounded host time for the oracle CPU baseline")
     ap.add_argument("--only", default=None,
                     choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
-                             "v1_decode_bf16", "snr_v1_decode"],
+                             "v1_decode_bf16", "snr_v1_decode", "v2_prefill_window_bf16",
+                             "v2_decode_window_bf16"],
                     help="run just this secondary workload (one GPU) and print its numbers")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="with --only: smaller decode batch (profiling runs)")

@@ -38,6 +38,10 @@ EXPORTS = (
     "diffattn_v2_decode_noalloc",
     "diffattn_v1_decode_workspace_size",
     "diffattn_v1_decode",
+    "diffattn_v1_fwd_window",
+    "diffattn_v2_prefill_window",
+    "diffattn_v2_decode_window",
+    "diffattn_v1_decode_window",
 )
 
 
@@ -90,6 +94,18 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.diffattn_v1_decode.restype = _i
     lib.diffattn_v1_decode.argtypes = [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp,
                                        _i, _vp, _f, _f, _vp, _sz, _vp, _vp]
+    lib.diffattn_v1_fwd_window.restype = _i
+    lib.diffattn_v1_fwd_window.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i,
+                                           _i, _i, _vp, _f, _f, _vp, _vp]
+    lib.diffattn_v2_prefill_window.restype = _i
+    lib.diffattn_v2_prefill_window.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp,
+                                               _i, _i, _vp, _vp]
+    lib.diffattn_v2_decode_window.restype = _i
+    lib.diffattn_v2_decode_window.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _vp, _i, _i, _i, _i,
+                                              _i, _vp, _vp, _sz, _vp, _vp]
+    lib.diffattn_v1_decode_window.restype = _i
+    lib.diffattn_v1_decode_window.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _vp, _i, _i, _i, _i,
+                                              _i, _vp, _i, _vp, _f, _f, _vp, _sz, _vp, _vp]
     _lib = lib
     return lib
 
@@ -244,4 +260,83 @@ def diffattn_v1_decode(q, k_cache, v_cache, lam, *, cache_lens=None, apply_norm=
         B, H, d2 // 2, dv, _ptr(lam), int(bool(apply_norm)), _ptr(norm_weight),
         float(norm_eps), float(lambda_init), _ptr(workspace), ws_bytes, _ptr(dev_status),
         _stream(stream)))
+    return out
+
+
+# ---- sliding-window variants: query i sees keys (i - window, i]; a decode
+# query the last `window` cache entries (window 0 = no window) -------------
+def diffattn_v1_fwd_window(q, k, v, lam, window, *, causal=True, apply_norm=False,
+                           norm_weight=None, norm_eps=1e-5, lambda_init=0.0, out=None,
+                           dev_status=None, stream=None):
+    """V1 prefill with a sliding window.  Shapes as diffattn_v1_fwd."""
+    _need_cuda(q, k, v, lam, norm_weight, dev_status)
+    B, N, H, d2 = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty(B, N, H, dv, dtype=q.dtype, device=q.device)
+    _check("diffattn_v1_fwd_window", load().diffattn_v1_fwd_window(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, N, H, d2 // 2, dv,
+        _ptr(lam), int(bool(causal)), int(window), int(bool(apply_norm)), _ptr(norm_weight),
+        float(norm_eps), float(lambda_init), _ptr(dev_status), _stream(stream)))
+    return out
+
+
+def diffattn_v2_prefill_window(q, k, v, lam, window, *, causal=True, out=None, dev_status=None,
+                               stream=None):
+    """V2 prefill with a sliding window.  Shapes as diffattn_v2_prefill."""
+    _need_cuda(q, k, v, lam, dev_status)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty(B, N, Hq // 2, d, dtype=q.dtype, device=q.device)
+    _check("diffattn_v2_prefill_window", load().diffattn_v2_prefill_window(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, N, Hq, Hkv, d, _ptr(lam),
+        int(bool(causal)), int(window), _ptr(dev_status), _stream(stream)))
+    return out
+
+
+def _span(L, window):
+    return min(int(window), L) if window and window > 0 else L
+
+
+def diffattn_v2_decode_window(q, k_cache, v_cache, lam, window, *, cache_lens=None,
+                              workspace=None, out=None, dev_status=None, stream=None):
+    """V2 decode over the last `window` cache entries.  Shapes as
+    diffattn_v2_decode; the workspace is sized for min(window, L) entries."""
+    _need_cuda(q, k_cache, v_cache, lam, cache_lens, dev_status)
+    B, Hq, d = q.shape
+    L, Hkv = k_cache.shape[1], k_cache.shape[2]
+    ws_need = diffattn_v2_decode_workspace_size(B, Hq, Hkv, d, _span(L, window))
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if out is None:
+        out = torch.empty(B, Hq // 2, d, dtype=q.dtype, device=q.device)
+    _check("diffattn_v2_decode_window", load().diffattn_v2_decode_window(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), L, int(window), _ptr(out),
+        _dtype_code(q), B, Hq, Hkv, d, _ptr(lam), _ptr(workspace), ws_bytes, _ptr(dev_status),
+        _stream(stream)))
+    return out
+
+
+def diffattn_v1_decode_window(q, k_cache, v_cache, lam, window, *, cache_lens=None,
+                              apply_norm=False, norm_weight=None, norm_eps=1e-5,
+                              lambda_init=0.0, workspace=None, out=None, dev_status=None,
+                              stream=None):
+    """V1 decode over the last `window` cache entries.  Shapes as
+    diffattn_v1_decode; the workspace is sized for min(window, L) entries."""
+    _need_cuda(q, k_cache, v_cache, lam, cache_lens, norm_weight, dev_status)
+    B, H, d2 = q.shape
+    L, dv = k_cache.shape[1], v_cache.shape[-1]
+    ws_need = diffattn_v1_decode_workspace_size(B, H, d2 // 2, dv, _span(L, window))
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if out is None:
+        out = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    _check("diffattn_v1_decode_window", load().diffattn_v1_decode_window(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), L, int(window), _ptr(out),
+        _dtype_code(q), B, H, d2 // 2, dv, _ptr(lam), int(bool(apply_norm)),
+        _ptr(norm_weight), float(norm_eps), float(lambda_init), _ptr(workspace), ws_bytes,
+        _ptr(dev_status), _stream(stream)))
     return out

@@ -122,7 +122,18 @@ int diffattn_v1_fwd(const void* q, const void* k, const void* v, void* out, da_d
                     int batch, int seqlen, int n_heads, int d_qk, int d_v, const float* lambda,
                     int causal, int apply_norm, const float* norm_weight, float norm_eps,
                     float lambda_init, int* dev_status, void* stream) {
+  return diffattn_v1_fwd_window(q, k, v, out, dtype, batch, seqlen, n_heads, d_qk, d_v, lambda,
+                                causal, 0, apply_norm, norm_weight, norm_eps, lambda_init,
+                                dev_status, stream);
+}
+
+int diffattn_v1_fwd_window(const void* q, const void* k, const void* v, void* out,
+                           da_dtype dtype, int batch, int seqlen, int n_heads, int d_qk, int d_v,
+                           const float* lambda, int causal, int window, int apply_norm,
+                           const float* norm_weight, float norm_eps, float lambda_init,
+                           int* dev_status, void* stream) {
   if (!q || !k || !v || !out || !lambda) return DA_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && !causal)) return DA_ERR_INVALID_ARG;
   if (!dtype_ok(dtype)) return DA_ERR_INVALID_ARG;
   if (batch < 1 || seqlen < 1 || n_heads < 1 || d_qk < 1 || d_v < 1) return DA_ERR_INVALID_ARG;
   if (apply_norm && !(norm_eps >= 0.f)) return DA_ERR_INVALID_ARG;
@@ -151,6 +162,7 @@ int diffattn_v1_fwd(const void* q, const void* k, const void* v, void* out, da_d
     a.kv_heads = n_heads;
     a.pairs_per_kv = 1;
     a.causal = causal ? 1 : 0;
+    a.window = window;
     a.lambda = lambda;
     a.apply_norm = apply_norm ? 1 : 0;
     a.norm_weight = norm_weight;
@@ -185,6 +197,7 @@ int diffattn_v1_fwd(const void* q, const void* k, const void* v, void* out, da_d
   P.o_batch = P.v_batch;
   P.n_keys = seqlen;
   P.causal = causal ? 1 : 0;
+  P.window = window;
   P.lens = nullptr;
   P.lambda = lambda;
   P.apply_norm = apply_norm ? 1 : 0;
@@ -197,7 +210,16 @@ int diffattn_v1_fwd(const void* q, const void* k, const void* v, void* out, da_d
 int diffattn_v2_prefill(const void* q, const void* k, const void* v, void* out, da_dtype dtype,
                         int batch, int seqlen, int n_q_heads, int n_kv_heads, int head_dim,
                         const float* lambda, int causal, int* dev_status, void* stream) {
+  return diffattn_v2_prefill_window(q, k, v, out, dtype, batch, seqlen, n_q_heads, n_kv_heads,
+                                    head_dim, lambda, causal, 0, dev_status, stream);
+}
+
+int diffattn_v2_prefill_window(const void* q, const void* k, const void* v, void* out,
+                               da_dtype dtype, int batch, int seqlen, int n_q_heads,
+                               int n_kv_heads, int head_dim, const float* lambda, int causal,
+                               int window, int* dev_status, void* stream) {
   if (!q || !k || !v || !out || !lambda) return DA_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && !causal)) return DA_ERR_INVALID_ARG;
   if (!dtype_ok(dtype)) return DA_ERR_INVALID_ARG;
   if (batch < 1 || seqlen < 1 || n_q_heads < 2 || n_kv_heads < 1 || head_dim < 1)
     return DA_ERR_INVALID_ARG;
@@ -226,6 +248,7 @@ int diffattn_v2_prefill(const void* q, const void* k, const void* v, void* out, 
     a.kv_heads = n_kv_heads;
     a.pairs_per_kv = group / 2;
     a.causal = causal ? 1 : 0;
+    a.window = window;
     a.lambda = lambda;
     a.apply_norm = 0;
     a.norm_weight = nullptr;
@@ -260,6 +283,7 @@ int diffattn_v2_prefill(const void* q, const void* k, const void* v, void* out, 
   P.o_batch = P.o_tok * seqlen;
   P.n_keys = seqlen;
   P.causal = causal ? 1 : 0;
+  P.window = window;
   P.lens = nullptr;
   P.lambda = lambda;
   P.apply_norm = 0;
@@ -283,7 +307,18 @@ int diffattn_v2_decode(const void* q, const void* k_cache, const void* v_cache,
                        const int* cache_lens, int max_len, void* out, da_dtype dtype, int batch,
                        int n_q_heads, int n_kv_heads, int head_dim, const float* lambda,
                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  return diffattn_v2_decode_window(q, k_cache, v_cache, cache_lens, max_len, 0, out, dtype,
+                                   batch, n_q_heads, n_kv_heads, head_dim, lambda, workspace,
+                                   workspace_bytes, dev_status, stream);
+}
+
+int diffattn_v2_decode_window(const void* q, const void* k_cache, const void* v_cache,
+                              const int* cache_lens, int max_len, int window, void* out,
+                              da_dtype dtype, int batch, int n_q_heads, int n_kv_heads,
+                              int head_dim, const float* lambda, void* workspace,
+                              size_t workspace_bytes, int* dev_status, void* stream) {
   if (!q || !k_cache || !v_cache || !out || !lambda) return DA_ERR_INVALID_ARG;
+  if (window < 0) return DA_ERR_INVALID_ARG;
   if (!dtype_ok(dtype)) return DA_ERR_INVALID_ARG;
   if (batch < 1 || max_len < 1 || n_q_heads < 2 || n_kv_heads < 1 || head_dim < 1)
     return DA_ERR_INVALID_ARG;
@@ -297,8 +332,11 @@ int diffattn_v2_decode(const void* q, const void* k_cache, const void* v_cache,
     return DA_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
+  // a window bounds the entries one query reads: plan the splits over that many
+  const int span = (window > 0 && window < max_len) ? window : max_len;
+
   if (dtype == DA_BF16 && v2_decode_fast(n_q_heads, n_kv_heads, head_dim)) {
-    da::V2DecodePlan plan = da::plan_v2_decode(batch, n_kv_heads, max_len, kPlanSMs);
+    da::V2DecodePlan plan = da::plan_v2_decode(batch, n_kv_heads, span, kPlanSMs);
     const size_t need = da::v2_decode_workspace_bytes(plan);
     if (!workspace || workspace_bytes < need) return DA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return DA_ERR_ALIGNMENT;
@@ -309,7 +347,7 @@ int diffattn_v2_decode(const void* q, const void* k_cache, const void* v_cache,
     if (make_tmap_4d(&tk, k_cache, 128, n_kv_heads, max_len, batch, 64, 1, 64, 1) ||
         make_tmap_4d(&tv, v_cache, 128, n_kv_heads, max_len, batch, 64, 1, 64, 1))
       return DA_ERR_CUDA;
-    return cuda_status(da::launch_v2_decode(tk, tv, q, cache_lens, max_len, out, batch,
+    return cuda_status(da::launch_v2_decode(tk, tv, q, cache_lens, max_len, window, out, batch,
                                             n_q_heads, n_kv_heads, lambda, plan, workspace,
                                             dev_status, st));
   }
@@ -338,6 +376,7 @@ int diffattn_v2_decode(const void* q, const void* k_cache, const void* v_cache,
   P.o_batch = (int64_t)(n_q_heads / 2) * head_dim;
   P.n_keys = max_len;
   P.causal = 0;
+  P.window = window;
   P.lens = cache_lens;
   P.lambda = lambda;
   P.apply_norm = 0;
@@ -360,8 +399,21 @@ int diffattn_v1_decode(const void* q, const void* k_cache, const void* v_cache,
                        int n_heads, int d_qk, int d_v, const float* lambda, int apply_norm,
                        const float* norm_weight, float norm_eps, float lambda_init,
                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  return diffattn_v1_decode_window(q, k_cache, v_cache, cache_lens, max_len, 0, out, dtype,
+                                   batch, n_heads, d_qk, d_v, lambda, apply_norm, norm_weight,
+                                   norm_eps, lambda_init, workspace, workspace_bytes, dev_status,
+                                   stream);
+}
+
+int diffattn_v1_decode_window(const void* q, const void* k_cache, const void* v_cache,
+                              const int* cache_lens, int max_len, int window, void* out,
+                              da_dtype dtype, int batch, int n_heads, int d_qk, int d_v,
+                              const float* lambda, int apply_norm, const float* norm_weight,
+                              float norm_eps, float lambda_init, void* workspace,
+                              size_t workspace_bytes, int* dev_status, void* stream) {
   (void)dev_status;  // the kernels used here never wait on asynchronous copies
   if (!q || !k_cache || !v_cache || !out || !lambda) return DA_ERR_INVALID_ARG;
+  if (window < 0) return DA_ERR_INVALID_ARG;
   if (!dtype_ok(dtype)) return DA_ERR_INVALID_ARG;
   if (batch < 1 || max_len < 1 || n_heads < 1 || d_qk < 1 || d_v < 1) return DA_ERR_INVALID_ARG;
   if (apply_norm && !(norm_eps >= 0.f)) return DA_ERR_INVALID_ARG;
@@ -373,12 +425,14 @@ int diffattn_v1_decode(const void* q, const void* k_cache, const void* v_cache,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float post_scale = 1.0f - lambda_init;
 
+  const int span = (window > 0 && window < max_len) ? window : max_len;
+
   if (dtype == DA_BF16 && v1_decode_fast(d_qk, d_v)) {
-    da::V1DecodePlan plan = da::plan_v1_decode(batch, n_heads, max_len, kPlanSMs);
+    da::V1DecodePlan plan = da::plan_v1_decode(batch, n_heads, span, kPlanSMs);
     const size_t need = da::v1_decode_workspace_bytes(plan);
     if (!workspace || workspace_bytes < need) return DA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return DA_ERR_ALIGNMENT;
-    return cuda_status(da::launch_v1_decode(q, k_cache, v_cache, cache_lens, max_len, out,
+    return cuda_status(da::launch_v1_decode(q, k_cache, v_cache, cache_lens, max_len, window, out,
                                             batch, n_heads, lambda, apply_norm ? 1 : 0,
                                             norm_weight, norm_eps, post_scale, plan, workspace,
                                             st));
@@ -408,6 +462,7 @@ int diffattn_v1_decode(const void* q, const void* k_cache, const void* v_cache,
   P.o_batch = (int64_t)n_heads * d_v;
   P.n_keys = max_len;
   P.causal = 0;
+  P.window = window;
   P.lens = cache_lens;
   P.lambda = lambda;
   P.apply_norm = apply_norm ? 1 : 0;

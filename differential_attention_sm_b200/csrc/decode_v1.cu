@@ -37,6 +37,7 @@ struct Params {
   const __nv_bfloat16* vc;  // [B, L, H, 128]
   const int* lens;
   int max_len, H;
+  int window;  // > 0: the query sees only the last `window` valid entries
   int split_len, n_split, n_items;
   float scale_log2;
   float* part_o;   // [n_items][2][128]
@@ -108,7 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1) v1_decode_split_kernel(const Para
   const int h = bh % p.H, b = bh / p.H;
   int len = p.lens ? p.lens[b] : p.max_len;
   len = len < 1 ? 1 : (len > p.max_len ? p.max_len : len);
-  const int t0 = s * p.split_len;
+  const int first = (p.window > 0 && len > p.window) ? len - p.window : 0;
+  const int t0 = first + s * p.split_len;
   const int t1 = min(t0 + p.split_len, len);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
@@ -307,16 +309,17 @@ size_t v1_decode_workspace_bytes(const V1DecodePlan& plan) {
 }
 
 cudaError_t launch_v1_decode(const void* q, const void* k_cache, const void* v_cache,
-                             const int* lens, int max_len, void* out, int batch, int n_heads,
-                             const float* lambda, int apply_norm, const float* norm_weight,
-                             float eps, float post_scale, const V1DecodePlan& plan,
-                             void* workspace, cudaStream_t stream) {
+                             const int* lens, int max_len, int window, void* out, int batch,
+                             int n_heads, const float* lambda, int apply_norm,
+                             const float* norm_weight, float eps, float post_scale,
+                             const V1DecodePlan& plan, void* workspace, cudaStream_t stream) {
   Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.kc = static_cast<const __nv_bfloat16*>(k_cache);
   p.vc = static_cast<const __nv_bfloat16*>(v_cache);
   p.lens = lens;
   p.max_len = max_len;
+  p.window = window;
   p.H = n_heads;
   p.split_len = plan.split_len;
   p.n_split = plan.n_split;

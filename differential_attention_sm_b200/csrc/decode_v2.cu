@@ -49,6 +49,7 @@ struct Params {
   const __nv_bfloat16* q;  // [B, Hq, 128]
   const int* lens;
   int max_len;
+  int window;  // > 0: the query sees only the last `window` valid entries
   int Hq, Hkv, group;
   int split_len, n_split, n_items;
   float scale_log2;
@@ -65,7 +66,8 @@ __device__ __forceinline__ void item_coords(const Params& p, int item, int& b, i
   b = bg / p.Hkv;
   int len = p.lens ? p.lens[b] : p.max_len;
   len = len < 1 ? 1 : (len > p.max_len ? p.max_len : len);
-  t0 = s * p.split_len;
+  const int first = (p.window > 0 && len > p.window) ? len - p.window : 0;
+  t0 = first + s * p.split_len;
   t1 = min(t0 + p.split_len, len);
 }
 
@@ -381,13 +383,15 @@ size_t v2_decode_workspace_bytes(const V2DecodePlan& plan) {
 }
 
 cudaError_t launch_v2_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
-                             const int* lens, int max_len, void* out, int batch, int n_q_heads,
-                             int n_kv_heads, const float* lambda, const V2DecodePlan& plan,
-                             void* workspace, int* dev_status, cudaStream_t stream) {
+                             const int* lens, int max_len, int window, void* out, int batch,
+                             int n_q_heads, int n_kv_heads, const float* lambda,
+                             const V2DecodePlan& plan, void* workspace, int* dev_status,
+                             cudaStream_t stream) {
   Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.lens = lens;
   p.max_len = max_len;
+  p.window = window;
   p.Hq = n_q_heads;
   p.Hkv = n_kv_heads;
   p.group = n_q_heads / n_kv_heads;

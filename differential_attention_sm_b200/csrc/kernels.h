@@ -27,6 +27,7 @@ struct GenericProblem {
   int64_t o_batch, o_tok;
   int n_keys;       // keys per sequence (prefill N, decode max_len)
   int causal;       // prefill: query i sees keys <= i
+  int window;       // > 0: only the last `window` of those keys (prefill and decode)
   const int* lens;  // decode: per-batch valid cache rows, or nullptr
   const float* lambda;
   int apply_norm;
@@ -54,8 +55,9 @@ V2DecodePlan plan_v2_decode_capped(int batch, int n_kv_heads, int max_len, int n
                                    size_t max_bytes);
 size_t v2_decode_workspace_bytes(const V2DecodePlan& plan);
 cudaError_t launch_v2_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
-                             const int* lens, int max_len, void* out, int batch, int n_q_heads,
-                             int n_kv_heads, const float* lambda, const V2DecodePlan& plan,
+                             const int* lens, int max_len, int window, void* out, int batch,
+                             int n_q_heads, int n_kv_heads, const float* lambda,
+                             const V2DecodePlan& plan,
                              void* workspace, int* dev_status, cudaStream_t stream);
 
 // ---- V1 split-KV decode (bf16, d_qk 64, d_v 128) --------------------------
@@ -65,8 +67,9 @@ struct V1DecodePlan {
 V1DecodePlan plan_v1_decode(int batch, int n_heads, int max_len, int num_sms);
 size_t v1_decode_workspace_bytes(const V1DecodePlan& plan);
 cudaError_t launch_v1_decode(const void* q, const void* k_cache, const void* v_cache,
-                             const int* lens, int max_len, void* out, int batch, int n_heads,
-                             const float* lambda, int apply_norm, const float* norm_weight,
+                             const int* lens, int max_len, int window, void* out, int batch,
+                             int n_heads, const float* lambda, int apply_norm,
+                             const float* norm_weight,
                              float eps, float post_scale, const V1DecodePlan& plan,
                              void* workspace, cudaStream_t stream);
 
@@ -87,6 +90,7 @@ struct PrefillArgs {
   int kv_heads;  // V1: heads; V2: n_kv_heads
   int pairs_per_kv;  // V2: group / 2; V1: 1
   int causal;
+  int window;  // > 0 (causal only): row i sees keys (i - window, i]
   const float* lambda;
   int apply_norm;
   const float* norm_weight;

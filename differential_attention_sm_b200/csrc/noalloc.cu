@@ -101,7 +101,7 @@ extern "C" DA_API int diffattn_v2_decode_noalloc(const void* q, const void* k_ca
   if (da::make_tmap_bf16_4d(&tk, k_cache, 128, n_kv_heads, max_len, batch, 64, 1, 64, 1) ||
       da::make_tmap_bf16_4d(&tv, v_cache, 128, n_kv_heads, max_len, batch, 64, 1, 64, 1))
     return DA_ERR_CUDA;
-  cudaError_t e = da::launch_v2_decode(tk, tv, q, cache_lens, max_len, out, batch, n_q_heads,
+  cudaError_t e = da::launch_v2_decode(tk, tv, q, cache_lens, max_len, 0, out, batch, n_q_heads,
                                        n_kv_heads, lambda, plan, scratch, dev_status,
                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : DA_ERR_CUDA;

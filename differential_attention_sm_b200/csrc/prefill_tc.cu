@@ -83,6 +83,7 @@ struct Params {
   int n_qtiles;
   int group;        // heads (V1) / pairs (V2) scheduled together for L2 reuse
   int causal;
+  int window;       // > 0: row i sees keys (i - window, i]
   float scale_log2;
   const float* lambda;
   int apply_norm;
@@ -97,7 +98,8 @@ __device__ __forceinline__ uint32_t s_col(int r, int buf) {
 }
 
 // kForm: 1 = V1 (d_qk 64 per branch, one head), 2 = V2 (d 128 per branch, a head pair).
-template <int kForm>
+// kWindow: sliding-window masking compiled in (p.window > 0) or out.
+template <int kForm, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
     diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
@@ -129,7 +131,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kvh = kForm == 1 ? hh : hh / p.pairs_per_kv;
   const int q0 = mt * kBM;
   const int key_end = p.causal ? min(q0 + kBM, p.seqlen) : p.seqlen;  // keys this tile needs
-  const int n_kv = (key_end + kBN - 1) / kBN;
+  // Sliding window: row i sees keys (i - window, i], so the tile's first row
+  // sets the first key tile it needs.  n_kv counts the tiles processed.
+  const int kv0 = kWindow ? max(0, q0 - p.window + 1) / kBN : 0;
+  const int n_kv = (key_end + kBN - 1) / kBN - kv0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -180,12 +185,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (uint32_t)(j / kStages) & 1u;
         if (!mbar_wait(&bars->k_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], kKVTile);
-        tma_load_4d(sK + s * kKVTile, &tm_k, &bars->k_full[s], 0, kvh, j * kBN, b);
-        tma_load_4d(sK + s * kKVTile + kKVBox, &tm_k, &bars->k_full[s], 64, kvh, j * kBN, b);
+        tma_load_4d(sK + s * kKVTile, &tm_k, &bars->k_full[s], 0, kvh, (kv0 + j) * kBN, b);
+        tma_load_4d(sK + s * kKVTile + kKVBox, &tm_k, &bars->k_full[s], 64, kvh, (kv0 + j) * kBN, b);
         if (!mbar_wait(&bars->v_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
         mbar_arrive_expect_tx(&bars->v_full[s], kKVTile);
-        tma_load_4d(sV + s * kKVTile, &tm_v, &bars->v_full[s], 0, kvh, j * kBN, b);
-        tma_load_4d(sV + s * kKVTile + kKVBox, &tm_v, &bars->v_full[s], 64, kvh, j * kBN, b);
+        tma_load_4d(sV + s * kKVTile, &tm_v, &bars->v_full[s], 0, kvh, (kv0 + j) * kBN, b);
+        tma_load_4d(sV + s * kKVTile + kKVBox, &tm_v, &bars->v_full[s], 64, kvh, (kv0 + j) * kBN, b);
       }
     }
   } else if (warp == 9 || warp == 10) {
@@ -258,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
     const uint32_t t_o = tmem + lane_off + (r == 0 ? kColO1 : kColO2);
     const int lim = p.causal ? min(qrow + 1, p.seqlen) : p.seqlen;  // keys < lim visible
+    const int lo = kWindow ? max(0, qrow - p.window + 1) : 0;         // and keys >= lo
     const float sc = p.scale_log2;
     float m_ref = -INFINITY, l_run = 0.f;
 
@@ -277,11 +283,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
       tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
       tc_wait_ld();
-      const int k0 = j * kBN;
+      const int k0 = (kv0 + j) * kBN;
       if (k0 + kBN > lim) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
+      }
+      if (kWindow && k0 < lo) {  // window start (a row may see none of this tile)
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (k0 + c < lo) sr[c] = __float_as_uint(-INFINITY);
       }
       // row maximum: 3-input max over 8 independent chains
       float m8[8];
@@ -453,6 +464,7 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   grp = grp < a.pairs_per_kv ? a.pairs_per_kv : grp;
   p.group = grp > bh_count ? bh_count : grp;
   p.causal = a.causal;
+  p.window = a.window;
   const double d = a.form == 1 ? 64.0 : 128.0;  // width of one branch's query
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(d));
   p.lambda = a.lambda;
@@ -465,7 +477,11 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
   const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +
                    4 * kBM * (int)sizeof(float) + 64;
-  auto kern = a.form == 1 ? diffattn_prefill_tc_kernel<1> : diffattn_prefill_tc_kernel<2>;
+  const bool win = a.window > 0;
+  auto kern = a.form == 1 ? (win ? diffattn_prefill_tc_kernel<1, true>
+                                 : diffattn_prefill_tc_kernel<1, false>)
+                          : (win ? diffattn_prefill_tc_kernel<2, true>
+                                 : diffattn_prefill_tc_kernel<2, false>);
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

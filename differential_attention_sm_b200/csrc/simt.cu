@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(32 * GEN_WARPS) generic_kernel(GenericProblem 
   } else {
     n_keys = P.causal ? i + 1 : P.n_keys;
   }
+  // sliding window: only the last `window` of the visible keys
+  const int key0 = (P.window > 0 && n_keys > P.window) ? n_keys - P.window : 0;
 
   for (int c = lane; c < P.d; c += 32) {
     qs[wib][0][c] = ld(q + c);
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(32 * GEN_WARPS) generic_kernel(GenericProblem 
 
   // pass 1: row maxima of both score rows
   float m1 = -INFINITY, m2 = -INFINITY;
-  for (int j = lane; j < n_keys; j += 32) {
+  for (int j = key0 + lane; j < n_keys; j += 32) {
     float s1, s2;
     scores(j, s1, s2);
     m1 = fmaxf(m1, s1);
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(32 * GEN_WARPS) generic_kernel(GenericProblem 
   }
   // pass 2: softmax denominators
   float l1 = 0.f, l2 = 0.f;
-  for (int j = lane; j < n_keys; j += 32) {
+  for (int j = key0 + lane; j < n_keys; j += 32) {
     float s1, s2;
     scores(j, s1, s2);
     l1 += expf(s1 - m1);
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(32 * GEN_WARPS) generic_kernel(GenericProblem 
   float acc[GEN_MAX_DV / 32];
 #pragma unroll
   for (int t = 0; t < GEN_MAX_DV / 32; ++t) acc[t] = 0.f;
-  for (int j0 = 0; j0 < n_keys; j0 += 32) {
+  for (int j0 = key0; j0 < n_keys; j0 += 32) {
     const int j = j0 + lane;
     float w = 0.f;
     if (j < n_keys) {

@@ -72,6 +72,13 @@ WORKLOADS = {
                                L=32768, Hq=64, Hkv=8, d=128),
     "v1_decode_bf16": Workload("v1_decode_bf16", "v1_decode", BF16, 4, B=64,
                                L=32768, H=32, d=64, dv=128, layer=12),
+    # sliding-window variants (hybrid DIFF + sliding-window models): the V2
+    # prefill and decode shapes above with a 1024-key / 4096-entry window
+    "v2_prefill_window_bf16": Workload("v2_prefill_window_bf16", "v2", BF16, 3, B=2, N=8192,
+                                       Hq=32, Hkv=8, d=128, causal=True,
+                                       extra={"window": 1024}),
+    "v2_decode_window_bf16": Workload("v2_decode_window_bf16", "v2_decode", BF16, 4, B=64,
+                                      L=32768, Hq=64, Hkv=8, d=128, extra={"window": 4096}),
     # noise-cancellation sweep: 3 noise amplitudes x 2 branch-noise correlations,
     # lambda 0, 0.1, ..., 1.0 as 11 heads, run through the V1 decode kernel
     "snr_v1_decode": Workload("snr_v1_decode", "snr", BF16, 5, B=48, L=1024, H=11,

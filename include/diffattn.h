@@ -197,6 +197,43 @@ DA_API int diffattn_v1_decode(const void* q, const void* k_cache, const void* v_
                        float lambda_init, void* workspace, size_t workspace_bytes,
                        int* dev_status, void* stream);
 
+/* ---- Sliding-window variants ---------------------------------------------
+ * The lesson "Atención Diferencial (V2)", section "Úselo", names models that
+ * combine differential attention with sliding-window attention.  Reading:
+ * with window W >= 1, query i sees only keys j with i - W < j <= i, in both
+ * branches (prefill requires causal = 1), and a decode query sees the last
+ * W of its len_b cache entries.  window = 0 is the unwindowed operator (the
+ * functions above are these with window 0).  Every other argument, layout,
+ * kernel choice and error is as for the function without "_window"; a
+ * negative window, or window > 0 with causal = 0, is DA_ERR_INVALID_ARG.
+ * The decode variants plan their cache splits over min(window, max_len)
+ * entries, so their workspace is diffattn_v2_decode_workspace_size (or
+ * diffattn_v1_decode_workspace_size) evaluated at that length. */
+DA_API int diffattn_v1_fwd_window(const void* q, const void* k, const void* v, void* out,
+                                  da_dtype dtype, int batch, int seqlen, int n_heads, int d_qk,
+                                  int d_v, const float* lambda, int causal, int window,
+                                  int apply_norm, const float* norm_weight, float norm_eps,
+                                  float lambda_init, int* dev_status, void* stream);
+
+DA_API int diffattn_v2_prefill_window(const void* q, const void* k, const void* v, void* out,
+                                      da_dtype dtype, int batch, int seqlen, int n_q_heads,
+                                      int n_kv_heads, int head_dim, const float* lambda,
+                                      int causal, int window, int* dev_status, void* stream);
+
+DA_API int diffattn_v2_decode_window(const void* q, const void* k_cache, const void* v_cache,
+                                     const int* cache_lens, int max_len, int window, void* out,
+                                     da_dtype dtype, int batch, int n_q_heads, int n_kv_heads,
+                                     int head_dim, const float* lambda, void* workspace,
+                                     size_t workspace_bytes, int* dev_status, void* stream);
+
+DA_API int diffattn_v1_decode_window(const void* q, const void* k_cache, const void* v_cache,
+                                     const int* cache_lens, int max_len, int window, void* out,
+                                     da_dtype dtype, int batch, int n_heads, int d_qk, int d_v,
+                                     const float* lambda, int apply_norm,
+                                     const float* norm_weight, float norm_eps, float lambda_init,
+                                     void* workspace, size_t workspace_bytes, int* dev_status,
+                                     void* stream);
+
 #ifdef __cplusplus
 }
 #endif

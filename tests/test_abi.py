@@ -133,3 +133,36 @@ def test_product_path_has_no_oracle_dependency():
                 text = open(os.path.join(dirpath, fn), encoding="utf-8").read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
                 assert "diffattn_oracle" not in text, fn
+
+
+def test_window_variants_host_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    f = lib.diffattn_v1_fwd_window
+    ok = [A, A, A, A, b.DA_BF16, 1, 128, 1, 64, 128, A, 1, 16, 1, None, 1e-5, 0.2, None, None]
+    bad = list(ok); bad[12] = -1                 # negative window
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[11] = 0                  # a window needs causal masking
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[1] = U
+    assert f(*bad) == b.DA_ERR_ALIGNMENT
+    g = lib.diffattn_v2_prefill_window
+    ok = [A, A, A, A, b.DA_BF16, 2, 256, 32, 8, 128, A, 1, 64, None, None]
+    bad = list(ok); bad[12] = -5
+    assert g(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[11] = 0
+    assert g(*bad) == b.DA_ERR_INVALID_ARG
+    # windowed decode plans over min(window, max_len) entries
+    ws_w = b.diffattn_v2_decode_workspace_size(64, 64, 8, 128, 4096)
+    h = lib.diffattn_v2_decode_window
+    args = [A, A, A, None, 32768, 4096, A, b.DA_BF16, 64, 64, 8, 128, A, A, ws_w - 16,
+            None, None]
+    assert h(*args) == b.DA_ERR_WORKSPACE
+    args[5] = -1
+    assert h(*args) == b.DA_ERR_INVALID_ARG
+    k = lib.diffattn_v1_decode_window
+    ws1 = b.diffattn_v1_decode_workspace_size(2, 4, 64, 128, 100)
+    args = [A, A, A, None, 1000, 100, A, b.DA_BF16, 2, 4, 64, 128, A, 1, None, 1e-5, 0.2, A,
+            ws1 - 1, None, None]
+    assert k(*args) == b.DA_ERR_WORKSPACE
+    args[5] = -2
+    assert k(*args) == b.DA_ERR_INVALID_ARG
