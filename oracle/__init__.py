@@ -15,4 +15,7 @@ from .oracle import (  # noqa: F401
     n_threads,
     v1_query_weights,
     snr,
+    v1_bwd,
+    v2_bwd,
+    lambda_params_bwd,
 )

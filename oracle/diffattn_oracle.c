@@ -363,3 +363,237 @@ int oracle_snr(const double *w, int64_t n, int64_t pos, double *out)
     *out = rms > 0.0 ? w[pos] / rms : (w[pos] > 0.0 ? INFINITY : (w[pos] < 0.0 ? -INFINITY : NAN));
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------
+ * Backward pass (gradients of a scalar loss with respect to every input).
+ * The pages give the forward only; the gradients below are those of that
+ * forward, obtained with the chain rule step by step (the "reading" is
+ * only that lambda, and in V1 the norm gain g, are trainable: the glossary
+ * page calls lambda learned, from four re-parameterised vectors).
+ * ------------------------------------------------------------------------ */
+
+/* One query row: given d(loss)/d(o) for the pre-norm output o (= do), the
+ * row's softmax maps a1, a2 (over n_keys keys starting at k1/k2/v), add the
+ * row's contributions to dq (this row), dk, dv (those keys) and return
+ * d(loss)/d(lambda) of this row.
+ *   o = sum_j (a1_j - lambda a2_j) v_j          (forward, [G])
+ *   dv_j   += (a1_j - lambda a2_j) do
+ *   dlambda = -sum_c do_c (sum_j a2_j v_j[c])
+ *   branch r with do_r = do (r = 1) or -lambda do (r = 2):
+ *     dp_j = do_r . v_j,   D = sum_j a_r,j dp_j,   ds_j = a_r,j (dp_j - D)
+ *     dq_r += sum_j ds_j k_r,j / sqrt(d),   dk_r,j += ds_j q_r / sqrt(d)
+ */
+static double diff_attention_row_bwd(const float *q1, const float *q2,
+                                     const float *k1, const float *k2, int64_t k_stride,
+                                     const float *v, int64_t v_stride, int64_t n_keys,
+                                     int d, int dv, double lambda,
+                                     const double *a1, const double *a2, const double *dout,
+                                     double *dq1, double *dq2,
+                                     double *dk1, double *dk2, int64_t dk_stride,
+                                     double *dvv, int64_t dv_stride)
+{
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    double dlam = 0.0;
+    for (int64_t j = 0; j < n_keys; ++j) {
+        const float *vj = v + j * v_stride;
+        double dp = 0.0;
+        for (int c = 0; c < dv; ++c) dp += dout[c] * (double)vj[c];
+        dlam -= a2[j] * dp;
+        double wj = a1[j] - lambda * a2[j];
+        double *dvj = dvv + j * dv_stride;
+        for (int c = 0; c < dv; ++c) dvj[c] += wj * dout[c];
+    }
+    for (int r = 0; r < 2; ++r) {
+        const double *a = r == 0 ? a1 : a2;
+        const double coef = r == 0 ? 1.0 : -lambda;
+        const float *qr = r == 0 ? q1 : q2;
+        const float *kr = r == 0 ? k1 : k2;
+        double *dqr = r == 0 ? dq1 : dq2;
+        double *dkr = r == 0 ? dk1 : dk2;
+        double D = 0.0;
+        for (int64_t j = 0; j < n_keys; ++j) {
+            const float *vj = v + j * v_stride;
+            double dp = 0.0;
+            for (int c = 0; c < dv; ++c) dp += coef * dout[c] * (double)vj[c];
+            D += a[j] * dp;
+        }
+        for (int64_t j = 0; j < n_keys; ++j) {
+            const float *vj = v + j * v_stride;
+            double dp = 0.0;
+            for (int c = 0; c < dv; ++c) dp += coef * dout[c] * (double)vj[c];
+            const double ds = a[j] * (dp - D) * inv_sqrt_d;
+            const float *kj = kr + j * k_stride;
+            double *dkj = dkr + j * dk_stride;
+            for (int c = 0; c < d; ++c) {
+                dqr[c] += ds * (double)kj[c];
+                dkj[c] += ds * (double)qr[c];
+            }
+        }
+    }
+    return dlam;
+}
+
+/* The two softmax maps of one row (as in diff_attention_row, without V). */
+static void softmax_maps(const float *q1, const float *q2, const float *k1, const float *k2,
+                         int64_t k_stride, int64_t n_keys, int d, double *a1, double *a2)
+{
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    for (int64_t j = 0; j < n_keys; ++j) {
+        double s1 = 0.0, s2 = 0.0;
+        for (int c = 0; c < d; ++c) {
+            s1 += (double)q1[c] * (double)k1[j * k_stride + c];
+            s2 += (double)q2[c] * (double)k2[j * k_stride + c];
+        }
+        a1[j] = s1 * inv_sqrt_d;
+        a2[j] = s2 * inv_sqrt_d;
+    }
+    softmax_row(a1, n_keys);
+    softmax_row(a2, n_keys);
+}
+
+/*
+ * V1 backward over the whole problem.  Inputs as oracle_v1_rows plus
+ * dout [B, N, H, dv] (gradient of the loss with respect to the output).
+ * Outputs (double, overwritten): dq, dk [B, N, H, 2d]; dvv [B, N, H, dv];
+ * dlambda [H] (summed over batch and rows); dnorm_weight [dv] (may be NULL;
+ * only with apply_norm).  With the norm,
+ *   y = o * g * c / r,  r = sqrt(mean(o^2) + eps),  c = 1 - lambda_init
+ *   do_k = (c / r) * (g_k dy_k - o_k * sum_m(g_m dy_m o_m) / (dv r^2))
+ *   dg_k += dy_k o_k c / r.
+ */
+int oracle_v1_bwd(const float *q, const float *k, const float *v, const float *dout,
+                  int B, int N, int H, int d, int dv, const double *lambda,
+                  int causal, int window, int apply_norm, const float *norm_weight,
+                  double eps, double lambda_init,
+                  double *dq, double *dk, double *dvv, double *dlambda, double *dnorm_weight)
+{
+    if (!q || !k || !v || !dout || !lambda || !dq || !dk || !dvv || !dlambda)
+        return ORACLE_ERR_ARG;
+    if (B < 1 || N < 1 || H < 1 || d < 1 || dv < 1) return ORACLE_ERR_ARG;
+    double *a1 = (double *)malloc(sizeof(double) * (size_t)N);
+    double *a2 = (double *)malloc(sizeof(double) * (size_t)N);
+    double *o = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *g_o = (double *)malloc(sizeof(double) * (size_t)dv);
+    if (!a1 || !a2 || !o || !g_o) { free(a1); free(a2); free(o); free(g_o); return ORACLE_ERR_NOMEM; }
+    const int64_t row_qk = 2LL * d, tok_qk = (int64_t)H * row_qk, tok_v = (int64_t)H * dv;
+    for (int64_t t = 0; t < (int64_t)B * N * tok_qk; ++t) { dq[t] = 0.0; dk[t] = 0.0; }
+    for (int64_t t = 0; t < (int64_t)B * N * tok_v; ++t) dvv[t] = 0.0;
+    for (int h = 0; h < H; ++h) dlambda[h] = 0.0;
+    if (dnorm_weight) for (int c = 0; c < dv; ++c) dnorm_weight[c] = 0.0;
+    const double cpost = 1.0 - lambda_init;
+    for (int b = 0; b < B; ++b)
+        for (int i = 0; i < N; ++i)
+            for (int h = 0; h < H; ++h) {
+                int64_t n_keys = causal ? (int64_t)i + 1 : (int64_t)N;
+                const int64_t first = window_start(n_keys, window);
+                const int64_t tq = ((int64_t)b * N + i) * tok_qk + (int64_t)h * row_qk;
+                const int64_t k0 = ((int64_t)b * N + first) * tok_qk + (int64_t)h * row_qk;
+                const int64_t v0 = ((int64_t)b * N + first) * tok_v + (int64_t)h * dv;
+                const int64_t nk = n_keys - first;
+                softmax_maps(q + tq, q + tq + d, k + k0, k + k0 + d, tok_qk, nk, d, a1, a2);
+                const float *dy = dout + ((int64_t)b * N + i) * tok_v + (int64_t)h * dv;
+                double *gro = g_o;   /* d(loss)/d(o) */
+                if (apply_norm) {
+                    for (int c = 0; c < dv; ++c) {
+                        double s = 0.0;
+                        for (int64_t j = 0; j < nk; ++j)
+                            s += (a1[j] - lambda[h] * a2[j]) * (double)v[v0 + j * tok_v + c];
+                        o[c] = s;
+                    }
+                    double ss = 0.0;
+                    for (int c = 0; c < dv; ++c) ss += o[c] * o[c];
+                    const double r = sqrt(ss / (double)dv + eps);
+                    double gdo = 0.0;
+                    for (int c = 0; c < dv; ++c) {
+                        const double gc = norm_weight ? (double)norm_weight[c] : 1.0;
+                        gdo += gc * (double)dy[c] * o[c];
+                    }
+                    for (int c = 0; c < dv; ++c) {
+                        const double gc = norm_weight ? (double)norm_weight[c] : 1.0;
+                        gro[c] = (cpost / r) * (gc * (double)dy[c] - o[c] * gdo / ((double)dv * r * r));
+                        if (dnorm_weight) dnorm_weight[c] += (double)dy[c] * o[c] * cpost / r;
+                    }
+                } else {
+                    for (int c = 0; c < dv; ++c) gro[c] = (double)dy[c];
+                }
+                dlambda[h] += diff_attention_row_bwd(
+                    q + tq, q + tq + d, k + k0, k + k0 + d, tok_qk, v + v0, tok_v, nk, d, dv,
+                    lambda[h], a1, a2, gro, dq + tq, dq + tq + d, dk + k0, dk + k0 + d, tok_qk,
+                    dvv + v0, tok_v);
+            }
+    free(a1); free(a2); free(o); free(g_o);
+    return ORACLE_OK;
+}
+
+/*
+ * V2 backward over the whole problem.  Inputs as oracle_v2_rows plus
+ * dout [B, N, Hq/2, d].  Outputs (double, overwritten): dq [B, N, Hq, d];
+ * dk, dvv [B, N, Hkv, d] (summed over the pairs that share a KV head);
+ * dlambda [Hq/2] (summed over batch and rows).
+ */
+int oracle_v2_bwd(const float *q, const float *k, const float *v, const float *dout,
+                  int B, int N, int Hq, int Hkv, int d, const double *lambda,
+                  int causal, int window,
+                  double *dq, double *dk, double *dvv, double *dlambda)
+{
+    if (!q || !k || !v || !dout || !lambda || !dq || !dk || !dvv || !dlambda)
+        return ORACLE_ERR_ARG;
+    if (B < 1 || N < 1 || Hq < 2 || Hkv < 1 || d < 1) return ORACLE_ERR_ARG;
+    if (Hq % 2 != 0 || Hq % Hkv != 0 || (Hq / Hkv) % 2 != 0) return ORACLE_ERR_ARG;
+    const int P = Hq / 2, group = Hq / Hkv;
+    double *a1 = (double *)malloc(sizeof(double) * (size_t)N);
+    double *a2 = (double *)malloc(sizeof(double) * (size_t)N);
+    double *gro = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!a1 || !a2 || !gro) { free(a1); free(a2); free(gro); return ORACLE_ERR_NOMEM; }
+    const int64_t tok_q = (int64_t)Hq * d, tok_kv = (int64_t)Hkv * d, tok_o = (int64_t)P * d;
+    for (int64_t t = 0; t < (int64_t)B * N * tok_q; ++t) dq[t] = 0.0;
+    for (int64_t t = 0; t < (int64_t)B * N * tok_kv; ++t) { dk[t] = 0.0; dvv[t] = 0.0; }
+    for (int p = 0; p < P; ++p) dlambda[p] = 0.0;
+    for (int b = 0; b < B; ++b)
+        for (int i = 0; i < N; ++i)
+            for (int p = 0; p < P; ++p) {
+                const int g = (2 * p) / group;
+                int64_t n_keys = causal ? (int64_t)i + 1 : (int64_t)N;
+                const int64_t first = window_start(n_keys, window);
+                const int64_t nk = n_keys - first;
+                const int64_t qa = ((int64_t)b * N + i) * tok_q + (int64_t)(2 * p) * d;
+                const int64_t qb = qa + d;
+                const int64_t k0 = ((int64_t)b * N + first) * tok_kv + (int64_t)g * d;
+                softmax_maps(q + qa, q + qb, k + k0, k + k0, tok_kv, nk, d, a1, a2);
+                const float *dy = dout + ((int64_t)b * N + i) * tok_o + (int64_t)p * d;
+                for (int c = 0; c < d; ++c) gro[c] = (double)dy[c];
+                dlambda[p] += diff_attention_row_bwd(
+                    q + qa, q + qb, k + k0, k + k0, tok_kv, v + k0, tok_kv, nk, d, d,
+                    lambda[p], a1, a2, gro, dq + qa, dq + qb, dk + k0, dk + k0, tok_kv,
+                    dvv + k0, tok_kv);
+            }
+    free(a1); free(a2); free(gro);
+    return ORACLE_OK;
+}
+
+/* Gradients of the four lambda vectors from d(loss)/d(lambda):
+ *   lambda = exp(lq1.lk1) - exp(lq2.lk2) + lambda_init   ([G], [L])
+ *   dlq1 = dl e1 lk1, dlk1 = dl e1 lq1, dlq2 = -dl e2 lk2, dlk2 = -dl e2 lq2. */
+int oracle_lambda_params_bwd(const float *lq1, const float *lk1, const float *lq2,
+                             const float *lk2, int H, int dim, const double *dlambda,
+                             double *dlq1, double *dlk1, double *dlq2, double *dlk2)
+{
+    if (!lq1 || !lk1 || !lq2 || !lk2 || !dlambda || !dlq1 || !dlk1 || !dlq2 || !dlk2 ||
+        H < 1 || dim < 1)
+        return ORACLE_ERR_ARG;
+    for (int h = 0; h < H; ++h) {
+        double dot1 = 0.0, dot2 = 0.0;
+        for (int c = 0; c < dim; ++c) {
+            dot1 += (double)lq1[h * dim + c] * (double)lk1[h * dim + c];
+            dot2 += (double)lq2[h * dim + c] * (double)lk2[h * dim + c];
+        }
+        const double e1 = exp(dot1) * dlambda[h], e2 = exp(dot2) * dlambda[h];
+        for (int c = 0; c < dim; ++c) {
+            dlq1[h * dim + c] = e1 * (double)lk1[h * dim + c];
+            dlk1[h * dim + c] = e1 * (double)lq1[h * dim + c];
+            dlq2[h * dim + c] = -e2 * (double)lk2[h * dim + c];
+            dlk2[h * dim + c] = -e2 * (double)lq2[h * dim + c];
+        }
+    }
+    return ORACLE_OK;
+}

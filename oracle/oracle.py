@@ -69,6 +69,19 @@ def _load():
         lib.oracle_v2_decode_rows.argtypes = [
             _f32p, _f32p, _f32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, _f64p, _i64p, ctypes.c_int64, _f64p]
+        lib.oracle_v1_bwd.restype = ctypes.c_int
+        lib.oracle_v1_bwd.argtypes = [
+            _f32p, _f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, _f64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p,
+            ctypes.c_double, ctypes.c_double, _f64p, _f64p, _f64p, _f64p, _f64p]
+        lib.oracle_v2_bwd.restype = ctypes.c_int
+        lib.oracle_v2_bwd.argtypes = [
+            _f32p, _f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, _f64p, ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p, _f64p]
+        lib.oracle_lambda_params_bwd.restype = ctypes.c_int
+        lib.oracle_lambda_params_bwd.argtypes = [
+            _f32p, _f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p,
+            _f64p, _f64p]
         lib.oracle_snr.restype = ctypes.c_int
         lib.oracle_snr.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64, _f64p]
         lib.oracle_v1_decode_rows.restype = ctypes.c_int
@@ -266,3 +279,58 @@ def snr(weights, pos: int):
             raise ValueError("oracle_snr status %d" % rc)
         out[i] = one[0]
     return out.reshape(w.shape[:-1])
+
+
+def v1_bwd(q, k, v, dout, lam, *, causal: bool, window: int = 0, apply_norm: bool = False,
+           norm_weight=None, eps: float = 1e-5, lambda_init_value: float = 0.0):
+    """Gradients of sum(out * dout) for the V1 forward: dict with dq, dk
+    [B, N, H, 2d], dv [B, N, H, dv], dlambda [H] and, with the norm,
+    dnorm_weight [dv] (all double)."""
+    qf, kf, vf, gf = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, N, H, d2 = qf.shape
+    dv = vf.shape[-1]
+    lamd = np.ascontiguousarray(np.asarray(lam, dtype=np.float64).reshape(-1))
+    g = _f32(norm_weight) if norm_weight is not None else None
+    res = {"dq": np.empty(qf.shape), "dk": np.empty(kf.shape), "dv": np.empty(vf.shape),
+           "dlambda": np.empty(H), "dnorm_weight": np.empty(dv) if apply_norm else None}
+    rc = _load().oracle_v1_bwd(
+        _ptr(qf, _f32p), _ptr(kf, _f32p), _ptr(vf, _f32p), _ptr(gf, _f32p), B, N, H, d2 // 2,
+        dv, _ptr(lamd, _f64p), int(causal), int(window), int(apply_norm), _ptr(g, _f32p),
+        float(eps), float(lambda_init_value), _ptr(res["dq"], _f64p), _ptr(res["dk"], _f64p),
+        _ptr(res["dv"], _f64p), _ptr(res["dlambda"], _f64p), _ptr(res["dnorm_weight"], _f64p))
+    if rc != 0:
+        raise ValueError("oracle_v1_bwd status %d" % rc)
+    return res
+
+
+def v2_bwd(q, k, v, dout, lam, *, causal: bool, window: int = 0):
+    """Gradients of sum(out * dout) for the V2 forward: dict with dq
+    [B, N, Hq, d], dk, dv [B, N, Hkv, d], dlambda [Hq/2] (double)."""
+    qf, kf, vf, gf = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, N, Hq, d = qf.shape
+    Hkv = kf.shape[2]
+    lamd = np.ascontiguousarray(np.asarray(lam, dtype=np.float64).reshape(-1))
+    res = {"dq": np.empty(qf.shape), "dk": np.empty(kf.shape), "dv": np.empty(vf.shape),
+           "dlambda": np.empty(Hq // 2)}
+    rc = _load().oracle_v2_bwd(
+        _ptr(qf, _f32p), _ptr(kf, _f32p), _ptr(vf, _f32p), _ptr(gf, _f32p), B, N, Hq, Hkv, d,
+        _ptr(lamd, _f64p), int(causal), int(window), _ptr(res["dq"], _f64p),
+        _ptr(res["dk"], _f64p), _ptr(res["dv"], _f64p), _ptr(res["dlambda"], _f64p))
+    if rc != 0:
+        raise ValueError("oracle_v2_bwd status %d" % rc)
+    return res
+
+
+def lambda_params_bwd(lq1, lk1, lq2, lk2, dlambda):
+    """Gradients of the four [H, dim] lambda vectors (double) given
+    d(loss)/d(lambda) [H]."""
+    a, b, c, d = (_f32(x) for x in (lq1, lk1, lq2, lk2))
+    H, dim = a.shape
+    dl = np.ascontiguousarray(np.asarray(dlambda, dtype=np.float64).reshape(-1))
+    outs = [np.empty((H, dim)) for _ in range(4)]
+    rc = _load().oracle_lambda_params_bwd(
+        _ptr(a, _f32p), _ptr(b, _f32p), _ptr(c, _f32p), _ptr(d, _f32p), H, dim,
+        _ptr(dl, _f64p), *(_ptr(o, _f64p) for o in outs))
+    if rc != 0:
+        raise ValueError("oracle_lambda_params_bwd status %d" % rc)
+    return dict(zip(("dlq1", "dlk1", "dlq2", "dlk2"), outs))

@@ -36,6 +36,17 @@ MUTANTS = [
      "        if (w) w += first;\n        diff_attention_row(qrow", "window not applied to values (V1)"),
     ("        const int64_t first = window_start(len, window);\n        kb += first * tok_kv;",
      "        const int64_t first = 0;\n        kb += first * tok_kv;", "window ignored in V2 decode"),
+    ("        dlam -= a2[j] * dp;", "        dlam += a2[j] * dp;", "backward: lambda gradient sign"),
+    ("const double ds = a[j] * (dp - D) * inv_sqrt_d;", "const double ds = a[j] * dp * inv_sqrt_d;",
+     "backward: softmax Jacobian without the row term"),
+    ("const double coef = r == 0 ? 1.0 : -lambda;", "const double coef = r == 0 ? 1.0 : lambda;",
+     "backward: branch-2 upstream sign"),
+    ("gro[c] = (cpost / r) * (gc * (double)dy[c] - o[c] * gdo / ((double)dv * r * r));",
+     "gro[c] = (cpost / r) * (gc * (double)dy[c]);", "backward: norm Jacobian without the RMS term"),
+    ("        for (int c = 0; c < dv; ++c) dvj[c] += wj * dout[c];",
+     "        for (int c = 0; c < dv; ++c) dvj[c] += a1[j] * dout[c];", "backward: dV from map 1 only"),
+    ("            dlk2[h * dim + c] = -e2 * (double)lq2[h * dim + c];",
+     "            dlk2[h * dim + c] = -e2 * (double)lk2[h * dim + c];", "backward: lambda vector swap"),
 ]
 
 

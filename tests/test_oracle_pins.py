@@ -466,3 +466,113 @@ def test_window_decode_equals_decode_over_the_last_entries():
                               x1["v_cache"][b:b + 1, n - W:n], lam1, np.arange(3),
                               apply_norm=True, lambda_init_value=0.5)
         assert np.abs(o1[b] - r1).max() < 1e-13
+
+
+# --------------------------------------------------------------------------
+# Backward pass: gradients of the forward defined by [G] / [L], pinned to
+# float64 torch autograd of an SDPA-based statement of the same forward and
+# to central finite differences of the oracle's own (pinned) forward.
+# --------------------------------------------------------------------------
+def _torch_v1_forward(q, k, v, lam, g, causal, window, apply_norm, lam_init, eps=1e-5):
+    d = q.shape[-1] // 2
+    N = q.shape[1]
+    mask = None
+    if causal:
+        mask = _band_mask(N, window if window > 0 else N)
+
+    def att(qh, kh):
+        qt, kt, vt = (x.permute(0, 2, 1, 3) for x in (qh, kh, v))
+        return F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask).permute(0, 2, 1, 3)
+
+    o = att(q[..., :d], k[..., :d]) - lam.view(1, 1, -1, 1) * att(q[..., d:], k[..., d:])
+    if apply_norm:
+        o = F.rms_norm(o, (o.shape[-1],), weight=g, eps=eps) * (1.0 - lam_init)
+    return o
+
+
+@pytest.mark.parametrize("causal,window,apply_norm", [(True, 0, True), (False, 0, False),
+                                                       (True, 6, True), (True, 0, False)])
+def test_v1_backward_matches_float64_autograd(causal, window, apply_norm):
+    B, N, H, d, dv = 2, 17, 3, 8, 16
+    q, k, v = rand(B, N, H, 2 * d, seed=80), rand(B, N, H, 2 * d, seed=81), rand(B, N, H, dv, seed=82)
+    dout = rand(B, N, H, dv, seed=83)
+    lam = torch.tensor([0.8, -0.25, 1.3], dtype=torch.float64)
+    g = (1.0 + 0.3 * rand(dv, seed=84)).double()
+    li = 0.55
+    res = O.v1_bwd(q, k, v, dout, lam, causal=causal, window=window, apply_norm=apply_norm,
+                   norm_weight=g.float() if apply_norm else None, lambda_init_value=li)
+    qt, kt, vt = (x.double().requires_grad_(True) for x in (q, k, v))
+    lt = lam.clone().requires_grad_(True)
+    gt = g.clone().requires_grad_(True)
+    y = _torch_v1_forward(qt, kt, vt, lt, gt, causal, window, apply_norm, li)
+    (y * dout.double()).sum().backward()
+    for name, ref in (("dq", qt.grad), ("dk", kt.grad), ("dv", vt.grad), ("dlambda", lt.grad)):
+        assert np.abs(res[name] - ref.numpy()).max() < 1e-11, name
+    if apply_norm:
+        assert np.abs(res["dnorm_weight"] - gt.grad.numpy()).max() < 1e-11
+
+
+@pytest.mark.parametrize("causal,window", [(True, 0), (False, 0), (True, 9)])
+def test_v2_backward_matches_float64_autograd(causal, window):
+    B, N, Hq, Hkv, d = 1, 19, 8, 2, 8
+    x = I.v2_inputs(B, N, Hq, Hkv, d, seed=85, dtype=torch.float32)
+    dout = rand(B, N, Hq // 2, d, seed=86)
+    res = O.v2_bwd(x["q"], x["k"], x["v"], dout, x["lam"], causal=causal, window=window)
+    qt, kt, vt = (x[n].double().requires_grad_(True) for n in ("q", "k", "v"))
+    lt = x["lam"].double().clone().requires_grad_(True)
+    mask = _band_mask(N, window if window > 0 else N) if causal else None
+
+    def att(qh):
+        return F.scaled_dot_product_attention(qh.permute(0, 2, 1, 3), kt.permute(0, 2, 1, 3),
+                                              vt.permute(0, 2, 1, 3), attn_mask=mask,
+                                              enable_gqa=True).permute(0, 2, 1, 3)
+
+    y = att(qt[:, :, 0::2]) - lt.view(1, 1, -1, 1) * att(qt[:, :, 1::2])
+    (y * dout.double()).sum().backward()
+    for name, ref in (("dq", qt.grad), ("dk", kt.grad), ("dv", vt.grad), ("dlambda", lt.grad)):
+        assert np.abs(res[name] - ref.numpy()).max() < 1e-11, name
+
+
+def test_v1_backward_matches_finite_differences_of_the_oracle():
+    B, N, H, d, dv = 1, 6, 2, 3, 4
+    q, k, v = rand(B, N, H, 2 * d, seed=87).double(), rand(B, N, H, 2 * d, seed=88).double(), rand(B, N, H, dv, seed=89).double()
+    dout = rand(B, N, H, dv, seed=90).double()
+    lam = np.array([0.7, -0.4])
+    li, eps_n = 0.3, 1e-5
+    rows = all_rows_v1(B, N, H)
+
+    def loss(qq, kk, vv, ll):
+        o = O.v1_rows(qq.float(), kk.float(), vv.float(), ll, rows, causal=True,
+                      apply_norm=True, lambda_init_value=li, eps=eps_n)
+        return float((o * dout.reshape(-1, dv).numpy()).sum())
+
+    # float32 inputs: step sizes well above float32 resolution, tolerance to match
+    res = O.v1_bwd(q, k, v, dout, lam, causal=True, apply_norm=True, lambda_init_value=li)
+    h = 1e-2
+    for name, t in (("dq", q), ("dk", k), ("dv", v)):
+        for idx in [(0, 0, 0, 0), (0, 3, 1, 2), (0, 5, 1, t.shape[-1] - 1)]:
+            tp, tm = t.clone(), t.clone()
+            tp[idx] += h
+            tm[idx] -= h
+            args_p = {"dq": (tp, k, v), "dk": (q, tp, v), "dv": (q, k, tp)}[name]
+            args_m = {"dq": (tm, k, v), "dk": (q, tm, v), "dv": (q, k, tm)}[name]
+            fd = (loss(*args_p, lam) - loss(*args_m, lam)) / (2 * h)
+            assert res[name][idx] == pytest.approx(fd, rel=2e-3, abs=2e-4), (name, idx)
+    for hh in range(H):
+        lp, lm = lam.copy(), lam.copy()
+        lp[hh] += 1e-4
+        lm[hh] -= 1e-4
+        fd = (loss(q, k, v, lp) - loss(q, k, v, lm)) / 2e-4
+        assert res["dlambda"][hh] == pytest.approx(fd, rel=1e-6, abs=1e-9)
+
+
+def test_lambda_params_backward_matches_autograd():
+    H, dim = 3, 5
+    vecs = [0.3 * rand(H, dim, seed=91 + i) for i in range(4)]
+    dl = np.array([0.5, -1.25, 2.0])
+    res = O.lambda_params_bwd(*vecs, dl)
+    ts = [x.double().requires_grad_(True) for x in vecs]
+    lam = torch.exp((ts[0] * ts[1]).sum(1)) - torch.exp((ts[2] * ts[3]).sum(1)) + 0.2
+    (lam * torch.tensor(dl)).sum().backward()
+    for name, t in zip(("dlq1", "dlk1", "dlq2", "dlk2"), ts):
+        assert np.abs(res[name] - t.grad.numpy()).max() < 1e-14, name
