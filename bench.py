@@ -45,6 +45,12 @@ def v1_flops_per_pair(d, dv):
     return 2 * (2 * d) + 2 * (2 * dv)          # two QK^T branches + two P.V
 
 
+def v1_bwd_flops_per_pair(d, dv):
+    """Backward work per visible pair, both branches: recomputed scores (2d),
+    dP = dO V^T (2dv), dQ (2d), dK (2d) and dV (2dv) per branch."""
+    return 2 * (6 * d + 4 * dv)
+
+
 def v2_flops_per_pair(d):
     return 2 * (2 * d) + 2 * (2 * d)
 
@@ -470,6 +476,27 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         del kc, vc, ws
         torch.cuda.empty_cache()
 
+    if want("v1_backward_bf16"):  # gradients at the V1 headline shape (B4 H16 N4096, norm)
+        w = wl("v1_prefill_bf16")
+        x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        dout = torch.randn(w.B, w.N, w.H, w.dv, device=dev).to(torch.bfloat16)
+        lamt = Bd.lambda_from_params(*(x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")),
+                                     w.layer)
+        li = Bd.diffattn_lambda_init(w.layer)
+        ws = torch.empty(Bd.diffattn_v1_bwd_workspace_size(w.B, w.N, w.H, w.d, w.dv),
+                         dtype=torch.uint8, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v1_bwd(q, k, v, dout, lamt, causal=True,
+                                                  apply_norm=True, norm_eps=w.eps,
+                                                  lambda_init=li, workspace=ws), 5, 2, stream)
+        flop = prefill_pairs(w.B, w.N, w.H) * v1_bwd_flops_per_pair(w.d, w.dv)
+        t = flop / (ms * 1e-3) / 1e12
+        out["v1_backward_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
+                                   "frac": round(t / peaks["bf16_tflops"], 4), "flop": flop,
+                                   "workspace_bytes": ws.numel()}
+        del q, k, v, dout, ws
+        torch.cuda.empty_cache()
+
     if want("snr_v1_decode"):  # noise-cancellation sweep, 6 configs x 11 lambdas, L 1024
         from differential_attention_sm_b200 import snr as S
         w = wl("snr_v1_decode")
@@ -581,7 +608,7 @@ def main():
     ap.add_argument("--only", default=None,
                     choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
                              "v1_decode_bf16", "snr_v1_decode", "v2_prefill_window_bf16",
-                             "v2_decode_window_bf16"],
+                             "v2_decode_window_bf16", "v1_backward_bf16"],
                     help="run just this secondary workload (one GPU) and print its numbers")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="with --only: smaller decode batch (profiling runs)")

@@ -42,6 +42,11 @@ EXPORTS = (
     "diffattn_v2_prefill_window",
     "diffattn_v2_decode_window",
     "diffattn_v1_decode_window",
+    "diffattn_v1_bwd_workspace_size",
+    "diffattn_v1_bwd",
+    "diffattn_v2_bwd_workspace_size",
+    "diffattn_v2_bwd",
+    "lambda_from_params_bwd",
 )
 
 
@@ -106,6 +111,19 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.diffattn_v1_decode_window.restype = _i
     lib.diffattn_v1_decode_window.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _vp, _i, _i, _i, _i,
                                               _i, _vp, _i, _vp, _f, _f, _vp, _sz, _vp, _vp]
+    lib.diffattn_v1_bwd_workspace_size.restype = _sz
+    lib.diffattn_v1_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+    lib.diffattn_v1_bwd.restype = _i
+    lib.diffattn_v1_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                    _i, _vp, _f, _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.diffattn_v2_bwd_workspace_size.restype = _sz
+    lib.diffattn_v2_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+    lib.diffattn_v2_bwd.restype = _i
+    lib.diffattn_v2_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                    _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.lambda_from_params_bwd.restype = _i
+    lib.lambda_from_params_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
+                                           _vp]
     _lib = lib
     return lib
 
@@ -340,3 +358,69 @@ def diffattn_v1_decode_window(q, k_cache, v_cache, lam, window, *, cache_lens=No
         _ptr(norm_weight), float(norm_eps), float(lambda_init), _ptr(workspace), ws_bytes,
         _ptr(dev_status), _stream(stream)))
     return out
+
+
+# ---- backward ---------------------------------------------------------------
+def diffattn_v1_bwd_workspace_size(batch, seqlen, n_heads, d_qk, d_v) -> int:
+    return int(load().diffattn_v1_bwd_workspace_size(batch, seqlen, n_heads, d_qk, d_v))
+
+
+def diffattn_v1_bwd(q, k, v, dout, lam, *, causal=True, window=0, apply_norm=False,
+                    norm_weight=None, norm_eps=1e-5, lambda_init=0.0, workspace=None,
+                    stream=None):
+    """V1 gradients.  Returns dict of fp32 device tensors dq, dk (like q),
+    dv (like v), dlambda [H] and, with the norm, dnorm_weight [dv]."""
+    _need_cuda(q, k, v, dout, lam, norm_weight)
+    B, N, H, d2 = q.shape
+    dvw = v.shape[-1]
+    if workspace is None:
+        workspace = torch.empty(diffattn_v1_bwd_workspace_size(B, N, H, d2 // 2, dvw),
+                                dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
+           "dv": torch.empty(v.shape, **f32), "dlambda": torch.empty(H, **f32),
+           "dnorm_weight": torch.empty(dvw, **f32) if apply_norm else None}
+    _check("diffattn_v1_bwd", load().diffattn_v1_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lam), _dtype_code(q), B, N, H, d2 // 2,
+        dvw, int(bool(causal)), int(window), int(bool(apply_norm)), _ptr(norm_weight),
+        float(norm_eps), float(lambda_init), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
+        _ptr(res["dlambda"]), _ptr(res["dnorm_weight"]), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return res
+
+
+def diffattn_v2_bwd_workspace_size(batch, seqlen, n_q_heads, n_kv_heads, head_dim) -> int:
+    return int(load().diffattn_v2_bwd_workspace_size(batch, seqlen, n_q_heads, n_kv_heads,
+                                                     head_dim))
+
+
+def diffattn_v2_bwd(q, k, v, dout, lam, *, causal=True, window=0, workspace=None, stream=None):
+    """V2 gradients.  Returns dict of fp32 device tensors dq (like q), dk,
+    dv (like k) and dlambda [Hq/2]."""
+    _need_cuda(q, k, v, dout, lam)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if workspace is None:
+        workspace = torch.empty(diffattn_v2_bwd_workspace_size(B, N, Hq, Hkv, d),
+                                dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
+           "dv": torch.empty(v.shape, **f32), "dlambda": torch.empty(Hq // 2, **f32)}
+    _check("diffattn_v2_bwd", load().diffattn_v2_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lam), _dtype_code(q), B, N, Hq, Hkv, d,
+        int(bool(causal)), int(window), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
+        _ptr(res["dlambda"]), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return res
+
+
+def lambda_from_params_bwd(lq1, lk1, lq2, lk2, dlambda, stream=None):
+    """Gradients of the four lambda vectors: dict of fp32 [H, dim] tensors."""
+    _need_cuda(lq1, lk1, lq2, lk2, dlambda)
+    H, dim = lq1.shape
+    outs = {n: torch.empty(H, dim, dtype=torch.float32, device=lq1.device)
+            for n in ("dlq1", "dlk1", "dlq2", "dlk2")}
+    _check("lambda_from_params_bwd", load().lambda_from_params_bwd(
+        _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), _ptr(dlambda), H, dim,
+        *(_ptr(outs[n]) for n in ("dlq1", "dlk1", "dlq2", "dlk2")), _stream(stream)))
+    return outs

@@ -234,6 +234,64 @@ DA_API int diffattn_v1_decode_window(const void* q, const void* k_cache, const v
                                      void* workspace, size_t workspace_bytes, int* dev_status,
                                      void* stream);
 
+/* ---- Backward pass ---------------------------------------------------------
+ * Gradients of a scalar loss L with respect to the inputs of the forward
+ * above, given dout = dL/d(out).  The pages define the forward only (the
+ * glossary page calls lambda learned, from four re-parameterised vectors);
+ * these are the chain-rule gradients of that forward.  With causal masking
+ * and an optional sliding window (window = 0: none; > 0 needs causal) as in
+ * the forward.  bf16 inputs only (else DA_ERR_UNSUPPORTED); gradients are
+ * fp32, written (not accumulated) in the layout of the matching input.
+ * Outputs must not overlap inputs or each other.
+ *
+ * This implementation materialises the two attention maps of one head (V1)
+ * or head pair (V2) for a chunk of batch entries at a time in `workspace`
+ * (size from the *_workspace_size query; about 10 N^2 bytes per batch entry
+ * of a chunk) and issues its six matrix products per branch as
+ * strided-batched cuBLAS GEMMs (bf16 operands, fp32 accumulation).  The
+ * first call on a device creates that device's cuBLAS handle, which
+ * allocates cuBLAS's own workspace; calls on one device are serialised on
+ * the host while they enqueue.  Errors: as for the forward, plus
+ * DA_ERR_WORKSPACE for a missing or short workspace. */
+
+/* V1.  q, k: device [batch, seqlen, n_heads, 2*d_qk]; v, dout: device
+ * [batch, seqlen, n_heads, d_v] (bf16); lambda [n_heads] fp32; norm as in
+ * diffattn_v1_fwd.  Outputs (device fp32): dq, dk like q; dv like v;
+ * dlambda [n_heads] (summed over batch and rows); dnorm_weight [d_v]
+ * (gradient of the norm gain, used only with apply_norm; may be NULL).
+ * Supported: d_qk <= 256, d_v <= 128, seqlen^2 <= 2^31. */
+DA_API size_t diffattn_v1_bwd_workspace_size(int batch, int seqlen, int n_heads, int d_qk,
+                                             int d_v);
+DA_API int diffattn_v1_bwd(const void* q, const void* k, const void* v, const void* dout,
+                           const float* lambda, da_dtype dtype, int batch, int seqlen,
+                           int n_heads, int d_qk, int d_v, int causal, int window,
+                           int apply_norm, const float* norm_weight, float norm_eps,
+                           float lambda_init, float* dq, float* dk, float* dv, float* dlambda,
+                           float* dnorm_weight, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* V2.  q: device [batch, seqlen, n_q_heads, head_dim]; k, v: device
+ * [batch, seqlen, n_kv_heads, head_dim]; dout: device [batch, seqlen,
+ * n_q_heads/2, head_dim] (bf16); lambda [n_q_heads/2] fp32.  Outputs
+ * (device fp32): dq like q; dk, dv like k (summed over the pairs that share
+ * a KV head); dlambda [n_q_heads/2].  Supported: head_dim <= 128. */
+DA_API size_t diffattn_v2_bwd_workspace_size(int batch, int seqlen, int n_q_heads,
+                                             int n_kv_heads, int head_dim);
+DA_API int diffattn_v2_bwd(const void* q, const void* k, const void* v, const void* dout,
+                           const float* lambda, da_dtype dtype, int batch, int seqlen,
+                           int n_q_heads, int n_kv_heads, int head_dim, int causal, int window,
+                           float* dq, float* dk, float* dv, float* dlambda, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Gradients of the four lambda vectors (device fp32 [n_heads, dim]) of
+ * lambda_from_params, from dlambda [n_heads]:
+ *   dlq1 = dlambda e^{lq1.lk1} lk1,  dlk1 = dlambda e^{lq1.lk1} lq1,
+ *   dlq2 = -dlambda e^{lq2.lk2} lk2, dlk2 = -dlambda e^{lq2.lk2} lq2. */
+DA_API int lambda_from_params_bwd(const float* lq1, const float* lk1, const float* lq2,
+                                  const float* lk2, const float* dlambda, int n_heads, int dim,
+                                  float* dlq1, float* dlk1, float* dlq2, float* dlk2,
+                                  void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,98 @@
+"""GPU parity of the backward pass against the fp64 oracle backward (itself
+pinned to float64 autograd and finite differences): dq, dk, dv, dlambda and,
+for V1 with the norm, the norm gain's gradient; both forms, causal,
+non-causal and sliding-window masks, ragged lengths, GQA, the lambda
+re-parameterisation, and one full-size V1 head (batch 4, 16 heads, 4096)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from differential_attention_sm_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+# bf16 operands (maps and dS rounded to bf16, fp32 accumulation): the same
+# relative bounds as the bf16 forward outputs, on |gpu - ref| / max|ref|.
+TOL_MAX, TOL_MEAN = 2e-2, 2e-3
+
+
+@pytest.fixture(scope="module")
+def B():
+    from differential_attention_sm_b200 import binding
+    binding.load()
+    return binding
+
+
+def cuda(t):
+    return t.cuda().contiguous()
+
+
+def close(got, ref, what):
+    g = got.detach().double().cpu().numpy() if isinstance(got, torch.Tensor) else np.asarray(got)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.isfinite(g).all(), what
+    scale = np.abs(r).max()
+    err = np.abs(g - r) / scale
+    assert err.max() <= TOL_MAX and err.mean() <= TOL_MEAN, (what, err.max(), err.mean())
+
+
+@pytest.mark.parametrize("N,causal,window,norm", [(300, True, 0, True), (256, False, 0, False),
+                                                  (333, True, 70, True), (129, True, 0, False)])
+def test_v1_backward(B, N, causal, window, norm):
+    Bn, H, d, dv, layer = 2, 3, 64, 128, 12
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=1100 + N)
+    dout = I.v1_inputs(Bn, N, H, d, dv, seed=1200 + N)["v"]
+    lam_dev = B.lambda_from_params(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")), layer)
+    lam = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], layer)
+    li = O.lambda_init(layer)
+    g = (1.0 + 0.2 * torch.randn(dv, generator=torch.Generator().manual_seed(5))).float()
+    res = B.diffattn_v1_bwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(dout), lam_dev,
+                            causal=causal, window=window, apply_norm=norm,
+                            norm_weight=cuda(g) if norm else None, lambda_init=li)
+    ref = O.v1_bwd(x["q"], x["k"], x["v"], dout, lam, causal=causal, window=window,
+                   apply_norm=norm, norm_weight=g if norm else None, lambda_init_value=li)
+    for name in ("dq", "dk", "dv", "dlambda"):
+        close(res[name], ref[name], "v1 %s N=%d" % (name, N))
+    if norm:
+        close(res["dnorm_weight"], ref["dnorm_weight"], "v1 dnorm_weight")
+    # lambda re-parameterisation: same dlambda into both sides
+    dl = res["dlambda"]
+    gp = B.lambda_from_params_bwd(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")), dl)
+    rp = O.lambda_params_bwd(x["lq1"], x["lk1"], x["lq2"], x["lk2"], dl.double().cpu().numpy())
+    for n in ("dlq1", "dlk1", "dlq2", "dlk2"):
+        assert np.abs(gp[n].double().cpu().numpy() - rp[n]).max() <= 1e-5 * max(1.0, np.abs(rp[n]).max())
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,causal,window", [(520, 8, 2, True, 0), (300, 8, 4, False, 0),
+                                                     (400, 16, 2, True, 100)])
+def test_v2_backward(B, N, Hq, Hkv, causal, window):
+    Bn, d = 1, 128
+    x = I.v2_inputs(Bn, N, Hq, Hkv, d, seed=1300 + N)
+    dout = I.v2_inputs(Bn, N, Hq, Hkv, d, seed=1400 + N)["q"][:, :, : Hq // 2].contiguous()
+    res = B.diffattn_v2_bwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(dout),
+                            cuda(x["lam"]), causal=causal, window=window)
+    ref = O.v2_bwd(x["q"], x["k"], x["v"], dout, x["lam"], causal=causal, window=window)
+    for name in ("dq", "dk", "dv", "dlambda"):
+        close(res[name], ref[name], "v2 %s N=%d" % (name, N))
+
+
+def test_v1_backward_full_size_one_head(B):
+    """The benchmark's V1 shape (batch 4, 16 heads, 4096, causal, norm): the
+    gradients of one (batch, head) unit depend on that unit alone, so the
+    oracle runs on its slice."""
+    w = I.WORKLOADS["v1_prefill_bf16"]
+    x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed)
+    dout = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed + 77)["v"]
+    lam_dev = B.lambda_from_params(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")), w.layer)
+    lam = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+    li = O.lambda_init(w.layer)
+    res = B.diffattn_v1_bwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(dout), lam_dev,
+                            causal=True, apply_norm=True, norm_eps=w.eps, lambda_init=li)
+    b, h = 2, 11
+    sl = lambda t: t[b:b + 1, :, h:h + 1].contiguous()
+    ref = O.v1_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(dout), lam[h:h + 1], causal=True,
+                   apply_norm=True, eps=w.eps, lambda_init_value=li)
+    for name in ("dq", "dk", "dv"):
+        close(res[name][b:b + 1, :, h:h + 1], ref[name], "v1 full %s" % name)
