@@ -115,12 +115,13 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.diffattn_v1_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
     lib.diffattn_v1_bwd.restype = _i
     lib.diffattn_v1_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
-                                    _i, _vp, _f, _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+                                    _i, _vp, _f, _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp,
+                                    _vp]
     lib.diffattn_v2_bwd_workspace_size.restype = _sz
     lib.diffattn_v2_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
     lib.diffattn_v2_bwd.restype = _i
     lib.diffattn_v2_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
-                                    _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+                                    _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
     lib.lambda_from_params_bwd.restype = _i
     lib.lambda_from_params_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
                                            _vp]
@@ -367,7 +368,7 @@ def diffattn_v1_bwd_workspace_size(batch, seqlen, n_heads, d_qk, d_v) -> int:
 
 def diffattn_v1_bwd(q, k, v, dout, lam, *, causal=True, window=0, apply_norm=False,
                     norm_weight=None, norm_eps=1e-5, lambda_init=0.0, workspace=None,
-                    stream=None):
+                    dev_status=None, stream=None):
     """V1 gradients.  Returns dict of fp32 device tensors dq, dk (like q),
     dv (like v), dlambda [H] and, with the norm, dnorm_weight [dv]."""
     _need_cuda(q, k, v, dout, lam, norm_weight)
@@ -385,7 +386,7 @@ def diffattn_v1_bwd(q, k, v, dout, lam, *, causal=True, window=0, apply_norm=Fal
         dvw, int(bool(causal)), int(window), int(bool(apply_norm)), _ptr(norm_weight),
         float(norm_eps), float(lambda_init), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
         _ptr(res["dlambda"]), _ptr(res["dnorm_weight"]), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)))
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
     return res
 
 
@@ -394,7 +395,8 @@ def diffattn_v2_bwd_workspace_size(batch, seqlen, n_q_heads, n_kv_heads, head_di
                                                      head_dim))
 
 
-def diffattn_v2_bwd(q, k, v, dout, lam, *, causal=True, window=0, workspace=None, stream=None):
+def diffattn_v2_bwd(q, k, v, dout, lam, *, causal=True, window=0, workspace=None,
+                    dev_status=None, stream=None):
     """V2 gradients.  Returns dict of fp32 device tensors dq (like q), dk,
     dv (like k) and dlambda [Hq/2]."""
     _need_cuda(q, k, v, dout, lam)
@@ -410,7 +412,7 @@ def diffattn_v2_bwd(q, k, v, dout, lam, *, causal=True, window=0, workspace=None
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lam), _dtype_code(q), B, N, Hq, Hkv, d,
         int(bool(causal)), int(window), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
         _ptr(res["dlambda"]), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(stream)))
+        _ptr(dev_status), _stream(stream)))
     return res
 
 

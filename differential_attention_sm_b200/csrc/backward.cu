@@ -32,6 +32,7 @@
 #include <mutex>
 
 #include "diffattn.h"
+#include "kernels.h"
 
 namespace da {
 namespace {
@@ -426,6 +427,13 @@ int run_bwd(const Geo& G, const __nv_bfloat16* q, const __nv_bfloat16* k,
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool fits_int(long long x) { return x >= 0 && x <= 0x7fffffffLL; }
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
 
 }  // namespace
 }  // namespace da
@@ -434,6 +442,7 @@ extern "C" {
 
 size_t diffattn_v1_bwd_workspace_size(int batch, int seqlen, int n_heads, int d_qk, int d_v) {
   if (batch < 1 || seqlen < 1 || n_heads < 1 || d_qk < 1 || d_v < 1) return 0;
+  if (d_qk == 64 && d_v == 128) return da::fused_bwd_workspace_bytes(batch, seqlen, n_heads);
   return da::bwd_workspace_bytes(batch, seqlen, d_v);
 }
 
@@ -442,7 +451,7 @@ int diffattn_v1_bwd(const void* q, const void* k, const void* v, const void* dou
                     int d_qk, int d_v, int causal, int window, int apply_norm,
                     const float* norm_weight, float norm_eps, float lambda_init, float* dq,
                     float* dk, float* dv, float* dlambda, float* dnorm_weight, void* workspace,
-                    size_t workspace_bytes, void* stream) {
+                    size_t workspace_bytes, int* dev_status, void* stream) {
   if (!q || !k || !v || !dout || !lambda || !dq || !dk || !dv || !dlambda)
     return DA_ERR_INVALID_ARG;
   if (batch < 1 || seqlen < 1 || n_heads < 1 || d_qk < 1 || d_v < 1) return DA_ERR_INVALID_ARG;
@@ -474,6 +483,41 @@ int diffattn_v1_bwd(const void* q, const void* k, const void* v, const void* dou
   G.o_row = G.v_row;
   G.o_b = G.v_b;
   G.o_unit = d_v;
+  if (d_qk == 64 && d_v == 128) {  // fused tcgen05 path
+    if (!workspace || workspace_bytes < da::fused_bwd_workspace_bytes(batch, seqlen, n_heads))
+      return DA_ERR_WORKSPACE;
+    if (!da::fits_int((long long)batch * seqlen)) return DA_ERR_UNSUPPORTED;
+    da::FusedBwdArgs a{};
+    a.fwd.form = 1;
+    a.fwd.batch = batch;
+    a.fwd.seqlen = seqlen;
+    a.fwd.heads = n_heads;
+    a.fwd.kv_heads = n_heads;
+    a.fwd.pairs_per_kv = 1;
+    a.fwd.causal = causal ? 1 : 0;
+    a.fwd.window = window;
+    a.fwd.lambda = lambda;
+    a.fwd.apply_norm = apply_norm ? 1 : 0;
+    a.fwd.norm_weight = norm_weight;
+    a.fwd.eps = norm_eps;
+    a.fwd.post_scale = 1.0f - lambda_init;
+    a.fwd.dev_status = dev_status;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.dout = dout;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.dlambda = dlambda;
+    a.dg = apply_norm ? dnorm_weight : nullptr;
+    a.workspace = workspace;
+    a.num_sms = da::sm_count();
+    if (a.num_sms < 1) return DA_ERR_CUDA;
+    return da::launch_fused_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DA_OK
+               : DA_ERR_CUDA;
+  }
   return da::run_bwd(G, static_cast<const __nv_bfloat16*>(q),
                      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
                      static_cast<const __nv_bfloat16*>(dout), lambda, causal ? 1 : 0, window,
@@ -485,6 +529,7 @@ int diffattn_v1_bwd(const void* q, const void* k, const void* v, const void* dou
 size_t diffattn_v2_bwd_workspace_size(int batch, int seqlen, int n_q_heads, int n_kv_heads,
                                       int head_dim) {
   if (batch < 1 || seqlen < 1 || n_q_heads < 2 || n_kv_heads < 1 || head_dim < 1) return 0;
+  if (head_dim == 128) return da::fused_bwd_workspace_bytes(batch, seqlen, n_q_heads / 2);
   return da::bwd_workspace_bytes(batch, seqlen, head_dim);
 }
 
@@ -492,7 +537,7 @@ int diffattn_v2_bwd(const void* q, const void* k, const void* v, const void* dou
                     const float* lambda, da_dtype dtype, int batch, int seqlen, int n_q_heads,
                     int n_kv_heads, int head_dim, int causal, int window, float* dq, float* dk,
                     float* dv, float* dlambda, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+                    int* dev_status, void* stream) {
   if (!q || !k || !v || !dout || !lambda || !dq || !dk || !dv || !dlambda)
     return DA_ERR_INVALID_ARG;
   if (batch < 1 || seqlen < 1 || n_q_heads < 2 || n_kv_heads < 1 || head_dim < 1)
@@ -527,6 +572,39 @@ int diffattn_v2_bwd(const void* q, const void* k, const void* v, const void* dou
   G.o_row = (long long)(n_q_heads / 2) * head_dim;
   G.o_b = G.o_row * seqlen;
   G.o_unit = head_dim;
+  if (head_dim == 128) {  // fused tcgen05 path
+    if (!workspace ||
+        workspace_bytes < da::fused_bwd_workspace_bytes(batch, seqlen, n_q_heads / 2))
+      return DA_ERR_WORKSPACE;
+    if (!da::fits_int((long long)batch * seqlen)) return DA_ERR_UNSUPPORTED;
+    da::FusedBwdArgs a{};
+    a.fwd.form = 2;
+    a.fwd.batch = batch;
+    a.fwd.seqlen = seqlen;
+    a.fwd.heads = n_q_heads / 2;
+    a.fwd.kv_heads = n_kv_heads;
+    a.fwd.pairs_per_kv = group / 2;
+    a.fwd.causal = causal ? 1 : 0;
+    a.fwd.window = window;
+    a.fwd.lambda = lambda;
+    a.fwd.apply_norm = 0;
+    a.fwd.post_scale = 1.f;
+    a.fwd.dev_status = dev_status;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.dout = dout;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.dlambda = dlambda;
+    a.workspace = workspace;
+    a.num_sms = da::sm_count();
+    if (a.num_sms < 1) return DA_ERR_CUDA;
+    return da::launch_fused_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DA_OK
+               : DA_ERR_CUDA;
+  }
   return da::run_bwd(G, static_cast<const __nv_bfloat16*>(q),
                      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
                      static_cast<const __nv_bfloat16*>(dout), lambda, causal ? 1 : 0, window, 0,

@@ -1,0 +1,808 @@
+// backward_tc.cu — fused backward of differential attention on the 5th-
+// generation tensor cores (tcgen05 + tensor memory + TMA), both forms.
+//
+// Forward: glossary page "Differential Transformer", section "Cómo funciona
+// la atención diferencial"; lesson "Atención Diferencial (V2)", sections "La
+// idea diferencial" and "V1 vs V2: la diferencia".  With P_r the two softmax
+// maps, o = P_1 V - lambda P_2 V, do the gradient of the pre-norm output,
+// do_1 = do, do_2 = -lambda do and D_r = do_r . (P_r V) per row, the
+// gradients of each branch are the usual ones of softmax attention:
+//     dP_r = do_r V^T,  dS_r = P_r (dP_r - D_r),
+//     dQ_r = dS_r K_r / sqrt(d),  dK_r += dS_r^T Q_r / sqrt(d),  dV += P_r^T do_r.
+// The training forward (prefill kernel with saves) provides the per-row
+// log2-sum-exp of each branch, so P_r = 2^(s sc - lse_r) is recomputed
+// tile by tile and nothing of size N x N ever reaches memory.
+//
+// Two kernels:
+//   * dq kernel, one CTA per 128 query rows of a head (V1) or head pair
+//     (V2), walking 64-key tiles like the forward: per branch, S_r and dP_r
+//     into tensor memory (two SS MMAs), dS_r written back over S_r as bf16
+//     by the softmax-backward warps, then dQ_r += dS_r K_r (TS MMA) in
+//     tensor memory.  Warps: 0-3 / 4-7 branch 1 / 2 (thread = query row),
+//     8 TMA producer, 9 / 10 score-and-dP issuers, 11 / 12 dQ issuers.
+//   * dkdv kernel, one CTA per 128 keys of a head (V1) or KV head (V2),
+//     walking 64-query tiles (and, for V2, every pair that reads the KV
+//     head): S^T = K_r Q_r^T and dP^T = V do_r^T (SS), P^T and dS^T written
+//     back as bf16 by the softmax-backward warps (thread = key row), then
+//     dV += P^T do_r and dK_r += dS^T Q_r (TS) in tensor memory.  Both
+//     accumulations are issued by one thread, so their order is fixed.
+//     Warps: 0-3 / 4-7 alternate steps (= branches), 8 producer,
+//     9 score-and-dP issuer, 10 accumulation issuer.
+// Every wait is bounded (DA_ERR_DEVICE_TIMEOUT in the status word).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace da {
+namespace {
+
+constexpr int kBox128 = 128 * 64 * 2;  // TMA box: 128 rows x 64 bf16 = 16 KB
+constexpr int kBox64 = 64 * 64 * 2;    // TMA box: 64 rows x 64 bf16 = 8 KB
+constexpr int kTile128 = 2 * kBox128;  // 128 x 128 bf16
+constexpr int kTile64 = 2 * kBox64;    // 64 x 128 bf16
+
+struct BwdParams {
+  int batch, seqlen, units, pairs_per_kv, causal, window;
+  int npad;          // row stride of lse and D (seqlen rounded up to 64)
+  float scale_log2;  // log2(e) / sqrt(d)
+  float scale;       // 1 / sqrt(d)
+  const float* lse;  // [B][units][2][npad]: p = 2^(s * scale_log2 - lse)
+  const float* Dv;   // [B][units][2][npad]: D_r = do_r . O_r
+  float* dq;         // like q
+  float* dk;         // like k
+  float* dv;         // like v
+  int q_heads, kv_heads;
+  int n_qtiles;      // dq grid: ceil(N / 128) per unit
+  int n_ktiles;      // dkdv grid: ceil(N / 128) per KV unit
+  int* dev_status;
+};
+
+// ===================================================================== dQ
+constexpr int kDqThreads = 416;
+constexpr int kDqStages = 2;
+
+struct DqBarriers {
+  uint64_t q_full;
+  uint64_t k_full[kDqStages], k_empty[kDqStages];
+  uint64_t v_full[kDqStages], v_empty[kDqStages];
+  uint64_t sd_full[2], ds_full[2], dq_done[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int kForm, bool kWindow>
+__global__ void __launch_bounds__(kDqThreads, 1)
+    diffattn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_do,
+                           const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
+  constexpr int D = kForm == 1 ? 64 : 128;  // one branch's query width
+  constexpr uint32_t kQBytes = kForm == 1 ? kTile128 : 2 * kTile128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sdO = sQ + kQBytes;                     // 2 branches x 128 x 128
+  uint8_t* sK = sdO + 2 * kTile128;                // stages x 64 x 128
+  uint8_t* sV = sK + kDqStages * kTile64;
+  DqBarriers* bars = reinterpret_cast<DqBarriers*>(sV + kDqStages * kTile64);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int mt = p.n_qtiles - 1 - (int)(blockIdx.x % p.n_qtiles);  // heavy tiles first
+  const int bu = (int)(blockIdx.x / p.n_qtiles);
+  const int hh = bu % p.units, b = bu / p.units;
+  const int kvh = kForm == 1 ? hh : hh / p.pairs_per_kv;
+  const int q0 = mt * 128;
+  const int key_end = p.causal ? min(q0 + 128, p.seqlen) : p.seqlen;
+  const int kv0 = kWindow ? max(0, q0 - p.window + 1) / 64 : 0;
+  const int n_kv = (key_end + 63) / 64 - kv0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kDqStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 4);  // both branches' S and dQ products read K
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 2);
+    }
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&bars->sd_full[r], 1);
+      mbar_init(&bars->ds_full[r], 128);
+      mbar_init(&bars->dq_done[r], 1);
+    }
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  // tensor-memory columns: S_r, dP_r (64 each), dQ_r (D each)
+  auto colS = [](int r) { return (uint32_t)(128 * r); };
+  auto colP = [](int r) { return (uint32_t)(128 * r + 64); };
+  auto colQ = [](int r) { return (uint32_t)(256 + D * r); };
+  bool failed = false;
+
+  if (warp == 8) {
+    if (lane == 0) {  // ---------------------------------------------- producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&bars->q_full, kQBytes + 2 * kTile128);
+      if (kForm == 1) {
+        tma_load_4d(sQ, &tm_q, &bars->q_full, 0, hh, q0, b);
+        tma_load_4d(sQ + kBox128, &tm_q, &bars->q_full, 64, hh, q0, b);
+      } else {
+        for (int r = 0; r < 2; ++r) {
+          tma_load_4d(sQ + r * kTile128, &tm_q, &bars->q_full, 0, 2 * hh + r, q0, b);
+          tma_load_4d(sQ + r * kTile128 + kBox128, &tm_q, &bars->q_full, 64, 2 * hh + r, q0, b);
+        }
+      }
+      for (int r = 0; r < 2; ++r) {
+        tma_load_4d(sdO + r * kTile128, &tm_do, &bars->q_full, 0, 2 * hh + r, q0, b);
+        tma_load_4d(sdO + r * kTile128 + kBox128, &tm_do, &bars->q_full, 64, 2 * hh + r, q0, b);
+      }
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kDqStages;
+        const uint32_t ph = (uint32_t)(j / kDqStages) & 1u;
+        const int row = (kv0 + j) * 64;
+        if (!mbar_wait(&bars->k_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
+        mbar_arrive_expect_tx(&bars->k_full[s], kTile64);
+        tma_load_4d(sK + s * kTile64, &tm_k, &bars->k_full[s], 0, kvh, row, b);
+        tma_load_4d(sK + s * kTile64 + kBox64, &tm_k, &bars->k_full[s], 64, kvh, row, b);
+        if (!mbar_wait(&bars->v_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
+        mbar_arrive_expect_tx(&bars->v_full[s], kTile64);
+        tma_load_4d(sV + s * kTile64, &tm_v, &bars->v_full[s], 0, kvh, row, b);
+        tma_load_4d(sV + s * kTile64 + kBox64, &tm_v, &bars->v_full[s], 64, kvh, row, b);
+      }
+    }
+  } else if (warp == 9 || warp == 10) {
+    if (lane == 0) {  // ------------------------- S_r and dP_r issuer, r = warp - 9
+      const int r = warp - 9;
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO) + r * kTile128;
+      constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
+      if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
+        for (int j = 0; j < n_kv; ++j) {
+          const int s = j % kDqStages;
+          const uint32_t ph = (uint32_t)(j / kDqStages) & 1u;
+          if (!mbar_wait(&bars->k_full[s], ph, p.dev_status, &failed)) break;
+          if (!mbar_wait(&bars->v_full[s], ph, p.dev_status, &failed)) break;
+          // S_r / dP_r buffers last held tile j-1: its dS_r must have been consumed
+          if (j > 0 && !mbar_wait(&bars->dq_done[r], (uint32_t)(j - 1) & 1u, p.dev_status,
+                                  &failed))
+            break;
+          tc_fence_after();
+          const uint32_t kt = smem_u32(sK) + s * kTile64, vt = smem_u32(sV) + s * kTile64;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t a, bb;
+            if (kForm == 1) {
+              a = q_addr + r * kBox128 + kk * 32;
+              bb = kt + r * kBox64 + kk * 32;
+            } else {
+              a = q_addr + r * kTile128 + (kk >> 2) * kBox128 + (kk & 3) * 32;
+              bb = kt + (kk >> 2) * kBox64 + (kk & 3) * 32;
+            }
+            tc_mma_ss(tmem + colS(r), smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bb, 16, 1024),
+                      idS, kk > 0 ? 1u : 0u);
+          }
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t a = do_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
+            const uint32_t bb = vt + (kk >> 2) * kBox64 + (kk & 3) * 32;
+            tc_mma_ss(tmem + colP(r), smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bb, 16, 1024),
+                      idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars->sd_full[r]);
+          tc_commit(&bars->v_empty[s]);
+          tc_commit(&bars->k_empty[s]);
+        }
+      }
+    }
+  } else if (warp == 11 || warp == 12) {
+    if (lane == 0) {  // ------------------------------------ dQ_r issuer, r = warp - 11
+      const int r = warp - 11;
+      constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kDqStages;
+        if (!mbar_wait(&bars->ds_full[r], (uint32_t)j & 1u, p.dev_status, &failed)) break;
+        if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kDqStages) & 1u, p.dev_status, &failed))
+          break;
+        tc_fence_after();
+        const uint32_t kt = smem_u32(sK) + s * kTile64 + (kForm == 1 ? r * kBox64 : 0);
+        for (int kk = 0; kk < 4; ++kk)  // 16 keys per step; B = K_r, MN-major
+          tc_mma_ts(tmem + colQ(r), tmem + colS(r) + kk * 8,
+                    smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bars->dq_done[r]);
+        tc_commit(&bars->k_empty[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------- softmax backward, branch r
+    const int r = warp / 4;
+    const int row = (warp & 3) * 32 + lane;
+    const int qrow = q0 + row;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int lim = p.causal ? min(qrow + 1, p.seqlen) : p.seqlen;
+    const int lo = kWindow ? max(0, qrow - p.window + 1) : 0;
+    const size_t vrow = (((size_t)b * p.units + hh) * 2 + r) * p.npad + qrow;
+    const float lse = qrow < p.seqlen ? p.lse[vrow] : 0.f;
+    const float Dr = qrow < p.seqlen ? p.Dv[vrow] : 0.f;
+    const float sc = p.scale_log2;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->sd_full[r], (uint32_t)j & 1u, p.dev_status,
+                                             &failed))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      const int k0 = (kv0 + j) * 64;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[32], dp[32], pk[16];
+        tmem_ld32(tmem + lane_off + colS(r) + 32 * half, sv);
+        tmem_ld32(tmem + lane_off + colP(r) + 32 * half, dp);
+        tc_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int key = k0 + 32 * half + 2 * e + u;
+            const bool vis = key < lim && (!kWindow || key >= lo);
+            const float pr = vis ? ex2(__uint_as_float(sv[2 * e + u]) * sc - lse) : 0.f;
+            ds[u] = vis ? pr * (__uint_as_float(dp[2 * e + u]) - Dr) : 0.f;
+          }
+          pk[e] = pack_bf16(ds[0], ds[1]);
+        }
+        tmem_st16(tmem + lane_off + colS(r) + 16 * half, pk);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_full[r]);
+    }
+    __syncwarp();
+    if (failed) bars->abort_flag = 1;
+    if (n_kv > 0)
+      mbar_wait(&bars->dq_done[r], (uint32_t)(n_kv - 1) & 1u, p.dev_status, &failed);
+    tc_fence_after();
+    const bool store = qrow < p.seqlen;
+    float* dst = kForm == 1
+                     ? p.dq + (((size_t)b * p.seqlen + qrow) * p.q_heads + hh) * 128 + 64 * r
+                     : p.dq + (((size_t)b * p.seqlen + qrow) * p.q_heads + 2 * hh + r) * 128;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + colQ(r) + 32 * c, v);
+      tc_wait_ld();
+      if (store && !bars->abort_flag) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float4 f;
+          f.x = __uint_as_float(v[e]) * p.scale;
+          f.y = __uint_as_float(v[e + 1]) * p.scale;
+          f.z = __uint_as_float(v[e + 2]) * p.scale;
+          f.w = __uint_as_float(v[e + 3]) * p.scale;
+          *reinterpret_cast<float4*>(dst + 32 * c + e) = f;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// =================================================================== dK, dV
+constexpr int kKvThreads = 352;
+constexpr int kKvStages = 3;
+constexpr int kStageQ = kTile64;                       // Q_r tile (V1 uses one box)
+// + dO_r tile + lse/D vectors; a multiple of 1 KB keeps every stage's
+// 128-byte-swizzled tiles on the 1 KB alignment their descriptors assume
+constexpr int kStageBytes = kStageQ + kTile64 + 1024;
+static_assert(kStageBytes % 1024 == 0, "stage alignment");
+
+struct KvBarriers {
+  uint64_t kv_full;
+  uint64_t qd_full[kKvStages], qd_empty[kKvStages];
+  uint64_t sd_full[2], ps_full[2], buf_free[2];
+  uint64_t acc_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int kForm, bool kWindow>
+__global__ void __launch_bounds__(kKvThreads, 1)
+    diffattn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                             const __grid_constant__ CUtensorMap tm_do,
+                             const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const BwdParams p) {
+  constexpr int D = kForm == 1 ? 64 : 128;
+  constexpr uint32_t kQStepBytes = kForm == 1 ? kBox64 : kTile64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;                  // 128 keys x 128
+  uint8_t* sV = sK + kTile128;
+  uint8_t* sStage = sV + kTile128;     // stages x (Q, dO, lse[64], D[64])
+  KvBarriers* bars = reinterpret_cast<KvBarriers*>(sStage + kKvStages * kStageBytes);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int kt_idx = (int)(blockIdx.x % p.n_ktiles);
+  const int bg = (int)(blockIdx.x / p.n_ktiles);
+  const int g = bg % p.kv_heads, b = bg / p.kv_heads;  // V1: g is the head
+  const int k0 = kt_idx * 128;
+  const int members = kForm == 1 ? 1 : p.pairs_per_kv;
+  const int n_qt = (p.seqlen + 63) / 64;
+  const int i0 = p.causal ? k0 / 64 : 0;
+  int i1 = n_qt;
+  if (kWindow) i1 = min(i1, (k0 + 127 + p.window - 1) / 64 + 1);
+  const int n_steps = (i1 - i0) * members * 2;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < kKvStages; ++s) {
+      mbar_init(&bars->qd_full[s], 1);
+      mbar_init(&bars->qd_empty[s], 2);  // both issuers read Q_r and dO_r
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars->sd_full[w], 1);
+      mbar_init(&bars->ps_full[w], 128);
+      mbar_init(&bars->buf_free[w], 1);
+    }
+    mbar_init(&bars->acc_done, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  // columns: S^T_w [128w, +64), dP^T_w [128w+64, +64), dV [256, 384), dK [384, 512)
+  constexpr uint32_t kColDV = 256, kColDK = 384;
+  bool failed = false;
+  // step s -> (query tile, member, branch): branch innermost
+  auto step_q0 = [&](int s) { return (i0 + (s >> 1) / members) * 64; };
+  auto step_unit = [&](int s) {
+    return kForm == 1 ? g : g * p.pairs_per_kv + (s >> 1) % members;
+  };
+
+  if (warp == 8) {
+    if (lane == 0) {  // ---------------------------------------------- producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * kTile128);
+      tma_load_4d(sK, &tm_k, &bars->kv_full, 0, g, k0, b);
+      tma_load_4d(sK + kBox128, &tm_k, &bars->kv_full, 64, g, k0, b);
+      tma_load_4d(sV, &tm_v, &bars->kv_full, 0, g, k0, b);
+      tma_load_4d(sV + kBox128, &tm_v, &bars->kv_full, 64, g, k0, b);
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s % kKvStages;
+        const uint32_t ph = (uint32_t)(s / kKvStages) & 1u;
+        const int r = s & 1, q0 = step_q0(s), u = step_unit(s);
+        if (!mbar_wait(&bars->qd_empty[st], ph ^ 1u, p.dev_status, &failed)) break;
+        uint8_t* sq = sStage + st * kStageBytes;
+        uint8_t* sdo = sq + kStageQ;
+        float* svec = reinterpret_cast<float*>(sdo + kTile64);
+        mbar_arrive_expect_tx(&bars->qd_full[st], kQStepBytes + kTile64 + 512);
+        if (kForm == 1) {
+          tma_load_4d(sq, &tm_q, &bars->qd_full[st], 64 * r, u, q0, b);
+        } else {
+          tma_load_4d(sq, &tm_q, &bars->qd_full[st], 0, 2 * u + r, q0, b);
+          tma_load_4d(sq + kBox64, &tm_q, &bars->qd_full[st], 64, 2 * u + r, q0, b);
+        }
+        tma_load_4d(sdo, &tm_do, &bars->qd_full[st], 0, 2 * u + r, q0, b);
+        tma_load_4d(sdo + kBox64, &tm_do, &bars->qd_full[st], 64, 2 * u + r, q0, b);
+        const size_t vrow = (((size_t)b * p.units + u) * 2 + r) * p.npad + q0;
+        bulk_load(svec, p.lse + vrow, 256, &bars->qd_full[st]);
+        bulk_load(svec + 64, p.Dv + vrow, 256, &bars->qd_full[st]);
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {  // ---------------------------------- S^T and dP^T issuer
+      constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      if (mbar_wait(&bars->kv_full, 0, p.dev_status, &failed)) {
+        for (int s = 0; s < n_steps; ++s) {
+          const int st = s % kKvStages, w = s & 1, r = s & 1;
+          if (!mbar_wait(&bars->qd_full[st], (uint32_t)(s / kKvStages) & 1u, p.dev_status,
+                         &failed))
+            break;
+          if (s >= 2 && !mbar_wait(&bars->buf_free[w], (uint32_t)((s - 2) >> 1) & 1u,
+                                   p.dev_status, &failed))
+            break;
+          tc_fence_after();
+          const uint32_t sq = smem_u32(sStage) + st * kStageBytes, sdo = sq + kStageQ;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t a, bb;
+            if (kForm == 1) {
+              a = k_addr + r * kBox128 + kk * 32;
+              bb = sq + kk * 32;
+            } else {
+              a = k_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
+              bb = sq + (kk >> 2) * kBox64 + (kk & 3) * 32;
+            }
+            tc_mma_ss(tmem + 128 * w, smem_desc_sw128(a, 16, 1024),
+                      smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          }
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t a = v_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
+            const uint32_t bb = sdo + (kk >> 2) * kBox64 + (kk & 3) * 32;
+            tc_mma_ss(tmem + 128 * w + 64, smem_desc_sw128(a, 16, 1024),
+                      smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars->sd_full[w]);
+          tc_commit(&bars->qd_empty[st]);
+        }
+      }
+    }
+  } else if (warp == 10) {
+    if (lane == 0) {  // ------------------------------ dV and dK accumulation issuer
+      constexpr uint32_t idV = idesc_bf16_f32(128, 128, false, true);
+      constexpr uint32_t idK = idesc_bf16_f32(128, D, false, true);
+      bool first_v = true, first_k[2] = {true, true};
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s % kKvStages, w = s & 1, r = s & 1;
+        if (!mbar_wait(&bars->ps_full[w], (uint32_t)(s >> 1) & 1u, p.dev_status, &failed))
+          break;
+        tc_fence_after();
+        const uint32_t sq = smem_u32(sStage) + st * kStageBytes, sdo = sq + kStageQ;
+        const int kb = kForm == 1 ? r : 0;
+        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step; B operands MN-major
+          tc_mma_ts(tmem + kColDV, tmem + 128 * w + kk * 8,
+                    smem_desc_sw128(sdo + kk * 2048, kBox64, 1024), idV,
+                    (first_v && kk == 0) ? 0u : 1u);
+          tc_mma_ts(tmem + kColDK + (kForm == 1 ? 64 * r : 0), tmem + 128 * w + 64 + kk * 8,
+                    smem_desc_sw128(sq + kk * 2048, kBox64, 1024), idK,
+                    (first_k[kb] && kk == 0) ? 0u : 1u);
+        }
+        first_v = false;
+        first_k[kb] = false;
+        tc_commit(&bars->buf_free[w]);
+        tc_commit(&bars->qd_empty[st]);
+      }
+      tc_commit(&bars->acc_done);
+    }
+  } else {
+    // --------------------------------- softmax backward, steps of parity w
+    const int w = warp / 4;
+    const int krow = (warp & 3) * 32 + lane;
+    const int key = k0 + krow;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float sc = p.scale_log2;
+    for (int s = w; s < n_steps; s += 2) {
+      const int st = s % kKvStages;
+      const bool ok = mbar_wait(&bars->qd_full[st], (uint32_t)(s / kKvStages) & 1u,
+                                p.dev_status, &failed) &&
+                      mbar_wait(&bars->sd_full[w], (uint32_t)(s >> 1) & 1u, p.dev_status,
+                                &failed);
+      if (!__all_sync(0xffffffffu, ok)) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      const int q0 = step_q0(s);
+      const float* svec =
+          reinterpret_cast<const float*>(sStage + st * kStageBytes + kStageQ + kTile64);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[32], dp[32], pp[16], pd[16];
+        tmem_ld32(tmem + lane_off + 128 * w + 32 * half, sv);
+        tmem_ld32(tmem + lane_off + 128 * w + 64 + 32 * half, dp);
+        tc_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = 32 * half + 2 * e + u;
+            const int q = q0 + c;
+            bool vis = q < p.seqlen && key < p.seqlen;
+            if (p.causal) vis = vis && q >= key;
+            if (kWindow) vis = vis && q - key < p.window;
+            pr[u] = vis ? ex2(__uint_as_float(sv[2 * e + u]) * sc - svec[c]) : 0.f;
+            ds[u] = vis ? pr[u] * (__uint_as_float(dp[2 * e + u]) - svec[64 + c]) : 0.f;
+          }
+          pp[e] = pack_bf16(pr[0], pr[1]);
+          pd[e] = pack_bf16(ds[0], ds[1]);
+        }
+        tmem_st16(tmem + lane_off + 128 * w + 16 * half, pp);
+        tmem_st16(tmem + lane_off + 128 * w + 64 + 16 * half, pd);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->ps_full[w]);
+    }
+    __syncwarp();
+    if (failed) bars->abort_flag = 1;
+    mbar_wait(&bars->acc_done, 0, p.dev_status, &failed);
+    tc_fence_after();
+    asm volatile("bar.sync 2, 256;" ::: "memory");
+    const bool store = key < p.seqlen && !bars->abort_flag;
+    // warpgroup 0 writes dV, warpgroup 1 writes dK (scaled by 1/sqrt(d))
+    float* dst = (w == 0 ? p.dv : p.dk) + (((size_t)b * p.seqlen + key) * p.kv_heads + g) * 128;
+    const uint32_t col = w == 0 ? kColDV : kColDK;
+    const float mul = w == 0 ? 1.f : p.scale;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + col + 32 * c, v);
+      tc_wait_ld();
+      if (store) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float4 f;
+          f.x = __uint_as_float(v[e]) * mul;
+          f.y = __uint_as_float(v[e + 1]) * mul;
+          f.z = __uint_as_float(v[e + 2]) * mul;
+          f.w = __uint_as_float(v[e + 3]) * mul;
+          *reinterpret_cast<float4*>(dst + 32 * c + e) = f;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Per row: the pre-norm output o = O_1 - lambda O_2 from the saved
+// normalised branch outputs, the norm backward (V1), do_1 = do and
+// do_2 = -lambda do (bf16, [B][N][units][2][128]), D_r = do_r . O_r and the
+// block's shares of dlambda and of the norm gain's gradient.
+constexpr int kPreWarps = 8;
+constexpr int kPreRows = 64;
+
+struct Pre2Args {
+  const __nv_bfloat16* obr;  // [B][N][units][2][128]
+  const __nv_bfloat16* dout; // [B][N][units][128]
+  __nv_bfloat16* dob;        // [B][N][units][2][128]
+  float* Dv;                 // [B][units][2][npad]
+  int B, N, units, npad;
+  const float* lambda;
+  int apply_norm;
+  const float* g;
+  float eps, post;
+  float* dlambda;
+  float* dg;
+};
+
+__global__ void __launch_bounds__(32 * kPreWarps) bwd_pre2_kernel(Pre2Args a) {
+  __shared__ float sh_dg[kPreWarps][128];
+  __shared__ float sh_dl[kPreWarps];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int u = blockIdx.y % a.units, b = blockIdx.y / a.units;
+  const float lam = a.lambda[u];
+  float dg[4] = {0.f, 0.f, 0.f, 0.f};
+  float dl = 0.f;
+  const int r0 = blockIdx.x * kPreRows;
+  for (int i = r0 + warp; i < min(r0 + kPreRows, a.N); i += kPreWarps) {
+    const size_t tok = ((size_t)b * a.N + i) * a.units + u;
+    float o1[4], o2[4], o[4], dy[4], d_o[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int c = lane + 32 * t;
+      o1[t] = __bfloat162float(a.obr[tok * 256 + c]);
+      o2[t] = __bfloat162float(a.obr[tok * 256 + 128 + c]);
+      o[t] = o1[t] - lam * o2[t];
+      dy[t] = __bfloat162float(a.dout[tok * 128 + c]);
+    }
+    if (a.apply_norm) {
+      float ss = 0.f, gdo = 0.f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float gc = a.g ? a.g[lane + 32 * t] : 1.f;
+        ss = fmaf(o[t], o[t], ss);
+        gdo = fmaf(gc * dy[t], o[t], gdo);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        gdo += __shfl_xor_sync(0xffffffffu, gdo, off);
+      }
+      const float rr = sqrtf(ss / 128.f + a.eps);
+      const float cr = a.post / rr, k2 = gdo / (128.f * rr * rr);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float gc = a.g ? a.g[lane + 32 * t] : 1.f;
+        d_o[t] = cr * (gc * dy[t] - o[t] * k2);
+        dg[t] = fmaf(dy[t] * o[t], cr, dg[t]);
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) d_o[t] = dy[t];
+    }
+    float s1 = 0.f, s2 = 0.f, sl = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int c = lane + 32 * t;
+      const __nv_bfloat16 b1 = __float2bfloat16_rn(d_o[t]);
+      const __nv_bfloat16 b2 = __float2bfloat16_rn(-lam * d_o[t]);
+      a.dob[tok * 256 + c] = b1;
+      a.dob[tok * 256 + 128 + c] = b2;
+      s1 = fmaf(__bfloat162float(b1), o1[t], s1);
+      s2 = fmaf(__bfloat162float(b2), o2[t], s2);
+      sl = fmaf(d_o[t], o2[t], sl);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+      sl += __shfl_xor_sync(0xffffffffu, sl, off);
+    }
+    if (lane == 0) {
+      const size_t vr = ((size_t)b * a.units + u) * 2 * a.npad + i;
+      a.Dv[vr] = s1;
+      a.Dv[vr + a.npad] = s2;
+    }
+    dl -= sl;
+  }
+#pragma unroll
+  for (int t = 0; t < 4; ++t) sh_dg[warp][lane + 32 * t] = dg[t];
+  if (lane == 0) sh_dl[warp] = dl;
+  __syncthreads();
+  if (threadIdx.x < 128 && a.dg) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPreWarps; ++w) s += sh_dg[w][threadIdx.x];
+    atomicAdd(a.dg + threadIdx.x, s);
+  }
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPreWarps; ++w) s += sh_dl[w];
+    atomicAdd(a.dlambda + u, s);
+  }
+}
+
+}  // namespace
+
+size_t fused_bwd_workspace_bytes(int batch, int seqlen, int units) {
+  const size_t npad = (size_t)((seqlen + 63) / 64) * 64;
+  const size_t vec = (size_t)batch * units * 2 * npad * 4;
+  const size_t big = (size_t)batch * seqlen * units * 256 * 2;
+  const size_t out = (size_t)batch * seqlen * units * 128 * 2;
+  return 2 * ((vec + 255) & ~size_t(255)) + 2 * ((big + 255) & ~size_t(255)) +
+         ((out + 255) & ~size_t(255)) + 256;
+}
+
+cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
+  const int B = a.fwd.batch, N = a.fwd.seqlen, U = a.fwd.heads;
+  const int npad = (N + 63) / 64 * 64;
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(a.workspace) + 255) & ~uintptr_t(255));
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base;
+    base += (bytes + 255) & ~size_t(255);
+    return p;
+  };
+  float* lse = reinterpret_cast<float*>(take((size_t)B * U * 2 * npad * 4));
+  float* Dv = reinterpret_cast<float*>(take((size_t)B * U * 2 * npad * 4));
+  __nv_bfloat16* obr = reinterpret_cast<__nv_bfloat16*>(take((size_t)B * N * U * 256 * 2));
+  __nv_bfloat16* dob = reinterpret_cast<__nv_bfloat16*>(take((size_t)B * N * U * 256 * 2));
+  void* fwd_out = take((size_t)B * N * U * 128 * 2);
+
+  // tensor maps: inputs as [B][N][heads][128] with 64-column boxes of 128
+  // or 64 rows, and the saved upstream gradients [B][N][2U][128]
+  const int qh = a.fwd.form == 1 ? U : 2 * U, kvh = a.fwd.kv_heads;
+  CUtensorMap tq128, tq64, tk64, tk128, tv64, tv128, tdo128, tdo64;
+  if (make_tmap_bf16_4d(&tq128, a.q, 128, qh, N, B, 64, 1, 128, 1) ||
+      make_tmap_bf16_4d(&tq64, a.q, 128, qh, N, B, 64, 1, 64, 1) ||
+      make_tmap_bf16_4d(&tk64, a.k, 128, kvh, N, B, 64, 1, 64, 1) ||
+      make_tmap_bf16_4d(&tk128, a.k, 128, kvh, N, B, 64, 1, 128, 1) ||
+      make_tmap_bf16_4d(&tv64, a.v, 128, kvh, N, B, 64, 1, 64, 1) ||
+      make_tmap_bf16_4d(&tv128, a.v, 128, kvh, N, B, 64, 1, 128, 1) ||
+      make_tmap_bf16_4d(&tdo128, dob, 128, 2 * U, N, B, 64, 1, 128, 1) ||
+      make_tmap_bf16_4d(&tdo64, dob, 128, 2 * U, N, B, 64, 1, 64, 1))
+    return cudaErrorInvalidValue;
+  // 1. training forward: lse and the normalised branch outputs (lse rows are
+  // read in 64-entry blocks, so the padding is zeroed first)
+  cudaError_t e = cudaMemsetAsync(lse, 0, (size_t)B * U * 2 * npad * 4, st);
+  if (e != cudaSuccess) return e;
+  PrefillArgs fa = a.fwd;
+  fa.out = fwd_out;
+  fa.lse = lse;
+  fa.lse_stride = npad;
+  fa.obr = obr;
+  e = launch_prefill_tc(tq128, tk64, tv64, fa, a.num_sms, st);
+  if (e != cudaSuccess) return e;
+  // 2. upstream gradients per branch, D, dlambda, gain gradient
+  if ((e = cudaMemsetAsync(Dv, 0, (size_t)B * U * 2 * npad * 4, st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(a.dlambda, 0, (size_t)U * 4, st)) != cudaSuccess ||
+      (a.dg && (e = cudaMemsetAsync(a.dg, 0, 128 * 4, st)) != cudaSuccess))
+    return e;
+  Pre2Args pa;
+  pa.obr = obr;
+  pa.dout = static_cast<const __nv_bfloat16*>(a.dout);
+  pa.dob = dob;
+  pa.Dv = Dv;
+  pa.B = B;
+  pa.N = N;
+  pa.units = U;
+  pa.npad = npad;
+  pa.lambda = a.fwd.lambda;
+  pa.apply_norm = a.fwd.apply_norm;
+  pa.g = a.fwd.norm_weight;
+  pa.eps = a.fwd.eps;
+  pa.post = a.fwd.post_scale;
+  pa.dlambda = a.dlambda;
+  pa.dg = a.fwd.apply_norm ? a.dg : nullptr;
+  bwd_pre2_kernel<<<dim3((N + kPreRows - 1) / kPreRows, B * U), 32 * kPreWarps, 0, st>>>(pa);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  BwdParams p;
+  p.batch = B;
+  p.seqlen = N;
+  p.units = U;
+  p.pairs_per_kv = a.fwd.pairs_per_kv;
+  p.causal = a.fwd.causal;
+  p.window = a.fwd.window;
+  p.npad = npad;
+  const double d = a.fwd.form == 1 ? 64.0 : 128.0;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(d));
+  p.scale = (float)(1.0 / std::sqrt(d));
+  p.lse = lse;
+  p.Dv = Dv;
+  p.dq = a.dq;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.q_heads = qh;
+  p.kv_heads = a.fwd.kv_heads;
+  p.n_qtiles = (N + 127) / 128;
+  p.n_ktiles = (N + 127) / 128;
+  p.dev_status = a.fwd.dev_status;
+  const bool win = a.fwd.window > 0;
+  // 4. dQ
+  {
+    const int qbytes = a.fwd.form == 1 ? kTile128 : 2 * kTile128;
+    const int smem = 1024 + qbytes + 2 * kTile128 + 2 * kDqStages * kTile64 +
+                     (int)sizeof(DqBarriers) + 64;
+    decltype(&diffattn_bwd_dq_kernel<1, false>) k =
+        a.fwd.form == 1 ? (win ? diffattn_bwd_dq_kernel<1, true> : diffattn_bwd_dq_kernel<1, false>)
+                        : (win ? diffattn_bwd_dq_kernel<2, true> : diffattn_bwd_dq_kernel<2, false>);
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return e;
+    k<<<p.n_qtiles * B * U, kDqThreads, smem, st>>>(tq128, tdo128, tk64, tv64, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 5. dK, dV
+  {
+    const int smem = 1024 + 2 * kTile128 + kKvStages * kStageBytes + (int)sizeof(KvBarriers) + 64;
+    decltype(&diffattn_bwd_dkdv_kernel<1, false>) k =
+        a.fwd.form == 1
+            ? (win ? diffattn_bwd_dkdv_kernel<1, true> : diffattn_bwd_dkdv_kernel<1, false>)
+            : (win ? diffattn_bwd_dkdv_kernel<2, true> : diffattn_bwd_dkdv_kernel<2, false>);
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return e;
+    k<<<p.n_ktiles * B * a.fwd.kv_heads, kKvThreads, smem, st>>>(tq64, tdo64, tk128, tv128, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace da

@@ -96,10 +96,31 @@ struct PrefillArgs {
   const float* norm_weight;
   float eps, post_scale;
   void* out;
+  float* lse;  // optional training saves (see the kernel's Params)
+  int lse_stride;
+  void* obr;
   int* dev_status;
 };
 cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                               const CUtensorMap& tm_v, const PrefillArgs& a, int num_sms,
                               cudaStream_t stream);
+
+// ---- fused tcgen05 backward (bf16; V1 d_qk 64 / d_v 128, V2 head_dim 128) --
+struct FusedBwdArgs {
+  PrefillArgs fwd;  // the forward's problem (out/lse/obr are set internally)
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;  // [B][N][units][128] bf16
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dlambda;    // [units]
+  float* dg;         // [128] or nullptr
+  void* workspace;   // fused_bwd_workspace_bytes
+  int num_sms;
+};
+size_t fused_bwd_workspace_bytes(int batch, int seqlen, int units);
+cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t stream);
 
 }  // namespace da

@@ -90,6 +90,12 @@ struct Params {
   const float* norm_weight;
   float eps, post_scale;
   __nv_bfloat16* out;
+  // training saves (nullptr when not wanted): per-row log2-sum-exp of each
+  // branch [B][units][2][lse_stride], and each branch's normalised output
+  // O_r / l_r as bf16 [B][N][units][2][128]
+  float* lse;
+  int lse_stride;  // row stride of lse (>= seqlen)
+  __nv_bfloat16* obr;
   int* dev_status;
 };
 
@@ -99,7 +105,8 @@ __device__ __forceinline__ uint32_t s_col(int r, int buf) {
 
 // kForm: 1 = V1 (d_qk 64 per branch, one head), 2 = V2 (d 128 per branch, a head pair).
 // kWindow: sliding-window masking compiled in (p.window > 0) or out.
-template <int kForm, bool kWindow>
+// kSave: also write the training saves p.lse and p.obr.
+template <int kForm, bool kWindow, bool kSave>
 __global__ void __launch_bounds__(kThreads, 1)
     diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
@@ -383,10 +390,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               &failed);
     tc_fence_after();
     x_inv_l[r * kBM + row] = 1.0f / l_run;
+    if (kSave && qrow < p.seqlen)  // p_ij = 2^(s_ij * sc - lse) for the backward
+      p.lse[(((size_t)b * p.heads + hh) * 2 + r) * p.lse_stride + qrow] =
+          (m_ref == -INFINITY ? 0.f : m_ref) + log2f(l_run);
     asm volatile("bar.sync 2, 256;" ::: "memory");
     tc_fence_after();
     const float inv1 = x_inv_l[row];
-    const float inv2 = x_inv_l[kBM + row] * p.lambda[hh];
+    const float inv2_raw = x_inv_l[kBM + row];
+    const float inv2 = inv2_raw * p.lambda[hh];
     float o[64];
     {
       uint32_t a[32], c2[32];
@@ -398,6 +409,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           o[half * 32 + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
+        if (kSave && qrow < p.seqlen) {
+          __nv_bfloat16* ob = p.obr + (((size_t)b * p.seqlen + qrow) * p.heads + hh) * 256 +
+                              64 * r + 32 * half;
+#pragma unroll
+          for (int v8 = 0; v8 < 4; ++v8) {
+            uint4 w1, w2;
+            w1.x = pack_bf16(__uint_as_float(a[8 * v8 + 0]) * inv1, __uint_as_float(a[8 * v8 + 1]) * inv1);
+            w1.y = pack_bf16(__uint_as_float(a[8 * v8 + 2]) * inv1, __uint_as_float(a[8 * v8 + 3]) * inv1);
+            w1.z = pack_bf16(__uint_as_float(a[8 * v8 + 4]) * inv1, __uint_as_float(a[8 * v8 + 5]) * inv1);
+            w1.w = pack_bf16(__uint_as_float(a[8 * v8 + 6]) * inv1, __uint_as_float(a[8 * v8 + 7]) * inv1);
+            w2.x = pack_bf16(__uint_as_float(c2[8 * v8 + 0]) * inv2_raw, __uint_as_float(c2[8 * v8 + 1]) * inv2_raw);
+            w2.y = pack_bf16(__uint_as_float(c2[8 * v8 + 2]) * inv2_raw, __uint_as_float(c2[8 * v8 + 3]) * inv2_raw);
+            w2.z = pack_bf16(__uint_as_float(c2[8 * v8 + 4]) * inv2_raw, __uint_as_float(c2[8 * v8 + 5]) * inv2_raw);
+            w2.w = pack_bf16(__uint_as_float(c2[8 * v8 + 6]) * inv2_raw, __uint_as_float(c2[8 * v8 + 7]) * inv2_raw);
+            *reinterpret_cast<uint4*>(ob + 8 * v8) = w1;
+            *reinterpret_cast<uint4*>(ob + 128 + 8 * v8) = w2;
+          }
+        }
       }
     }
     float mul = 1.f;
@@ -473,15 +502,25 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.eps = a.eps;
   p.post_scale = a.post_scale;
   p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.lse_stride = a.lse_stride;
+  p.obr = static_cast<__nv_bfloat16*>(a.obr);
   p.dev_status = a.dev_status;
   const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
   const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +
                    4 * kBM * (int)sizeof(float) + 64;
   const bool win = a.window > 0;
-  auto kern = a.form == 1 ? (win ? diffattn_prefill_tc_kernel<1, true>
-                                 : diffattn_prefill_tc_kernel<1, false>)
-                          : (win ? diffattn_prefill_tc_kernel<2, true>
-                                 : diffattn_prefill_tc_kernel<2, false>);
+  decltype(&diffattn_prefill_tc_kernel<1, false, false>) kern;
+  if (a.lse && a.obr)  // training forward
+    kern = a.form == 1 ? (win ? diffattn_prefill_tc_kernel<1, true, true>
+                              : diffattn_prefill_tc_kernel<1, false, true>)
+                       : (win ? diffattn_prefill_tc_kernel<2, true, true>
+                              : diffattn_prefill_tc_kernel<2, false, true>);
+  else
+    kern = a.form == 1 ? (win ? diffattn_prefill_tc_kernel<1, true, false>
+                              : diffattn_prefill_tc_kernel<1, false, false>)
+                       : (win ? diffattn_prefill_tc_kernel<2, true, false>
+                              : diffattn_prefill_tc_kernel<2, false, false>);
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

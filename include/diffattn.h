@@ -244,7 +244,7 @@ DA_API int diffattn_v1_decode_window(const void* q, const void* k_cache, const v
  * fp32, written (not accumulated) in the layout of the matching input.
  * Outputs must not overlap inputs or each other.
  *
- * This implementation materialises the two attention maps of one head (V1)
+ * For widths outside the tensor-core forward the implementation materialises the two attention maps of one head (V1)
  * or head pair (V2) for a chunk of batch entries at a time in `workspace`
  * (size from the *_workspace_size query; about 10 N^2 bytes per batch entry
  * of a chunk) and issues its six matrix products per branch as
@@ -252,7 +252,16 @@ DA_API int diffattn_v1_decode_window(const void* q, const void* k_cache, const v
  * first call on a device creates that device's cuBLAS handle, which
  * allocates cuBLAS's own workspace; calls on one device are serialised on
  * the host while they enqueue.  Errors: as for the forward, plus
- * DA_ERR_WORKSPACE for a missing or short workspace. */
+ * DA_ERR_WORKSPACE for a missing or short workspace.
+ *
+ * The shapes of the tensor-core forward (V1 d_qk 64 / d_v 128, V2 head_dim
+ * 128) take a fused path instead: the forward kernel re-runs with saves
+ * (per-row log-sum-exp and normalised branch outputs), then one kernel
+ * accumulates dQ per query tile and one accumulates dK and dV per key tile
+ * in tensor memory, recomputing the maps tile by tile; no N x N buffer
+ * exists and the workspace is about (8 units + 2 units) x N x 128 bf16 per
+ * batch entry.  `dev_status` (optional) receives DA_ERR_DEVICE_TIMEOUT if
+ * one of its bounded waits ever times out. */
 
 /* V1.  q, k: device [batch, seqlen, n_heads, 2*d_qk]; v, dout: device
  * [batch, seqlen, n_heads, d_v] (bf16); lambda [n_heads] fp32; norm as in
@@ -268,7 +277,7 @@ DA_API int diffattn_v1_bwd(const void* q, const void* k, const void* v, const vo
                            int apply_norm, const float* norm_weight, float norm_eps,
                            float lambda_init, float* dq, float* dk, float* dv, float* dlambda,
                            float* dnorm_weight, void* workspace, size_t workspace_bytes,
-                           void* stream);
+                           int* dev_status, void* stream);
 
 /* V2.  q: device [batch, seqlen, n_q_heads, head_dim]; k, v: device
  * [batch, seqlen, n_kv_heads, head_dim]; dout: device [batch, seqlen,
@@ -281,7 +290,7 @@ DA_API int diffattn_v2_bwd(const void* q, const void* k, const void* v, const vo
                            const float* lambda, da_dtype dtype, int batch, int seqlen,
                            int n_q_heads, int n_kv_heads, int head_dim, int causal, int window,
                            float* dq, float* dk, float* dv, float* dlambda, void* workspace,
-                           size_t workspace_bytes, void* stream);
+                           size_t workspace_bytes, int* dev_status, void* stream);
 
 /* Gradients of the four lambda vectors (device fp32 [n_heads, dim]) of
  * lambda_from_params, from dlambda [n_heads]:

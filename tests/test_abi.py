@@ -170,12 +170,14 @@ def test_window_variants_host_validation(lib):
 
 def test_backward_host_validation(lib):
     from differential_attention_sm_b200 import binding as b
-    ws = b.diffattn_v1_bwd_workspace_size(4, 4096, 16, 64, 128)
-    assert ws >= 4 * 10 * 4096 * 4096
+    ws = b.diffattn_v1_bwd_workspace_size(4, 4096, 16, 64, 128)   # fused path
+    assert ws >= 4 * 4096 * 16 * 128 * 2 * 5                       # no N x N buffers
+    assert ws < 4 * 10 * 4096 * 4096                               # vs 10 N^2 per entry
+    assert b.diffattn_v1_bwd_workspace_size(4, 4096, 16, 32, 64) >= 4 * 10 * 4096 * 4096
     assert b.diffattn_v1_bwd_workspace_size(0, 4096, 16, 64, 128) == 0
     f = lib.diffattn_v1_bwd
     ok = [A, A, A, A, A, b.DA_BF16, 4, 4096, 16, 64, 128, 1, 0, 1, None, 1e-5, 0.2, A, A, A, A,
-          None, A, ws, None]
+          None, A, ws, None, None]
     bad = list(ok); bad[22] = None
     assert f(*bad) == b.DA_ERR_WORKSPACE
     bad = list(ok); bad[23] = ws - 1
@@ -190,7 +192,7 @@ def test_backward_host_validation(lib):
     assert f(*bad) == b.DA_ERR_ALIGNMENT
     g = lib.diffattn_v2_bwd
     ws2 = b.diffattn_v2_bwd_workspace_size(2, 8192, 32, 8, 128)
-    ok = [A, A, A, A, A, b.DA_BF16, 2, 8192, 32, 8, 128, 1, 0, A, A, A, A, A, ws2, None]
+    ok = [A, A, A, A, A, b.DA_BF16, 2, 8192, 32, 8, 128, 1, 0, A, A, A, A, A, ws2, None, None]
     bad = list(ok); bad[8] = 6                         # group 32/6 not an integer
     assert g(*bad) == b.DA_ERR_INVALID_ARG
     bad = list(ok); bad[10] = 256
