@@ -19,15 +19,16 @@
 //     into tensor memory (two SS MMAs), dS_r written back over S_r as bf16
 //     by the softmax-backward warps, then dQ_r += dS_r K_r (TS MMA) in
 //     tensor memory.  Warps: 0-3 / 4-7 branch 1 / 2 (thread = query row),
-//     8 TMA producer, 9 / 10 score-and-dP issuers, 11 / 12 dQ issuers.
+//     8 TMA producer, 9-12 the S_r and dP_r issuers (one thread per product
+//     stream, as in the forward), 13 / 14 dQ issuers.
 //   * dkdv kernel, one CTA per 128 keys of a head (V1) or KV head (V2),
 //     walking 64-query tiles (and, for V2, every pair that reads the KV
 //     head): S^T = K_r Q_r^T and dP^T = V do_r^T (SS), P^T and dS^T written
 //     back as bf16 by the softmax-backward warps (thread = key row), then
-//     dV += P^T do_r and dK_r += dS^T Q_r (TS) in tensor memory.  Both
-//     accumulations are issued by one thread, so their order is fixed.
+//     dV += P^T do_r and dK_r += dS^T Q_r (TS) in tensor memory.  Each
+//     accumulator has one issuing thread, so its order is fixed.
 //     Warps: 0-3 / 4-7 alternate steps (= branches), 8 producer,
-//     9 score-and-dP issuer, 10 accumulation issuer.
+//     9 S^T issuer, 10 dP^T issuer, 11 dV issuer, 12 dK issuer.
 // Every wait is bounded (DA_ERR_DEVICE_TIMEOUT in the status word).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -64,7 +65,7 @@ struct BwdParams {
 };
 
 // ===================================================================== dQ
-constexpr int kDqThreads = 416;
+constexpr int kDqThreads = 480;
 constexpr int kDqStages = 2;
 
 struct DqBarriers {
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       mbar_init(&bars->v_empty[s], 2);
     }
     for (int r = 0; r < 2; ++r) {
-      mbar_init(&bars->sd_full[r], 1);
+      mbar_init(&bars->sd_full[r], 2);  // S_r and dP_r, from their own issuers
       mbar_init(&bars->ds_full[r], 128);
       mbar_init(&bars->dq_done[r], 1);
     }
@@ -167,50 +168,57 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tma_load_4d(sV + s * kTile64 + kBox64, &tm_v, &bars->v_full[s], 64, kvh, row, b);
       }
     }
-  } else if (warp == 9 || warp == 10) {
-    if (lane == 0) {  // ------------------------- S_r and dP_r issuer, r = warp - 9
-      const int r = warp - 9;
+  } else if (warp >= 9 && warp <= 12) {
+    if (lane == 0) {  // ---- S_r issuer (kind 0) or dP_r issuer (kind 1): warp 9 + 2r + kind
+      const int r = (warp - 9) >> 1, kind = (warp - 9) & 1;
       const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO) + r * kTile128;
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
         for (int j = 0; j < n_kv; ++j) {
           const int s = j % kDqStages;
           const uint32_t ph = (uint32_t)(j / kDqStages) & 1u;
-          if (!mbar_wait(&bars->k_full[s], ph, p.dev_status, &failed)) break;
-          if (!mbar_wait(&bars->v_full[s], ph, p.dev_status, &failed)) break;
-          // S_r / dP_r buffers last held tile j-1: its dS_r must have been consumed
-          if (j > 0 && !mbar_wait(&bars->dq_done[r], (uint32_t)(j - 1) & 1u, p.dev_status,
-                                  &failed))
+          if (!mbar_wait(kind == 0 ? &bars->k_full[s] : &bars->v_full[s], ph, p.dev_status,
+                         &failed))
+            break;
+          // S_r's buffer last held dS_r(j-1): the dQ product must have read it;
+          // dP_r's buffer is free once the softmax backward has read dP_r(j-1)
+          if (j > 0 && !mbar_wait(kind == 0 ? &bars->dq_done[r] : &bars->ds_full[r],
+                                  (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
             break;
           tc_fence_after();
-          const uint32_t kt = smem_u32(sK) + s * kTile64, vt = smem_u32(sV) + s * kTile64;
-          for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t a, bb;
-            if (kForm == 1) {
-              a = q_addr + r * kBox128 + kk * 32;
-              bb = kt + r * kBox64 + kk * 32;
-            } else {
-              a = q_addr + r * kTile128 + (kk >> 2) * kBox128 + (kk & 3) * 32;
-              bb = kt + (kk >> 2) * kBox64 + (kk & 3) * 32;
+          if (kind == 0) {
+            const uint32_t kt = smem_u32(sK) + s * kTile64;
+            for (int kk = 0; kk < D / 16; ++kk) {
+              uint32_t a, bb;
+              if (kForm == 1) {
+                a = q_addr + r * kBox128 + kk * 32;
+                bb = kt + r * kBox64 + kk * 32;
+              } else {
+                a = q_addr + r * kTile128 + (kk >> 2) * kBox128 + (kk & 3) * 32;
+                bb = kt + (kk >> 2) * kBox64 + (kk & 3) * 32;
+              }
+              tc_mma_ss(tmem + colS(r), smem_desc_sw128(a, 16, 1024),
+                        smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
-            tc_mma_ss(tmem + colS(r), smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bb, 16, 1024),
-                      idS, kk > 0 ? 1u : 0u);
+            tc_commit(&bars->sd_full[r]);
+            tc_commit(&bars->k_empty[s]);
+          } else {
+            const uint32_t vt = smem_u32(sV) + s * kTile64;
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t a = do_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
+              const uint32_t bb = vt + (kk >> 2) * kBox64 + (kk & 3) * 32;
+              tc_mma_ss(tmem + colP(r), smem_desc_sw128(a, 16, 1024),
+                        smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars->sd_full[r]);
+            tc_commit(&bars->v_empty[s]);
           }
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a = do_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
-            const uint32_t bb = vt + (kk >> 2) * kBox64 + (kk & 3) * 32;
-            tc_mma_ss(tmem + colP(r), smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bb, 16, 1024),
-                      idS, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&bars->sd_full[r]);
-          tc_commit(&bars->v_empty[s]);
-          tc_commit(&bars->k_empty[s]);
         }
       }
     }
-  } else if (warp == 11 || warp == 12) {
-    if (lane == 0) {  // ------------------------------------ dQ_r issuer, r = warp - 11
-      const int r = warp - 11;
+  } else if (warp == 13 || warp == 14) {
+    if (lane == 0) {  // ------------------------------------ dQ_r issuer, r = warp - 13
+      const int r = warp - 13;
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kDqStages;
@@ -308,7 +316,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 }
 
 // =================================================================== dK, dV
-constexpr int kKvThreads = 352;
+constexpr int kKvThreads = 416;
 constexpr int kKvStages = 3;
 constexpr int kStageQ = kTile64;                       // Q_r tile (V1 uses one box)
 // + dO_r tile + lse/D vectors; a multiple of 1 KB keeps every stage's
@@ -319,7 +327,7 @@ static_assert(kStageBytes % 1024 == 0, "stage alignment");
 struct KvBarriers {
   uint64_t kv_full;
   uint64_t qd_full[kKvStages], qd_empty[kKvStages];
-  uint64_t sd_full[2], ps_full[2], buf_free[2];
+  uint64_t sd_full[2], ps_full[2], pt_free[2], dst_free[2];
   uint64_t acc_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -357,14 +365,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < kKvStages; ++s) {
       mbar_init(&bars->qd_full[s], 1);
-      mbar_init(&bars->qd_empty[s], 2);  // both issuers read Q_r and dO_r
+      mbar_init(&bars->qd_empty[s], 4);  // all four products read Q_r or dO_r
     }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&bars->sd_full[w], 1);
+      mbar_init(&bars->sd_full[w], 2);  // S^T and dP^T, from their own issuers
       mbar_init(&bars->ps_full[w], 128);
-      mbar_init(&bars->buf_free[w], 1);
+      mbar_init(&bars->pt_free[w], 1);
+      mbar_init(&bars->dst_free[w], 1);
     }
-    mbar_init(&bars->acc_done, 1);
+    mbar_init(&bars->acc_done, 2);
     bars->abort_flag = 0;
     fence_barrier_init();
   }
@@ -418,8 +427,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         bulk_load(svec + 64, p.Dv + vrow, 256, &bars->qd_full[st]);
       }
     }
-  } else if (warp == 9) {
-    if (lane == 0) {  // ---------------------------------- S^T and dP^T issuer
+  } else if (warp == 9 || warp == 10) {
+    if (lane == 0) {  // ------------------ S^T issuer (warp 9) and dP^T issuer (warp 10)
+      const bool is_s = warp == 9;
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       if (mbar_wait(&bars->kv_full, 0, p.dev_status, &failed)) {
@@ -428,57 +438,64 @@ __global__ void __launch_bounds__(kKvThreads, 1)
           if (!mbar_wait(&bars->qd_full[st], (uint32_t)(s / kKvStages) & 1u, p.dev_status,
                          &failed))
             break;
-          if (s >= 2 && !mbar_wait(&bars->buf_free[w], (uint32_t)((s - 2) >> 1) & 1u,
-                                   p.dev_status, &failed))
+          // the buffer last held step s-2's P^T (read by the dV product) or
+          // dS^T (read by the dK product)
+          if (s >= 2 && !mbar_wait(is_s ? &bars->pt_free[w] : &bars->dst_free[w],
+                                   (uint32_t)((s - 2) >> 1) & 1u, p.dev_status, &failed))
             break;
           tc_fence_after();
           const uint32_t sq = smem_u32(sStage) + st * kStageBytes, sdo = sq + kStageQ;
-          for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t a, bb;
-            if (kForm == 1) {
-              a = k_addr + r * kBox128 + kk * 32;
-              bb = sq + kk * 32;
-            } else {
-              a = k_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
-              bb = sq + (kk >> 2) * kBox64 + (kk & 3) * 32;
+          if (is_s) {
+            for (int kk = 0; kk < D / 16; ++kk) {
+              uint32_t a, bb;
+              if (kForm == 1) {
+                a = k_addr + r * kBox128 + kk * 32;
+                bb = sq + kk * 32;
+              } else {
+                a = k_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
+                bb = sq + (kk >> 2) * kBox64 + (kk & 3) * 32;
+              }
+              tc_mma_ss(tmem + 128 * w, smem_desc_sw128(a, 16, 1024),
+                        smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
-            tc_mma_ss(tmem + 128 * w, smem_desc_sw128(a, 16, 1024),
-                      smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
-          }
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a = v_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
-            const uint32_t bb = sdo + (kk >> 2) * kBox64 + (kk & 3) * 32;
-            tc_mma_ss(tmem + 128 * w + 64, smem_desc_sw128(a, 16, 1024),
-                      smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          } else {
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t a = v_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
+              const uint32_t bb = sdo + (kk >> 2) * kBox64 + (kk & 3) * 32;
+              tc_mma_ss(tmem + 128 * w + 64, smem_desc_sw128(a, 16, 1024),
+                        smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
           }
           tc_commit(&bars->sd_full[w]);
           tc_commit(&bars->qd_empty[st]);
         }
       }
     }
-  } else if (warp == 10) {
-    if (lane == 0) {  // ------------------------------ dV and dK accumulation issuer
+  } else if (warp == 11 || warp == 12) {
+    if (lane == 0) {  // -------------- dV issuer (warp 11) and dK issuer (warp 12)
+      // each accumulator has one issuing thread, so its order is fixed
+      const bool is_v = warp == 11;
       constexpr uint32_t idV = idesc_bf16_f32(128, 128, false, true);
       constexpr uint32_t idK = idesc_bf16_f32(128, D, false, true);
-      bool first_v = true, first_k[2] = {true, true};
+      bool first[2] = {true, true};
       for (int s = 0; s < n_steps; ++s) {
         const int st = s % kKvStages, w = s & 1, r = s & 1;
         if (!mbar_wait(&bars->ps_full[w], (uint32_t)(s >> 1) & 1u, p.dev_status, &failed))
           break;
         tc_fence_after();
         const uint32_t sq = smem_u32(sStage) + st * kStageBytes, sdo = sq + kStageQ;
-        const int kb = kForm == 1 ? r : 0;
+        const int fb = (is_v || kForm == 2) ? 0 : r;  // accumulator of this step
         for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step; B operands MN-major
-          tc_mma_ts(tmem + kColDV, tmem + 128 * w + kk * 8,
-                    smem_desc_sw128(sdo + kk * 2048, kBox64, 1024), idV,
-                    (first_v && kk == 0) ? 0u : 1u);
-          tc_mma_ts(tmem + kColDK + (kForm == 1 ? 64 * r : 0), tmem + 128 * w + 64 + kk * 8,
-                    smem_desc_sw128(sq + kk * 2048, kBox64, 1024), idK,
-                    (first_k[kb] && kk == 0) ? 0u : 1u);
+          const uint32_t acc = (first[fb] && kk == 0) ? 0u : 1u;
+          if (is_v)
+            tc_mma_ts(tmem + kColDV, tmem + 128 * w + kk * 8,
+                      smem_desc_sw128(sdo + kk * 2048, kBox64, 1024), idV, acc);
+          else
+            tc_mma_ts(tmem + kColDK + (kForm == 1 ? 64 * r : 0), tmem + 128 * w + 64 + kk * 8,
+                      smem_desc_sw128(sq + kk * 2048, kBox64, 1024), idK, acc);
         }
-        first_v = false;
-        first_k[kb] = false;
-        tc_commit(&bars->buf_free[w]);
+        first[fb] = false;
+        tc_commit(is_v ? &bars->pt_free[w] : &bars->dst_free[w]);
         tc_commit(&bars->qd_empty[st]);
       }
       tc_commit(&bars->acc_done);
