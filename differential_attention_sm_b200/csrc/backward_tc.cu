@@ -247,6 +247,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const float lse = qrow < p.seqlen ? p.lse[vrow] : 0.f;
     const float Dr = qrow < p.seqlen ? p.Dv[vrow] : 0.f;
     const float sc = p.scale_log2;
+    const uint64_t sc2 = f2pack(sc, sc), nl2 = f2pack(-lse, -lse), nd2 = f2pack(-Dr, -Dr);
     for (int j = 0; j < n_kv; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->sd_full[r], (uint32_t)j & 1u, p.dev_status,
                                              &failed))) {
@@ -255,6 +256,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       }
       tc_fence_after();
       const int k0 = (kv0 + j) * 64;
+      // tiles fully inside every row's visible range skip the masks
+      const bool full = __all_sync(0xffffffffu, k0 + 64 <= lim && (!kWindow || k0 >= lo));
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t sv[32], dp[32], pk[16];
@@ -263,15 +266,24 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tc_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = k0 + 32 * half + 2 * e + u;
-            const bool vis = key < lim && (!kWindow || key >= lo);
-            const float pr = vis ? ex2(__uint_as_float(sv[2 * e + u]) * sc - lse) : 0.f;
-            ds[u] = vis ? pr * (__uint_as_float(dp[2 * e + u]) - Dr) : 0.f;
+          // p = 2^(s sc - lse), ds = p (dP - D): packed pairs
+          float x0, x1;
+          f2unpack(fma2(f2pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                        sc2, nl2),
+                   x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          if (!full) {
+            const int key = k0 + 32 * half + 2 * e;
+            p0 = (key < lim && (!kWindow || key >= lo)) ? p0 : 0.f;
+            p1 = (key + 1 < lim && (!kWindow || key + 1 >= lo)) ? p1 : 0.f;
           }
-          pk[e] = pack_bf16(ds[0], ds[1]);
+          float ds0, ds1;
+          f2unpack(fma2(f2pack(p0, p1),
+                        add2(f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                             nd2),
+                        0ull),
+                   ds0, ds1);
+          pk[e] = pack_bf16(ds0, ds1);
         }
         tmem_st16(tmem + lane_off + colS(r) + 16 * half, pk);
       }
@@ -521,6 +533,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       const int q0 = step_q0(s);
       const float* svec =
           reinterpret_cast<const float*>(sStage + st * kStageBytes + kStageQ + kTile64);
+      // query columns this key row sees in the step: [c_lo, c_hi)
+      int c_lo = 0, c_hi = min(64, p.seqlen - q0);
+      if (key >= p.seqlen) c_hi = 0;
+      if (p.causal) c_lo = max(0, key - q0);
+      if (kWindow) c_hi = min(c_hi, key + p.window - q0);
+      const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == 64);
+      const uint64_t sc2 = f2pack(sc, sc);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t sv[32], dp[32], pp[16], pd[16];
@@ -528,20 +547,35 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         tmem_ld32(tmem + lane_off + 128 * w + 64 + 32 * half, dp);
         tc_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pr[2], ds[2];
+        for (int e4 = 0; e4 < 8; ++e4) {  // 4 query columns: lse and D by broadcast loads
+          const int c = 32 * half + 4 * e4;
+          const float4 L = *reinterpret_cast<const float4*>(svec + c);
+          const float4 Dd = *reinterpret_cast<const float4*>(svec + 64 + c);
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 32 * half + 2 * e + u;
-            const int q = q0 + c;
-            bool vis = q < p.seqlen && key < p.seqlen;
-            if (p.causal) vis = vis && q >= key;
-            if (kWindow) vis = vis && q - key < p.window;
-            pr[u] = vis ? ex2(__uint_as_float(sv[2 * e + u]) * sc - svec[c]) : 0.f;
-            ds[u] = vis ? pr[u] * (__uint_as_float(dp[2 * e + u]) - svec[64 + c]) : 0.f;
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e4 + h2;
+            const float l0 = h2 ? L.z : L.x, l1 = h2 ? L.w : L.y;
+            const float d0 = h2 ? Dd.z : Dd.x, d1 = h2 ? Dd.w : Dd.y;
+            // p = 2^(s sc - lse), ds = p (dP - D): packed pairs
+            float x0, x1;
+            f2unpack(fma2(f2pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                          sc2, f2pack(-l0, -l1)),
+                     x0, x1);
+            float p0 = ex2(x0), p1 = ex2(x1);
+            if (!full) {
+              const int cc = c + 2 * h2;
+              p0 = (cc >= c_lo && cc < c_hi) ? p0 : 0.f;
+              p1 = (cc + 1 >= c_lo && cc + 1 < c_hi) ? p1 : 0.f;
+            }
+            const uint64_t pr = f2pack(p0, p1);
+            const uint64_t dd = add2(
+                f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                f2pack(-d0, -d1));
+            float ds0, ds1;
+            f2unpack(fma2(pr, dd, 0ull), ds0, ds1);
+            pp[e] = pack_bf16(p0, p1);
+            pd[e] = pack_bf16(ds0, ds1);
           }
-          pp[e] = pack_bf16(pr[0], pr[1]);
-          pd[e] = pack_bf16(ds[0], ds[1]);
         }
         tmem_st16(tmem + lane_off + 128 * w + 16 * half, pp);
         tmem_st16(tmem + lane_off + 128 * w + 64 + 16 * half, pd);
