@@ -47,7 +47,7 @@ def v1_flops_per_pair(d, dv):
 
 def v1_bwd_flops_per_pair(d, dv):
     """Backward work per visible pair, both branches: recomputed scores (2d),
-    dP = dO V^T (2dv), dQ (2d), dK (2d) and dV (2dv) per branch."""
+    dP = dO V^T (2dv), dQ (2d), dK (2d) and dV (2dv) per branch (V2: d = dv)."""
     return 2 * (6 * d + 4 * dv)
 
 
@@ -497,6 +497,23 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         del q, k, v, dout, ws
         torch.cuda.empty_cache()
 
+    if want("v2_backward_bf16"):  # gradients at the V2 prefill shape (B2 Hq32 Hkv8 N8192)
+        w = wl("v2_prefill_bf16")
+        x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
+        q, k, v, lamt = (x[n].to(dev) for n in ("q", "k", "v", "lam"))
+        dout = torch.randn(w.B, w.N, w.Hq // 2, w.d, device=dev).to(torch.bfloat16)
+        ws = torch.empty(Bd.diffattn_v2_bwd_workspace_size(w.B, w.N, w.Hq, w.Hkv, w.d),
+                         dtype=torch.uint8, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v2_bwd(q, k, v, dout, lamt, causal=True,
+                                                  workspace=ws), 5, 2, stream)
+        flop = prefill_pairs(w.B, w.N, w.Hq // 2) * v1_bwd_flops_per_pair(w.d, w.d)
+        t = flop / (ms * 1e-3) / 1e12
+        out["v2_backward_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
+                                   "frac": round(t / peaks["bf16_tflops"], 4), "flop": flop,
+                                   "workspace_bytes": ws.numel()}
+        del q, k, v, dout, ws
+        torch.cuda.empty_cache()
+
     if want("snr_v1_decode"):  # noise-cancellation sweep, 6 configs x 11 lambdas, L 1024
         from differential_attention_sm_b200 import snr as S
         w = wl("snr_v1_decode")
@@ -608,7 +625,8 @@ def main():
     ap.add_argument("--only", default=None,
                     choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
                              "v1_decode_bf16", "snr_v1_decode", "v2_prefill_window_bf16",
-                             "v2_decode_window_bf16", "v1_backward_bf16"],
+                             "v2_decode_window_bf16", "v1_backward_bf16",
+                             "v2_backward_bf16"],
                     help="run just this secondary workload (one GPU) and print its numbers")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="with --only: smaller decode batch (profiling runs)")

@@ -128,3 +128,26 @@ def test_v1_backward_full_size_one_head(B):
                    apply_norm=True, eps=w.eps, lambda_init_value=li)
     for name in ("dq", "dk", "dv"):
         close(res[name][b:b + 1, :, h:h + 1], ref[name], "v1 full %s" % name)
+
+
+def test_v2_backward_full_size_one_pair(B):
+    """The V2 prefill shape (batch 2, 32 query heads on 8 KV heads, 8192,
+    causal): dQ of one head pair depends on that pair alone, so the oracle
+    runs on its slice (both pairs of the group stay in the slice, since dK
+    and dV sum over them)."""
+    w = I.WORKLOADS["v2_prefill_bf16"]
+    x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
+    dout = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed + 77)["q"][:, :, : w.Hq // 2].contiguous()
+    st = status_word()
+    res = B.diffattn_v2_bwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(dout), cuda(x["lam"]),
+                            causal=True, dev_status=st)
+    assert_status_ok(st)
+    # batch 1, KV head 5: query heads 20..23 (pairs 10, 11); a 2048-token prefix
+    # keeps the oracle in seconds (causal: rows < n depend on keys < n only)
+    b, g, n = 1, 5, 2048
+    qs = x["q"][b:b + 1, :n, 4 * g:4 * g + 4].contiguous()
+    ks = x["k"][b:b + 1, :n, g:g + 1].contiguous()
+    vs = x["v"][b:b + 1, :n, g:g + 1].contiguous()
+    ds = dout[b:b + 1, :n, 2 * g:2 * g + 2].contiguous()
+    ref = O.v2_bwd(qs, ks, vs, ds, x["lam"][2 * g:2 * g + 2], causal=True)
+    close(res["dq"][b:b + 1, :n, 4 * g:4 * g + 4], ref["dq"], "v2 full dq")
