@@ -514,6 +514,28 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         del q, k, v, dout, ws
         torch.cuda.empty_cache()
 
+    if want("v2_prefill_oproj_bf16"):  # V2 prefill + output projection to d_model 2048
+        w = wl("v2_prefill_bf16")
+        dm = 2048
+        x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
+        q, k, v, lamt = (x[n].to(dev) for n in ("q", "k", "v", "lam"))
+        W = (torch.randn(w.Hq // 2 * w.d, dm, device=dev) / (w.Hq // 2 * w.d) ** 0.5).to(
+            torch.bfloat16)
+        ws = torch.empty(Bd.diffattn_v2_prefill_oproj_workspace_size(w.B, w.N, w.Hq, w.d),
+                         dtype=torch.uint8, device=dev)
+        o = torch.empty(w.B, w.N, dm, dtype=torch.bfloat16, device=dev)
+        ms = time_call(lambda: Bd.diffattn_v2_prefill_oproj(q, k, v, lamt, W, workspace=ws,
+                                                            out=o), 20, 3, stream)
+        flop_att = prefill_pairs(w.B, w.N, w.Hq // 2) * v2_flops_per_pair(w.d)
+        flop_gemm = 2 * w.B * w.N * (w.Hq // 2 * w.d) * dm
+        t = (flop_att + flop_gemm) / (ms * 1e-3) / 1e12
+        out["v2_prefill_oproj_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s",
+                                        "ms": round(ms, 4),
+                                        "frac": round(t / peaks["bf16_tflops"], 4),
+                                        "flop": flop_att + flop_gemm, "d_model": dm}
+        del q, k, v, W, ws, o
+        torch.cuda.empty_cache()
+
     if want("snr_v1_decode"):  # noise-cancellation sweep, 6 configs x 11 lambdas, L 1024
         from differential_attention_sm_b200 import snr as S
         w = wl("snr_v1_decode")
@@ -626,7 +648,7 @@ def main():
                     choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
                              "v1_decode_bf16", "snr_v1_decode", "v2_prefill_window_bf16",
                              "v2_decode_window_bf16", "v1_backward_bf16",
-                             "v2_backward_bf16"],
+                             "v2_backward_bf16", "v2_prefill_oproj_bf16"],
                     help="run just this secondary workload (one GPU) and print its numbers")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="with --only: smaller decode batch (profiling runs)")

@@ -47,6 +47,8 @@ EXPORTS = (
     "diffattn_v2_bwd_workspace_size",
     "diffattn_v2_bwd",
     "lambda_from_params_bwd",
+    "diffattn_v2_prefill_oproj_workspace_size",
+    "diffattn_v2_prefill_oproj",
 )
 
 
@@ -125,6 +127,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.lambda_from_params_bwd.restype = _i
     lib.lambda_from_params_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
                                            _vp]
+    lib.diffattn_v2_prefill_oproj_workspace_size.restype = _sz
+    lib.diffattn_v2_prefill_oproj_workspace_size.argtypes = [_i, _i, _i, _i]
+    lib.diffattn_v2_prefill_oproj.restype = _i
+    lib.diffattn_v2_prefill_oproj.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                              _i, _i, _i, _i, _vp, _sz, _vp, _vp]
     _lib = lib
     return lib
 
@@ -426,3 +433,29 @@ def lambda_from_params_bwd(lq1, lk1, lq2, lk2, dlambda, stream=None):
         _ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), _ptr(dlambda), H, dim,
         *(_ptr(outs[n]) for n in ("dlq1", "dlk1", "dlq2", "dlk2")), _stream(stream)))
     return outs
+
+
+# ---- V2 prefill + output projection ------------------------------------------
+def diffattn_v2_prefill_oproj_workspace_size(batch, seqlen, n_q_heads, head_dim) -> int:
+    return int(load().diffattn_v2_prefill_oproj_workspace_size(batch, seqlen, n_q_heads,
+                                                                head_dim))
+
+
+def diffattn_v2_prefill_oproj(q, k, v, lam, w_o, *, causal=True, window=0, workspace=None,
+                              out=None, dev_status=None, stream=None):
+    """V2 prefill followed by out = o . w_o.  q [B, N, Hq, d]; k, v
+    [B, N, Hkv, d]; w_o [Hq/2 * d, d_model] bf16.  Returns [B, N, d_model]."""
+    _need_cuda(q, k, v, lam, w_o, dev_status)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    d_model = w_o.shape[1]
+    if workspace is None:
+        workspace = torch.empty(diffattn_v2_prefill_oproj_workspace_size(B, N, Hq, d),
+                                dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty(B, N, d_model, dtype=q.dtype, device=q.device)
+    _check("diffattn_v2_prefill_oproj", load().diffattn_v2_prefill_oproj(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(w_o), _ptr(out), _dtype_code(q), B, N, Hq,
+        Hkv, d, d_model, int(bool(causal)), int(window), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+    return out

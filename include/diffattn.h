@@ -301,6 +301,27 @@ DA_API int lambda_from_params_bwd(const float* lq1, const float* lk1, const floa
                                   float* dlq1, float* dlk1, float* dlq2, float* dlk2,
                                   void* stream);
 
+/* ---- V2 prefill + output projection ---------------------------------------
+ * Lesson "Atención Diferencial (V2)", "V1 vs V2: la diferencia" and step 5:
+ * the paired subtraction brings V2's doubled query heads back to Hq/2 heads
+ * of width head_dim, which then go through the output projection O_W.
+ * out[b, i, :] = o[b, i, :, :].flatten() . w_o, with o the output of
+ * diffattn_v2_prefill_window (same arguments) and
+ *   w_o : device [n_q_heads/2 * head_dim, d_model] bf16 (row-major)
+ *   out : device [batch, seqlen, d_model] bf16
+ * The attention output goes to `workspace` (size from the query), then one
+ * plain GEMM (cuBLAS; bf16 operands, fp32 accumulation) writes `out`.  The
+ * first call on a device creates that device's cuBLAS handle.  bf16 only.
+ * Errors as for diffattn_v2_prefill_window, plus DA_ERR_WORKSPACE. */
+DA_API size_t diffattn_v2_prefill_oproj_workspace_size(int batch, int seqlen, int n_q_heads,
+                                                       int head_dim);
+DA_API int diffattn_v2_prefill_oproj(const void* q, const void* k, const void* v,
+                                     const float* lambda, const void* w_o, void* out,
+                                     da_dtype dtype, int batch, int seqlen, int n_q_heads,
+                                     int n_kv_heads, int head_dim, int d_model, int causal,
+                                     int window, void* workspace, size_t workspace_bytes,
+                                     int* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -198,3 +198,23 @@ def test_backward_host_validation(lib):
     bad = list(ok); bad[10] = 256
     assert g(*bad) == b.DA_ERR_UNSUPPORTED
     assert lib.lambda_from_params_bwd(A, A, A, A, A, 0, 4, A, A, A, A, None) == b.DA_ERR_INVALID_ARG
+
+
+def test_oproj_host_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    ws = b.diffattn_v2_prefill_oproj_workspace_size(2, 8192, 32, 128)
+    assert ws >= 2 * 8192 * 16 * 128 * 2
+    f = lib.diffattn_v2_prefill_oproj
+    ok = [A, A, A, A, A, A, b.DA_BF16, 2, 8192, 32, 8, 128, 2048, 1, 0, A, ws, None, None]
+    bad = list(ok); bad[15] = None
+    assert f(*bad) == b.DA_ERR_WORKSPACE
+    bad = list(ok); bad[16] = ws - 1
+    assert f(*bad) == b.DA_ERR_WORKSPACE
+    bad = list(ok); bad[4] = None
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[12] = 0
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[6] = b.DA_FP32
+    assert f(*bad) == b.DA_ERR_UNSUPPORTED
+    bad = list(ok); bad[5] = U
+    assert f(*bad) == b.DA_ERR_ALIGNMENT
