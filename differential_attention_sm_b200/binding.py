@@ -49,6 +49,7 @@ EXPORTS = (
     "lambda_from_params_bwd",
     "diffattn_v2_prefill_oproj_workspace_size",
     "diffattn_v2_prefill_oproj",
+    "diffattn_selftest_wait_timeout",
 )
 
 
@@ -132,6 +133,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.diffattn_v2_prefill_oproj.restype = _i
     lib.diffattn_v2_prefill_oproj.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                               _i, _i, _i, _i, _vp, _sz, _vp, _vp]
+    lib.diffattn_selftest_wait_timeout.restype = _i
+    lib.diffattn_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp, _vp, _vp]
     _lib = lib
     return lib
 
@@ -459,3 +462,11 @@ def diffattn_v2_prefill_oproj(q, k, v, lam, w_o, *, causal=True, window=0, works
         Hkv, d, d_model, int(bool(causal)), int(window), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
     return out
+
+
+def diffattn_selftest_wait_timeout(timeout_us, dev_status, waited_ns=None, stream=None):
+    """Run the bounded-wait path to its timeout (see the header); the status
+    word then holds DA_ERR_DEVICE_TIMEOUT."""
+    _need_cuda(dev_status, waited_ns)
+    _check("diffattn_selftest_wait_timeout", load().diffattn_selftest_wait_timeout(
+        int(timeout_us), _ptr(dev_status), _ptr(waited_ns), _stream(stream)))

@@ -173,13 +173,13 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Bounded wait: returns false (after recording DA_ERR_DEVICE_TIMEOUT) if the
 // phase never completes.  `*failed` is sticky so later waits return at once.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* dev_status,
-                                          bool* failed) {
+                                          bool* failed, uint64_t limit_ns = DA_WAIT_NS) {
   if (*failed) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1; i < DA_WAIT_POLLS; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_ns() - t0 > DA_WAIT_NS) break;
+    if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) break;
   }
   *failed = true;
   report(dev_status, DA_ERR_DEVICE_TIMEOUT);

@@ -322,6 +322,17 @@ DA_API int diffattn_v2_prefill_oproj(const void* q, const void* k, const void* v
                                      int window, void* workspace, size_t workspace_bytes,
                                      int* dev_status, void* stream);
 
+/* ---- Self-test of the failure report ----------------------------------------
+ * No counterpart on the pages.  Launches one CTA whose thread waits on an
+ * mbarrier that nothing arrives on, using the pipelines' own bounded wait
+ * with a limit of `timeout_us` microseconds (1 .. 1000000).  The wait gives
+ * up, stores DA_ERR_DEVICE_TIMEOUT in *dev_status (device int, required;
+ * first error wins, zero it beforehand) and the kernel returns, leaving the
+ * context usable.  `waited_ns` (optional, device) receives the time waited.
+ * Returns DA_ERR_INVALID_ARG for a null status word or a limit out of range. */
+DA_API int diffattn_selftest_wait_timeout(unsigned int timeout_us, int* dev_status,
+                                          unsigned long long* waited_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -218,3 +218,11 @@ def test_oproj_host_validation(lib):
     assert f(*bad) == b.DA_ERR_UNSUPPORTED
     bad = list(ok); bad[5] = U
     assert f(*bad) == b.DA_ERR_ALIGNMENT
+
+
+def test_selftest_host_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    f = lib.diffattn_selftest_wait_timeout
+    assert f(1000, None, None, None) == b.DA_ERR_INVALID_ARG
+    assert f(0, A, None, None) == b.DA_ERR_INVALID_ARG
+    assert f(2000000, A, None, None) == b.DA_ERR_INVALID_ARG
