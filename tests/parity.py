@@ -1,6 +1,6 @@
 """Shared helpers of the GPU parity tests: tolerances and error measures.
 
-Tolerances (fixed by the task's accuracy statement for this operator):
+Tolerances (the operator's accuracy bounds):
   * fp32 workload: max |gpu - oracle| <= 1e-5;
   * bf16 V1 with the per-head norm (outputs are O(1)): max abs <= 2e-2 and
     mean abs <= 2e-3;
