@@ -72,7 +72,8 @@ struct DqBarriers {
   uint64_t q_full;
   uint64_t k_full[kDqStages], k_empty[kDqStages];
   uint64_t v_full[kDqStages], v_empty[kDqStages];
-  uint64_t sd_full[2], ds_full[2], dq_done[2];
+  uint64_t sd_full[2], ds_full[2];
+  uint64_t dq_done[2][2];  // [branch][S buffer]: the dQ product of a tile has read its dS
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -115,7 +116,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     for (int r = 0; r < 2; ++r) {
       mbar_init(&bars->sd_full[r], 2);  // S_r and dP_r, from their own issuers
       mbar_init(&bars->ds_full[r], 128);
-      mbar_init(&bars->dq_done[r], 1);
+      mbar_init(&bars->dq_done[r][0], 1);
+      mbar_init(&bars->dq_done[r][1], 1);
     }
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -128,8 +130,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  // tensor-memory columns: S_r, dP_r (64 each), dQ_r (D each)
-  auto colS = [](int r) { return (uint32_t)(128 * r); };
+  // tensor-memory columns: S_r, dP_r (64 each), dQ_r (D each); V1 leaves room
+  // for a second S buffer per branch at [384, 512), so S_r(j+1) can be computed
+  // while dS_r(j) still waits for its dQ product
+  constexpr int kSBufs = kForm == 1 ? 2 : 1;
+  auto colS = [](int r, int j) {
+    return (uint32_t)((kSBufs == 2 && (j & 1)) ? 384 + 64 * r : 128 * r);
+  };
   auto colP = [](int r) { return (uint32_t)(128 * r + 64); };
   auto colQ = [](int r) { return (uint32_t)(256 + D * r); };
   bool failed = false;
@@ -180,10 +187,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           if (!mbar_wait(kind == 0 ? &bars->k_full[s] : &bars->v_full[s], ph, p.dev_status,
                          &failed))
             break;
-          // S_r's buffer last held dS_r(j-1): the dQ product must have read it;
-          // dP_r's buffer is free once the softmax backward has read dP_r(j-1)
-          if (j > 0 && !mbar_wait(kind == 0 ? &bars->dq_done[r] : &bars->ds_full[r],
-                                  (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
+          // S_r's buffer last held dS_r(j - kSBufs): its dQ product must have
+          // read it; dP_r's buffer is free once the softmax backward has read
+          // dP_r(j-1)
+          if (kind == 0 && j >= kSBufs &&
+              !mbar_wait(&bars->dq_done[r][(j - kSBufs) & 1], (uint32_t)((j - kSBufs) >> 1) & 1u,
+                         p.dev_status, &failed))
+            break;
+          if (kind == 1 && j > 0 &&
+              !mbar_wait(&bars->ds_full[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
             break;
           tc_fence_after();
           if (kind == 0) {
@@ -197,7 +209,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 a = q_addr + r * kTile128 + (kk >> 2) * kBox128 + (kk & 3) * 32;
                 bb = kt + (kk >> 2) * kBox64 + (kk & 3) * 32;
               }
-              tc_mma_ss(tmem + colS(r), smem_desc_sw128(a, 16, 1024),
+              tc_mma_ss(tmem + colS(r, j), smem_desc_sw128(a, 16, 1024),
                         smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
             tc_commit(&bars->sd_full[r]);
@@ -228,10 +240,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tc_fence_after();
         const uint32_t kt = smem_u32(sK) + s * kTile64 + (kForm == 1 ? r * kBox64 : 0);
         for (int kk = 0; kk < 4; ++kk)  // 16 keys per step; B = K_r, MN-major
-          tc_mma_ts(tmem + colQ(r), tmem + colS(r) + kk * 8,
+          tc_mma_ts(tmem + colQ(r), tmem + colS(r, j) + kk * 8,
                     smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
                     (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&bars->dq_done[r]);
+        tc_commit(&bars->dq_done[r][j & 1]);
         tc_commit(&bars->k_empty[s]);
       }
     }
@@ -261,7 +273,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t sv[32], dp[32], pk[16];
-        tmem_ld32(tmem + lane_off + colS(r) + 32 * half, sv);
+        tmem_ld32(tmem + lane_off + colS(r, j) + 32 * half, sv);
         tmem_ld32(tmem + lane_off + colP(r) + 32 * half, dp);
         tc_wait_ld();
 #pragma unroll
@@ -285,7 +297,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                    ds0, ds1);
           pk[e] = pack_bf16(ds0, ds1);
         }
-        tmem_st16(tmem + lane_off + colS(r) + 16 * half, pk);
+        tmem_st16(tmem + lane_off + colS(r, j) + 16 * half, pk);
       }
       tc_wait_st();
       tc_fence_before();
@@ -294,7 +306,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     __syncwarp();
     if (failed) bars->abort_flag = 1;
     if (n_kv > 0)
-      mbar_wait(&bars->dq_done[r], (uint32_t)(n_kv - 1) & 1u, p.dev_status, &failed);
+      mbar_wait(&bars->dq_done[r][(n_kv - 1) & 1], (uint32_t)((n_kv - 1) >> 1) & 1u,
+                p.dev_status, &failed);
     tc_fence_after();
     const bool store = qrow < p.seqlen;
     float* dst = kForm == 1
