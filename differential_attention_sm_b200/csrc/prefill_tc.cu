@@ -8,7 +8,7 @@
 // Diferencial (V2)", section "V1 vs V2: la diferencia" (V2: paired query
 // heads on shared GQA KV heads, full head width, no per-head norm).
 //
-// One CTA computes 128 query rows of one head (V1) or one head pair (V2).
+// A query tile is 128 query rows of one head (V1) or one head pair (V2).
 // Both branches see the same K and V tiles, so each 64-key tile is loaded
 // once by TMA for the pair.  Tensor memory (512 columns x 128 lanes fp32):
 //     S1 [0,64) [64,128)   S2 [128,192) [192,256)   O1 [256,384)   O2 [384,512)
@@ -23,7 +23,8 @@
 // Warp roles (416 threads):
 //   warps 0-3  softmax for branch 1 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax for branch 2
-//   warp  8    TMA producer (Q once; K and V tiles through 4-stage rings)
+//   warp  8    TMA producer (Q per tile; K and V tiles through 4-stage rings;
+//              requests the next tile)
 //   warp  9    issues branch 1's score MMAs (Q1.K^T); owns the tensor memory
 //   warp 10    issues branch 2's score MMAs (Q2.K^T)
 //   warp 11    issues branch 1's P1.V MMAs
@@ -36,14 +37,31 @@
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
 // Causal masking is applied only on the tiles that cross the diagonal (and
-// the ragged tail).  CTAs are ordered by groups of heads whose K/V fit in L2,
-// heaviest query tiles first within a group.  Every wait is bounded; a
-// timed-out wait records DA_ERR_DEVICE_TIMEOUT in the caller's status word
-// and the CTA unwinds, still freeing its tensor memory.
+// the ragged tail).
+//
+// Scheduling.  The grid has one CTA per query tile; tiles are numbered by
+// groups of heads whose K/V fit in L2, heaviest query tiles first within a
+// group.  Only one CTA fits on an SM, and a resident CTA does not exit
+// after its tile: near the end of each tile the producer asks the hardware
+// scheduler (cluster launch control) to cancel a CTA that has not started
+// and takes over its share of the work.  Which tile a unit of work (a CTA
+// that starts, or one it cancels) computes comes from a ticket counter, so
+// the SMs pull tiles strictly in the order above, whatever order the
+// hardware starts or cancels CTAs in.  The rings, the score buffers and
+// their barrier phases run on counters that continue across tiles: the
+// next tile's Q load and first Q.K^T proceed during the current tile's
+// last P.V and epilogue, with no barrier set-up or tensor-memory
+// allocation between tiles.  The first P.V of a tile overwrites O, so it
+// waits for the previous epilogue to have read O out of tensor memory.
+// Every wait is bounded (the softmax warps exchange their normalisers
+// through mbarriers, not named barriers); a timed-out wait records
+// DA_ERR_DEVICE_TIMEOUT in the caller's status word and the CTA unwinds,
+// still freeing its tensor memory.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -68,19 +86,31 @@ constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBN, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
 
 struct Barriers {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t s_full[2][2], p_full[2][2];   // [branch][buffer]
   uint64_t o_done[2][2];                  // [branch][buffer]: P_r(j).V complete
+  uint64_t o_free;                        // the epilogue has read O out of tensor memory
+  uint64_t t_full[2], t_empty[2];         // tile numbers handed to the roles [buffer]
+  uint64_t xchg[2], nchg[2];              // softmax threads' exchanges [tile parity]
+  uint64_t clc_full;                      // response of a cancellation request
+  alignas(16) uint32_t clc_resp[4];
+  int t_id[2];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// Arrivals that release a tile-number buffer: the two score issuers, the two
+// P.V issuers and the eight softmax warps.
+constexpr uint32_t kTileReaders = 12;
 
 struct Params {
   int form;
   int batch, seqlen, heads, pairs_per_kv;
   int n_qtiles;
+  int n_tiles;      // query tiles in the grid (= CTAs launched)
+  int ticket_slot;  // tile counter of this launch (see take_ticket)
   int group;        // heads (V1) / pairs (V2) scheduled together for L2 reuse
   int causal;
   int window;       // > 0: row i sees keys (i - window, i]
@@ -103,6 +133,62 @@ __device__ __forceinline__ uint32_t s_col(int r, int buf) {
   return (r == 0 ? kColS1 : kColS2) + 64u * (uint32_t)buf;
 }
 
+// One query tile: 128 rows of one head (V1) or head pair (V2).
+struct Tile {
+  int b, hh, kvh, q0, kv0, n_kv;
+};
+
+// Tile number -> coordinates.  Tiles are numbered by groups of heads whose
+// K/V fit in L2, heaviest query tiles first within a group, and handed out
+// in that order.
+__device__ __forceinline__ Tile tile_at(const Params& p, int id, int form, bool window) {
+  const int bh_count = p.batch * p.heads;
+  const int per_group = p.group * p.n_qtiles;
+  const int g = id / per_group;
+  const int rr = id % per_group;
+  const int g_size = min(p.group, bh_count - g * p.group);
+  const int mt = p.n_qtiles - 1 - rr / g_size;
+  const int bh = g * p.group + rr % g_size;
+  Tile t;
+  t.hh = bh % p.heads;
+  t.b = bh / p.heads;
+  t.kvh = form == 1 ? t.hh : t.hh / p.pairs_per_kv;
+  t.q0 = mt * kBM;
+  const int key_end = p.causal ? min(t.q0 + kBM, p.seqlen) : p.seqlen;  // keys this tile needs
+  // Sliding window: row i sees keys (i - window, i], so the tile's first row
+  // sets the first key tile it needs.  n_kv counts the tiles processed.
+  t.kv0 = window ? max(0, t.q0 - p.window + 1) / kBN : 0;
+  t.n_kv = (key_end + kBN - 1) / kBN - t.kv0;
+  return t;
+}
+
+// Tile counters.  A launch takes one of these slots in turn, so launches
+// that run at the same time (on different streams) count on different
+// counters as long as fewer than kTicketSlots are in flight together.
+constexpr int kTicketSlots = 64;
+__device__ unsigned g_tickets[kTicketSlots];
+
+// One ticket per unit of work (a CTA that starts, or a CTA it cancels): the
+// counter runs modulo n_tiles, so a launch takes each tile number exactly
+// once and leaves the counter where it found it (zero).  A counter left
+// elsewhere by an aborted launch only rotates the next launch's order; a
+// value at or above n_tiles (left by a larger launch) wraps to zero on the
+// first ticket and is skipped.
+__device__ __forceinline__ int take_ticket(unsigned* ctr, int n_tiles) {
+  for (int i = 0; i < 4; ++i) {
+    const unsigned t = atomicInc(ctr, (unsigned)n_tiles - 1u);
+    if (t < (unsigned)n_tiles) return (int)t;
+  }
+  return -1;
+}
+
+// Tile number of this role's tile tc, published by the producer (-1: no
+// tile left, or the wait failed and *failed is set).
+__device__ __forceinline__ int read_tile(Barriers* bars, int tc, int* dev_status, bool* failed) {
+  if (!mbar_wait(&bars->t_full[tc & 1], (uint32_t)(tc >> 1) & 1u, dev_status, failed)) return -1;
+  return *(volatile int*)&bars->t_id[tc & 1];
+}
+
 // kForm: 1 = V1 (d_qk 64 per branch, one head), 2 = V2 (d 128 per branch, a head pair).
 // kWindow: sliding-window masking compiled in (p.window > 0) or out.
 // kSave: also write the training saves p.lse and p.obr.
@@ -119,32 +205,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem + qbytes;                         // kStages x kKVTile
   uint8_t* sV = sK + kStages * kKVTile;                // kStages x kKVTile
   Barriers* bars = reinterpret_cast<Barriers*>(sV + kStages * kKVTile);
-  float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [2][128]
-  float* x_ss = x_inv_l + 2 * kBM;                       // [2][128]
+  float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [tile parity][2][128]
+  float* x_ss = x_inv_l + 4 * kBM;                       // [tile parity][2][128]
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
 
-  // ---- tile coordinates: groups of heads, heaviest query tiles first ----
-  const int bh_count = p.batch * p.heads;
-  const int per_group = p.group * p.n_qtiles;
-  const int g = (int)(blockIdx.x / per_group);
-  const int rr = (int)(blockIdx.x % per_group);
-  const int g_size = min(p.group, bh_count - g * p.group);
-  const int mt = p.n_qtiles - 1 - rr / g_size;
-  const int bh = g * p.group + rr % g_size;
-  const int hh = bh % p.heads;          // V1 head or V2 pair
-  const int b = bh / p.heads;
-  const int kvh = kForm == 1 ? hh : hh / p.pairs_per_kv;
-  const int q0 = mt * kBM;
-  const int key_end = p.causal ? min(q0 + kBM, p.seqlen) : p.seqlen;  // keys this tile needs
-  // Sliding window: row i sees keys (i - window, i], so the tile's first row
-  // sets the first key tile it needs.  n_kv counts the tiles processed.
-  const int kv0 = kWindow ? max(0, q0 - p.window + 1) / kBN : 0;
-  const int n_kv = (key_end + kBN - 1) / kBN - kv0;
-
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 2);        // released by both branches' score MMAs
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 2);   // released by both branches' MMAs
@@ -158,6 +227,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars->o_done[r][u], 1);
       }
     }
+    mbar_init(&bars->o_free, 256);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bars->xchg[u], 256);
+      mbar_init(&bars->nchg[u], 256);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bars->t_full[u], 1);
+      mbar_init(&bars->t_empty[u], kTileReaders);
+    }
+    mbar_init(&bars->clc_full, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
   }
@@ -171,33 +250,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   bool failed = false;
 
+  // Every role walks the same tile sequence, one tile per unit of work (this
+  // CTA, then each CTA it cancels), as published by the producer.  Ring
+  // slots and buffer phases run on counters (tc tiles, J key tiles) that
+  // continue across tiles.
   if (warp == 8) {
     // ------------------------------ TMA producer ---------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, qbytes);
-      if (kForm == 1) {
-        tma_load_4d(sQ, &tm_q, &bars->q_full, 0, hh, q0, b);
-        tma_load_4d(sQ + kQBox, &tm_q, &bars->q_full, 64, hh, q0, b);
-      } else {
-        tma_load_4d(sQ, &tm_q, &bars->q_full, 0, 2 * hh, q0, b);
-        tma_load_4d(sQ + kQBox, &tm_q, &bars->q_full, 64, 2 * hh, q0, b);
-        tma_load_4d(sQ + 2 * kQBox, &tm_q, &bars->q_full, 0, 2 * hh + 1, q0, b);
-        tma_load_4d(sQ + 3 * kQBox, &tm_q, &bars->q_full, 64, 2 * hh + 1, q0, b);
-      }
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % kStages;
-        const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-        if (!mbar_wait(&bars->k_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
-        mbar_arrive_expect_tx(&bars->k_full[s], kKVTile);
-        tma_load_4d(sK + s * kKVTile, &tm_k, &bars->k_full[s], 0, kvh, (kv0 + j) * kBN, b);
-        tma_load_4d(sK + s * kKVTile + kKVBox, &tm_k, &bars->k_full[s], 64, kvh, (kv0 + j) * kBN, b);
-        if (!mbar_wait(&bars->v_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
-        mbar_arrive_expect_tx(&bars->v_full[s], kKVTile);
-        tma_load_4d(sV + s * kKVTile, &tm_v, &bars->v_full[s], 0, kvh, (kv0 + j) * kBN, b);
-        tma_load_4d(sV + s * kKVTile + kKVBox, &tm_v, &bars->v_full[s], 64, kvh, (kv0 + j) * kBN, b);
+      uint32_t J = 0;
+      int id = take_ticket(g_tickets + p.ticket_slot, p.n_tiles);
+      for (int tc = 0;; ++tc) {
+        // publish the tile number once every role has read the one before last
+        const uint32_t u = (uint32_t)tc >> 1;
+        if (u > 0 && !mbar_wait(&bars->t_empty[tc & 1], (u - 1) & 1u, p.dev_status, &failed))
+          break;
+        bars->t_id[tc & 1] = id;
+        mbar_arrive(&bars->t_full[tc & 1]);
+        if (id < 0) break;
+        // Q of the previous tile must be consumed by both branches' score MMAs
+        if (tc > 0 && !mbar_wait(&bars->q_empty, (uint32_t)(tc - 1) & 1u, p.dev_status, &failed))
+          break;
+        const Tile T = tile_at(p, id, kForm, kWindow);
+        mbar_arrive_expect_tx(&bars->q_full, qbytes);
+        if (kForm == 1) {
+          tma_load_4d(sQ, &tm_q, &bars->q_full, 0, T.hh, T.q0, T.b);
+          tma_load_4d(sQ + kQBox, &tm_q, &bars->q_full, 64, T.hh, T.q0, T.b);
+        } else {
+          tma_load_4d(sQ, &tm_q, &bars->q_full, 0, 2 * T.hh, T.q0, T.b);
+          tma_load_4d(sQ + kQBox, &tm_q, &bars->q_full, 64, 2 * T.hh, T.q0, T.b);
+          tma_load_4d(sQ + 2 * kQBox, &tm_q, &bars->q_full, 0, 2 * T.hh + 1, T.q0, T.b);
+          tma_load_4d(sQ + 3 * kQBox, &tm_q, &bars->q_full, 64, 2 * T.hh + 1, T.q0, T.b);
+        }
+        for (int j = 0; j < T.n_kv; ++j, ++J) {
+          const int s = J % kStages;
+          const uint32_t ph = (J / kStages) & 1u;
+          const int key = (T.kv0 + j) * kBN;
+          if (!mbar_wait(&bars->k_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
+          mbar_arrive_expect_tx(&bars->k_full[s], kKVTile);
+          tma_load_4d(sK + s * kKVTile, &tm_k, &bars->k_full[s], 0, T.kvh, key, T.b);
+          tma_load_4d(sK + s * kKVTile + kKVBox, &tm_k, &bars->k_full[s], 64, T.kvh, key, T.b);
+          if (!mbar_wait(&bars->v_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
+          mbar_arrive_expect_tx(&bars->v_full[s], kKVTile);
+          tma_load_4d(sV + s * kKVTile, &tm_v, &bars->v_full[s], 0, T.kvh, key, T.b);
+          tma_load_4d(sV + s * kKVTile + kKVBox, &tm_v, &bars->v_full[s], 64, T.kvh, key, T.b);
+        }
+        if (failed || *(volatile int*)&bars->abort_flag) break;
+        // Next unit of work: cancel a CTA that has not started, and take a
+        // ticket for it.  Once a request finds none, no request follows.
+        mbar_arrive_expect_tx(&bars->clc_full, 16);
+        clc_try_cancel(bars->clc_resp, &bars->clc_full);
+        if (!mbar_wait(&bars->clc_full, (uint32_t)tc & 1u, p.dev_status, &failed)) break;
+        id = clc_response(bars->clc_resp) >= 0 ? take_ticket(g_tickets + p.ticket_slot, p.n_tiles)
+                                                : -1;
       }
     }
   } else if (warp == 9 || warp == 10) {
@@ -207,14 +314,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const int nk = kForm == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T
-      if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
-        for (int j = 0; j < n_kv; ++j) {
-          const int s = j % kStages;
-          if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
-            break;
-          // buffer j % 2 last held P_r(j-2): its P.V must have completed
-          if (j >= 2 && !mbar_wait(&bars->o_done[r][j & 1], (uint32_t)((j - 2) >> 1) & 1u,
-                                   p.dev_status, &failed))
+      uint32_t J = 0;
+      for (int tc = 0;; ++tc) {
+        const int id = read_tile(bars, tc, p.dev_status, &failed);
+        mbar_arrive(&bars->t_empty[tc & 1]);
+        if (id < 0) break;
+        const Tile T = tile_at(p, id, kForm, kWindow);
+        if (!mbar_wait(&bars->q_full, (uint32_t)tc & 1u, p.dev_status, &failed)) break;
+        for (int j = 0; j < T.n_kv; ++j, ++J) {
+          const int s = J % kStages;
+          if (!mbar_wait(&bars->k_full[s], (J / kStages) & 1u, p.dev_status, &failed)) break;
+          // buffer J % 2 last held P_r(J-2): its P.V must have completed
+          if (J >= 2 && !mbar_wait(&bars->o_done[r][J & 1], ((J - 2) >> 1) & 1u, p.dev_status,
+                                   &failed))
             break;
           tc_fence_after();
           const uint32_t kt = k_addr + s * kKVTile;
@@ -227,12 +339,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
               bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
             }
-            tc_mma_ss(tmem + s_col(r, j & 1), smem_desc_sw128(a, 16, 1024),
+            tc_mma_ss(tmem + s_col(r, J & 1), smem_desc_sw128(a, 16, 1024),
                       smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
           }
-          tc_commit(&bars->s_full[r][j & 1]);
+          tc_commit(&bars->s_full[r][J & 1]);
           tc_commit(&bars->k_empty[s]);
         }
+        if (failed) break;
+        tc_commit(&bars->q_empty);  // Q free once this branch's score MMAs are done
       }
     }
   } else if (warp == 11 || warp == 12) {
@@ -242,23 +356,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t v_addr = smem_u32(sV);
       const uint32_t pcol0 = tmem + s_col(r, 0);
       const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(&bars->v_full[s], (uint32_t)(j / kStages) & 1u, p.dev_status, &failed))
-          break;
-        if (!mbar_wait(&bars->p_full[r][j & 1], (uint32_t)(j >> 1) & 1u, p.dev_status,
-                       &failed))
-          break;
-        tc_fence_after();
-        const uint32_t vt = v_addr + s * kKVTile;
-        const uint32_t pcol = pcol0 + 64u * (uint32_t)(j & 1);
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
-          tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
-                    kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+      uint32_t J = 0;
+      for (int tc = 0;; ++tc) {
+        const int id = read_tile(bars, tc, p.dev_status, &failed);
+        mbar_arrive(&bars->t_empty[tc & 1]);
+        if (id < 0) break;
+        const Tile T = tile_at(p, id, kForm, kWindow);
+        for (int j = 0; j < T.n_kv; ++j, ++J) {
+          const int s = J % kStages;
+          if (!mbar_wait(&bars->v_full[s], (J / kStages) & 1u, p.dev_status, &failed)) break;
+          if (!mbar_wait(&bars->p_full[r][J & 1], (J >> 1) & 1u, p.dev_status, &failed)) break;
+          // the first P.V of a tile overwrites O: the previous tile's
+          // epilogue must have read it out
+          if (j == 0 && tc > 0 &&
+              !mbar_wait(&bars->o_free, (uint32_t)(tc - 1) & 1u, p.dev_status, &failed))
+            break;
+          tc_fence_after();
+          const uint32_t vt = v_addr + s * kKVTile;
+          const uint32_t pcol = pcol0 + 64u * (J & 1u);
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
+            tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
+                      kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&bars->o_done[r][J & 1]);
+          tc_commit(&bars->v_empty[s]);
         }
-        tc_commit(&bars->o_done[r][j & 1]);
-        tc_commit(&bars->v_empty[s]);
+        if (failed) break;
       }
     }
   } else {
@@ -266,199 +390,218 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = warp / 4;                  // branch
     const int sub = warp & 3;                // TMEM lane quarter
     const int row = sub * 32 + lane;         // query row within the tile
-    const int qrow = q0 + row;               // query row within the sequence
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
     const uint32_t t_o = tmem + lane_off + (r == 0 ? kColO1 : kColO2);
-    const int lim = p.causal ? min(qrow + 1, p.seqlen) : p.seqlen;  // keys < lim visible
-    const int lo = kWindow ? max(0, qrow - p.window + 1) : 0;         // and keys >= lo
     const float sc = p.scale_log2;
-    float m_ref = -INFINITY, l_run = 0.f;
+    uint32_t J = 0;
+    for (int tc = 0;; ++tc) {
+      // tensor-memory accesses below are warp-collective: the tile decision
+      // is taken by the whole warp
+      int id = read_tile(bars, tc, p.dev_status, &failed);
+      id = __shfl_sync(0xffffffffu, __all_sync(0xffffffffu, !failed) ? id : -1, 0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->t_empty[tc & 1]);
+      if (id < 0) break;
+      const Tile T = tile_at(p, id, kForm, kWindow);
+      const int qrow = T.q0 + row;             // query row within the sequence
+      const int lim = p.causal ? min(qrow + 1, p.seqlen) : p.seqlen;  // keys < lim visible
+      const int lo = kWindow ? max(0, qrow - p.window + 1) : 0;         // and keys >= lo
+      float m_ref = -INFINITY, l_run = 0.f;
 
-    for (int j = 0; j < n_kv; ++j) {
-      const int buf = j & 1;
-      // Tensor-memory loads and stores below are warp-collective, so a failed
-      // wait in any lane ends the loop for the whole warp.
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(&bars->s_full[r][buf], (uint32_t)(j >> 1) & 1u, p.dev_status,
-                                &failed))) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t t_s = tmem + lane_off + s_col(r, buf);
-      uint32_t sr[64];  // raw S row of this tile (masked entries set to -inf)
-      tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
-      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-      tc_wait_ld();
-      const int k0 = (kv0 + j) * kBN;
-      if (k0 + kBN > lim) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
-      }
-      if (kWindow && k0 < lo) {  // window start (a row may see none of this tile)
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (k0 + c < lo) sr[c] = __float_as_uint(-INFINITY);
-      }
-      // row maximum: 3-input max over 8 independent chains
-      float m8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float m = max3(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]),
-                       __uint_as_float(sr[16 + i]));
-        m = max3(m, __uint_as_float(sr[24 + i]), __uint_as_float(sr[32 + i]));
-        m = max3(m, __uint_as_float(sr[40 + i]), __uint_as_float(sr[48 + i]));
-        m8[i] = fmaxf(m, __uint_as_float(sr[56 + i]));
-      }
-      const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
-                            fmaxf(m8[6], m8[7])) * sc;  // sc > 0 commutes with max
-      float alpha = 1.f;
-      bool resc = false;
-      if (j == 0) {
-        m_ref = mx;
-      } else {
-        const float m_new = fmaxf(m_ref, mx);
-        resc = m_new > m_ref + kLazyTau;
-        if (resc) {
-          alpha = ex2(m_ref - m_new);
-          m_ref = m_new;
-        }
-      }
-      const float u = m_ref == -INFINITY ? 0.f : m_ref;
-      // p = 2^(s*sc - u): pairs on the f32x2 pipe; one pair in four takes the
-      // polynomial 2^x, the rest the multi-function unit.
-      const uint64_t sc2 = f2pack(sc, sc), nu2 = f2pack(-u, -u);
-      uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int qt = 0; qt < 2; ++qt) {  // 32 logits -> 16 packed bf16 pairs per store
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = qt * 32 + 2 * e;
-          const uint64_t x2 = fma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
-                                   sc2, nu2);
-          float x0, x1, p0, p1;
-          f2unpack(x2, x0, x1);
-          // Share of exponentials on the polynomial: V1's shorter Q.K^T leaves
-          // the softmax the critical path, so it offloads more (measured).
-          if (kForm == 1 ? (e & 3) == 3 : (e & 7) == 7) {
-            exp2_poly2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          ps2[e & 3] = add2(ps2[e & 3], f2pack(p0, p1));
-          pk[e] = pack_bf16(p0, p1);
-        }
-        tmem_st16(t_s + 16 * qt, pk);
-      }
-      float psum, psum_hi;
-      f2unpack(add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3])), psum, psum_hi);
-      psum += psum_hi;
-      if (__any_sync(0xffffffffu, resc)) {
-        // O_r must be quiescent (the previous tile's P.V into O_r done) before
-        // it is rescaled in place; rows that keep their reference use alpha 1.
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[r][(j - 1) & 1],
-                                                (uint32_t)((j - 1) >> 1) & 1u, p.dev_status,
-                                                &failed))) {
+      for (int j = 0; j < T.n_kv; ++j, ++J) {
+        const int buf = J & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[r][buf], (J >> 1) & 1u,
+                                                p.dev_status, &failed))) {
           failed = true;
           break;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t ov[16];
-          tmem_ld16(t_o + 16 * c, ov);
-          tc_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st16(t_o + 16 * c, ov);
-        }
-      }
-      l_run = l_run * alpha + psum;
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[r][buf]);
-    }
-
-    // ---- epilogue: o = O1/l1 - lambda O2/l2 (+ V1 norm), channels [64 r, 64 r + 64) ----
-    __syncwarp();
-    if (failed) bars->abort_flag = 1;
-    // own branch's last P.V done; the named barrier then orders both branches
-    mbar_wait(&bars->o_done[r][(n_kv - 1) & 1], (uint32_t)((n_kv - 1) >> 1) & 1u, p.dev_status,
-              &failed);
-    tc_fence_after();
-    x_inv_l[r * kBM + row] = 1.0f / l_run;
-    if (kSave && qrow < p.seqlen)  // p_ij = 2^(s_ij * sc - lse) for the backward
-      p.lse[(((size_t)b * p.heads + hh) * 2 + r) * p.lse_stride + qrow] =
-          (m_ref == -INFINITY ? 0.f : m_ref) + log2f(l_run);
-    asm volatile("bar.sync 2, 256;" ::: "memory");
-    tc_fence_after();
-    const float inv1 = x_inv_l[row];
-    const float inv2_raw = x_inv_l[kBM + row];
-    const float inv2 = inv2_raw * p.lambda[hh];
-    float o[64];
-    {
-      uint32_t a[32], c2[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(tmem + lane_off + kColO1 + 64 * r + 32 * half, a);
-        tmem_ld32(tmem + lane_off + kColO2 + 64 * r + 32 * half, c2);
+        const uint32_t t_s = tmem + lane_off + s_col(r, buf);
+        uint32_t sr[64];  // raw S row of this tile (masked entries set to -inf)
+        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
         tc_wait_ld();
+        const int k0 = (T.kv0 + j) * kBN;
+        if (k0 + kBN > lim) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          o[half * 32 + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
-        if (kSave && qrow < p.seqlen) {
-          __nv_bfloat16* ob = p.obr + (((size_t)b * p.seqlen + qrow) * p.heads + hh) * 256 +
-                              64 * r + 32 * half;
+          for (int c = 0; c < 64; ++c)
+            if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        if (kWindow && k0 < lo) {  // window start (a row may see none of this tile)
 #pragma unroll
-          for (int v8 = 0; v8 < 4; ++v8) {
-            uint4 w1, w2;
-            w1.x = pack_bf16(__uint_as_float(a[8 * v8 + 0]) * inv1, __uint_as_float(a[8 * v8 + 1]) * inv1);
-            w1.y = pack_bf16(__uint_as_float(a[8 * v8 + 2]) * inv1, __uint_as_float(a[8 * v8 + 3]) * inv1);
-            w1.z = pack_bf16(__uint_as_float(a[8 * v8 + 4]) * inv1, __uint_as_float(a[8 * v8 + 5]) * inv1);
-            w1.w = pack_bf16(__uint_as_float(a[8 * v8 + 6]) * inv1, __uint_as_float(a[8 * v8 + 7]) * inv1);
-            w2.x = pack_bf16(__uint_as_float(c2[8 * v8 + 0]) * inv2_raw, __uint_as_float(c2[8 * v8 + 1]) * inv2_raw);
-            w2.y = pack_bf16(__uint_as_float(c2[8 * v8 + 2]) * inv2_raw, __uint_as_float(c2[8 * v8 + 3]) * inv2_raw);
-            w2.z = pack_bf16(__uint_as_float(c2[8 * v8 + 4]) * inv2_raw, __uint_as_float(c2[8 * v8 + 5]) * inv2_raw);
-            w2.w = pack_bf16(__uint_as_float(c2[8 * v8 + 6]) * inv2_raw, __uint_as_float(c2[8 * v8 + 7]) * inv2_raw);
-            *reinterpret_cast<uint4*>(ob + 8 * v8) = w1;
-            *reinterpret_cast<uint4*>(ob + 128 + 8 * v8) = w2;
+          for (int c = 0; c < 64; ++c)
+            if (k0 + c < lo) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // row maximum: 3-input max over 8 independent chains
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float m = max3(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]),
+                         __uint_as_float(sr[16 + i]));
+          m = max3(m, __uint_as_float(sr[24 + i]), __uint_as_float(sr[32 + i]));
+          m = max3(m, __uint_as_float(sr[40 + i]), __uint_as_float(sr[48 + i]));
+          m8[i] = fmaxf(m, __uint_as_float(sr[56 + i]));
+        }
+        const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
+                              fmaxf(m8[6], m8[7])) * sc;  // sc > 0 commutes with max
+        float alpha = 1.f;
+        bool resc = false;
+        if (j == 0) {
+          m_ref = mx;
+        } else {
+          const float m_new = fmaxf(m_ref, mx);
+          resc = m_new > m_ref + kLazyTau;
+          if (resc) {
+            alpha = ex2(m_ref - m_new);
+            m_ref = m_new;
+          }
+        }
+        const float u = m_ref == -INFINITY ? 0.f : m_ref;
+        // p = 2^(s*sc - u): pairs on the f32x2 pipe; one pair in four takes the
+        // polynomial 2^x, the rest the multi-function unit.
+        const uint64_t sc2 = f2pack(sc, sc), nu2 = f2pack(-u, -u);
+        uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int qt = 0; qt < 2; ++qt) {  // 32 logits -> 16 packed bf16 pairs per store
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = qt * 32 + 2 * e;
+            const uint64_t x2 = fma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                     sc2, nu2);
+            float x0, x1, p0, p1;
+            f2unpack(x2, x0, x1);
+            // Share of exponentials on the polynomial: V1's shorter Q.K^T leaves
+            // the softmax the critical path, so it offloads more (measured).
+            if (kForm == 1 ? (e & 3) == 3 : (e & 7) == 7) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            ps2[e & 3] = add2(ps2[e & 3], f2pack(p0, p1));
+            pk[e] = pack_bf16(p0, p1);
+          }
+          tmem_st16(t_s + 16 * qt, pk);
+        }
+        float psum, psum_hi;
+        f2unpack(add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3])), psum, psum_hi);
+        psum += psum_hi;
+        if (__any_sync(0xffffffffu, resc)) {
+          // O_r must be quiescent (the previous tile's P.V into O_r done) before
+          // it is rescaled in place; rows that keep their reference use alpha 1.
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[r][(J - 1) & 1],
+                                                  ((J - 1) >> 1) & 1u, p.dev_status,
+                                                  &failed))) {
+            failed = true;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t ov[16];
+            tmem_ld16(t_o + 16 * c, ov);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st16(t_o + 16 * c, ov);
+          }
+        }
+        l_run = l_run * alpha + psum;
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[r][buf]);
+      }
+
+      // ---- epilogue: o = O1/l1 - lambda O2/l2 (+ V1 norm), channels [64 r, 64 r + 64) ----
+      __syncwarp();
+      if (failed) bars->abort_flag = 1;
+      // own branch's last P.V done; the named barrier then orders both branches
+      const uint32_t Jl = J - 1;
+      mbar_wait(&bars->o_done[r][Jl & 1], (Jl >> 1) & 1u, p.dev_status, &failed);
+      tc_fence_after();
+      float* inv_l = x_inv_l + (tc & 1) * 2 * kBM;
+      inv_l[r * kBM + row] = 1.0f / l_run;
+      if (kSave && qrow < p.seqlen)  // p_ij = 2^(s_ij * sc - lse) for the backward
+        p.lse[(((size_t)T.b * p.heads + T.hh) * 2 + r) * p.lse_stride + qrow] =
+            (m_ref == -INFINITY ? 0.f : m_ref) + log2f(l_run);
+      // both branches' normalisers (bounded wait, unlike a named barrier)
+      mbar_arrive(&bars->xchg[tc & 1]);
+      mbar_wait(&bars->xchg[tc & 1], (uint32_t)(tc >> 1) & 1u, p.dev_status, &failed);
+      const bool stop = *(volatile int*)&bars->abort_flag != 0;
+      tc_fence_after();
+      const float inv1 = inv_l[row];
+      const float inv2_raw = inv_l[kBM + row];
+      const float inv2 = inv2_raw * p.lambda[T.hh];
+      float o[64];
+      {
+        uint32_t a[32], c2[32];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          tmem_ld32(tmem + lane_off + kColO1 + 64 * r + 32 * half, a);
+          tmem_ld32(tmem + lane_off + kColO2 + 64 * r + 32 * half, c2);
+          tc_wait_ld();
+          if (half == 1) {  // O fully read: the next tile's first P.V may overwrite it
+            tc_fence_before();
+            mbar_arrive(&bars->o_free);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            o[half * 32 + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
+          if (kSave && qrow < p.seqlen) {
+            __nv_bfloat16* ob = p.obr + (((size_t)T.b * p.seqlen + qrow) * p.heads + T.hh) * 256 +
+                                64 * r + 32 * half;
+#pragma unroll
+            for (int v8 = 0; v8 < 4; ++v8) {
+              uint4 w1, w2;
+              w1.x = pack_bf16(__uint_as_float(a[8 * v8 + 0]) * inv1, __uint_as_float(a[8 * v8 + 1]) * inv1);
+              w1.y = pack_bf16(__uint_as_float(a[8 * v8 + 2]) * inv1, __uint_as_float(a[8 * v8 + 3]) * inv1);
+              w1.z = pack_bf16(__uint_as_float(a[8 * v8 + 4]) * inv1, __uint_as_float(a[8 * v8 + 5]) * inv1);
+              w1.w = pack_bf16(__uint_as_float(a[8 * v8 + 6]) * inv1, __uint_as_float(a[8 * v8 + 7]) * inv1);
+              w2.x = pack_bf16(__uint_as_float(c2[8 * v8 + 0]) * inv2_raw, __uint_as_float(c2[8 * v8 + 1]) * inv2_raw);
+              w2.y = pack_bf16(__uint_as_float(c2[8 * v8 + 2]) * inv2_raw, __uint_as_float(c2[8 * v8 + 3]) * inv2_raw);
+              w2.z = pack_bf16(__uint_as_float(c2[8 * v8 + 4]) * inv2_raw, __uint_as_float(c2[8 * v8 + 5]) * inv2_raw);
+              w2.w = pack_bf16(__uint_as_float(c2[8 * v8 + 6]) * inv2_raw, __uint_as_float(c2[8 * v8 + 7]) * inv2_raw);
+              *reinterpret_cast<uint4*>(ob + 8 * v8) = w1;
+              *reinterpret_cast<uint4*>(ob + 128 + 8 * v8) = w2;
+            }
           }
         }
       }
-    }
-    float mul = 1.f;
-    if (p.apply_norm) {
-      float ss4[4] = {0.f, 0.f, 0.f, 0.f};
+      float mul = 1.f;
+      if (p.apply_norm) {
+        float* ssq = x_ss + (tc & 1) * 2 * kBM;
+        float ss4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < 64; ++e) ss4[e & 3] = fmaf(o[e], o[e], ss4[e & 3]);
-      x_ss[r * kBM + row] = (ss4[0] + ss4[1]) + (ss4[2] + ss4[3]);
-      asm volatile("bar.sync 2, 256;" ::: "memory");
-      const float tot = x_ss[row] + x_ss[kBM + row];
-      mul = p.post_scale / sqrtf(tot * (1.0f / 128.0f) + p.eps);
-    }
-    if (qrow < p.seqlen && !bars->abort_flag) {
-      __nv_bfloat16* dst =
-          p.out + (((size_t)b * p.seqlen + qrow) * p.heads + hh) * 128 + 64 * r;
-#pragma unroll
-      for (int v8 = 0; v8 < 8; ++v8) {
-        float y[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = v8 * 8 + e;
-          const float gm = (p.apply_norm && p.norm_weight) ? __ldg(p.norm_weight + 64 * r + c)
-                                                           : 1.f;
-          y[e] = o[c] * mul * gm;
-        }
-        uint4 w;
-        w.x = pack_bf16(y[0], y[1]);
-        w.y = pack_bf16(y[2], y[3]);
-        w.z = pack_bf16(y[4], y[5]);
-        w.w = pack_bf16(y[6], y[7]);
-        *reinterpret_cast<uint4*>(dst + v8 * 8) = w;
+        for (int e = 0; e < 64; ++e) ss4[e & 3] = fmaf(o[e], o[e], ss4[e & 3]);
+        ssq[r * kBM + row] = (ss4[0] + ss4[1]) + (ss4[2] + ss4[3]);
+        mbar_arrive(&bars->nchg[tc & 1]);
+        mbar_wait(&bars->nchg[tc & 1], (uint32_t)(tc >> 1) & 1u, p.dev_status, &failed);
+        const float tot = ssq[row] + ssq[kBM + row];
+        mul = p.post_scale / sqrtf(tot * (1.0f / 128.0f) + p.eps);
       }
+      if (qrow < p.seqlen && !stop && !failed) {
+        __nv_bfloat16* dst =
+            p.out + (((size_t)T.b * p.seqlen + qrow) * p.heads + T.hh) * 128 + 64 * r;
+#pragma unroll
+        for (int v8 = 0; v8 < 8; ++v8) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = v8 * 8 + e;
+            const float gm = (p.apply_norm && p.norm_weight) ? __ldg(p.norm_weight + 64 * r + c)
+                                                             : 1.f;
+            y[e] = o[c] * mul * gm;
+          }
+          uint4 w;
+          w.x = pack_bf16(y[0], y[1]);
+          w.y = pack_bf16(y[2], y[3]);
+          w.z = pack_bf16(y[4], y[5]);
+          w.w = pack_bf16(y[6], y[7]);
+          *reinterpret_cast<uint4*>(dst + v8 * 8) = w;
+        }
+      }
+      if (__any_sync(0xffffffffu, failed) || stop) break;
     }
   }
 
@@ -471,7 +614,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
 }
-
 }  // namespace
 
 cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
@@ -485,6 +627,8 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.heads = a.heads;
   p.pairs_per_kv = a.pairs_per_kv;
   p.n_qtiles = (a.seqlen + kBM - 1) / kBM;
+  static std::atomic<unsigned> next_slot{0};
+  p.ticket_slot = (int)(next_slot.fetch_add(1u, std::memory_order_relaxed) % kTicketSlots);
   // Heads (V1) or pairs (V2) scheduled together: as many as keep their K and
   // V (2 x seqlen x 128 bf16 per KV head) within about half of the L2.
   const double kv_bytes = 2.0 * a.seqlen * 128 * 2;
@@ -508,7 +652,7 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.dev_status = a.dev_status;
   const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
   const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +
-                   4 * kBM * (int)sizeof(float) + 64;
+                   8 * kBM * (int)sizeof(float) + 64;
   const bool win = a.window > 0;
   decltype(&diffattn_prefill_tc_kernel<1, false, false>) kern;
   if (a.lse && a.obr)  // training forward
@@ -526,6 +670,7 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   if (e != cudaSuccess) return e;
   const long long grid = (long long)p.n_qtiles * bh_count;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  p.n_tiles = (int)grid;
   kern<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
   return cudaGetLastError();
 }

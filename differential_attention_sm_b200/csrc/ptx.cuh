@@ -187,6 +187,40 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* d
 }
 
 // ---------------------------------------------------------------------------
+// Cluster launch control (sm_100): a running CTA asks the hardware scheduler
+// to cancel one CTA of the same grid that has not started yet and takes over
+// its work.  The 16-byte response is written to shared memory and completes
+// 16 transaction bytes on the mbarrier.  Once a response has reported "not
+// cancelled" (the grid has no CTA left to start), no further request may be
+// issued.  Plain form only (no cluster-wide broadcast of the response).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+      " [%0], [%1];" ::"r"(smem_u32(resp)),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Reads a response: the cancelled CTA's blockIdx.x, or -1 if none was
+// cancelled.  The fence orders this generic-proxy read before the next
+// asynchronous write of the same buffer.
+__device__ __forceinline__ int clc_response(const void* resp) {
+  uint32_t x = 0, ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %1, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%0, _, _, _}, r;\n\t}"
+      : "+r"(x), "=r"(ok)
+      : "r"(smem_u32(resp))
+      : "memory");
+  fence_proxy_async_smem();
+  return ok ? (int)x : -1;
+}
+
+// ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {

@@ -26,8 +26,17 @@
  *    asynchronous copies bound every wait; if one ever times out the kernel
  *    stores DA_ERR_DEVICE_TIMEOUT there (first error wins; the caller zeroes
  *    it beforehand) and returns early, leaving the output undefined.
- *  - Thread safety: no mutable global state; concurrent calls on different
- *    streams are independent.
+ *  - Thread safety: concurrent calls on different streams are independent,
+ *    with two exceptions: diffattn_v2_decode_noalloc's shared scratch array
+ *    (see that entry point) and the prefill's tile counters (next).  Global
+ *    state: a per-device cuBLAS handle for the backward and the output
+ *    projection, created under a lock on first use, and, for the bf16
+ *    tensor-core prefill (diffattn_v1_fwd / diffattn_v2_prefill and their
+ *    window, training and projection variants), 64 tile counters per device
+ *    in a statically allocated array.  Each such launch takes the next
+ *    counter in turn and leaves it at zero when it completes, so at most 64
+ *    of them may execute on one device at the same time (on several streams,
+ *    or as replays of CUDA graphs).
  */
 #ifndef DIFFATTN_H_
 #define DIFFATTN_H_
