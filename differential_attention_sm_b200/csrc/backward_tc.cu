@@ -18,7 +18,8 @@
 //     (V2), walking 64-key tiles like the forward: per branch, S_r and dP_r
 //     into tensor memory (two SS MMAs), dS_r written back over S_r as bf16
 //     by the softmax-backward warps, then dQ_r += dS_r K_r (TS MMA) in
-//     tensor memory.  Warps: 0-3 / 4-7 branch 1 / 2 (thread = query row),
+//     tensor memory.  The softmax-backward warps form P as soon as S_r has
+//     landed and wait for dP_r only after that.  Warps: 0-3 / 4-7 branch 1 / 2 (thread = query row),
 //     8 TMA producer, 9-12 the S_r and dP_r issuers (one thread per product
 //     stream, as in the forward), 13 / 14 dQ issuers.
 //   * dkdv kernel, one CTA per 128 keys of a head (V1) or KV head (V2),
@@ -26,7 +27,10 @@
 //     head): S^T = K_r Q_r^T and dP^T = V do_r^T (SS), P^T and dS^T written
 //     back as bf16 by the softmax-backward warps (thread = key row), then
 //     dV += P^T do_r and dK_r += dS^T Q_r (TS) in tensor memory.  Each
-//     accumulator has one issuing thread, so its order is fixed.
+//     accumulator has one issuing thread, so its order is fixed.  The two
+//     halves of each step's handshake are separate: P^T is written (and the
+//     dV product released) as soon as S^T lands, dS^T once dP^T has; the
+//     next S^T into a buffer waits only for dV, the next dP^T only for dK.
 //     Warps: 0-3 / 4-7 alternate steps (= branches), 8 producer,
 //     9 S^T issuer, 10 dP^T issuer, 11 dV issuer, 12 dK issuer.
 // Every wait is bounded (DA_ERR_DEVICE_TIMEOUT in the status word).
@@ -72,7 +76,9 @@ struct DqBarriers {
   uint64_t q_full;
   uint64_t k_full[kDqStages], k_empty[kDqStages];
   uint64_t v_full[kDqStages], v_empty[kDqStages];
-  uint64_t sd_full[2], ds_full[2];
+  uint64_t s_full[2][2];   // [branch][S buffer]: S_r landed
+  uint64_t dp_full[2];     // [branch]: dP_r landed
+  uint64_t ds_full[2];     // [branch]: dS_r written back (and dP_r read)
   uint64_t dq_done[2][2];  // [branch][S buffer]: the dQ product of a tile has read its dS
   uint32_t tmem_base;
   int abort_flag;
@@ -114,7 +120,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       mbar_init(&bars->v_empty[s], 2);
     }
     for (int r = 0; r < 2; ++r) {
-      mbar_init(&bars->sd_full[r], 2);  // S_r and dP_r, from their own issuers
+      mbar_init(&bars->s_full[r][0], 1);
+      mbar_init(&bars->s_full[r][1], 1);
+      mbar_init(&bars->dp_full[r], 1);
       mbar_init(&bars->ds_full[r], 128);
       mbar_init(&bars->dq_done[r][0], 1);
       mbar_init(&bars->dq_done[r][1], 1);
@@ -212,7 +220,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
               tc_mma_ss(tmem + colS(r, j), smem_desc_sw128(a, 16, 1024),
                         smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
-            tc_commit(&bars->sd_full[r]);
+            tc_commit(&bars->s_full[r][j % kSBufs]);
             tc_commit(&bars->k_empty[s]);
           } else {
             const uint32_t vt = smem_u32(sV) + s * kTile64;
@@ -222,7 +230,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
               tc_mma_ss(tmem + colP(r), smem_desc_sw128(a, 16, 1024),
                         smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
-            tc_commit(&bars->sd_full[r]);
+            tc_commit(&bars->dp_full[r]);
             tc_commit(&bars->v_empty[s]);
           }
         }
@@ -260,8 +268,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const float Dr = qrow < p.seqlen ? p.Dv[vrow] : 0.f;
     const float sc = p.scale_log2;
     const uint64_t sc2 = f2pack(sc, sc), nl2 = f2pack(-lse, -lse), nd2 = f2pack(-Dr, -Dr);
+    // Two passes per tile: P = 2^(s sc - lse) as soon as S_r has landed (the
+    // dP_r product may still be in flight), then dS = P (dP - D) from the same
+    // P, kept in registers as bf16 pairs, written back over S_r.
     for (int j = 0; j < n_kv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->sd_full[r], (uint32_t)j & 1u, p.dev_status,
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[r][j % kSBufs],
+                                             (uint32_t)(j / kSBufs) & 1u, p.dev_status,
                                              &failed))) {
         failed = true;
         break;
@@ -270,15 +282,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       const int k0 = (kv0 + j) * 64;
       // tiles fully inside every row's visible range skip the masks
       const bool full = __all_sync(0xffffffffu, k0 + 64 <= lim && (!kWindow || k0 >= lo));
+      uint32_t pp[32];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        uint32_t sv[32], dp[32], pk[16];
+        uint32_t sv[32];
         tmem_ld32(tmem + lane_off + colS(r, j) + 32 * half, sv);
-        tmem_ld32(tmem + lane_off + colP(r) + 32 * half, dp);
         tc_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          // p = 2^(s sc - lse), ds = p (dP - D): packed pairs
           float x0, x1;
           f2unpack(fma2(f2pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
                         sc2, nl2),
@@ -289,8 +300,25 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             p0 = (key < lim && (!kWindow || key >= lo)) ? p0 : 0.f;
             p1 = (key + 1 < lim && (!kWindow || key + 1 >= lo)) ? p1 : 0.f;
           }
+          pp[16 * half + e] = pack_bf16(p0, p1);
+        }
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full[r], (uint32_t)j & 1u, p.dev_status,
+                                             &failed))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dp[32], pk[16];
+        tmem_ld32(tmem + lane_off + colP(r) + 32 * half, dp);
+        tc_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const uint32_t pb = pp[16 * half + e];
           float ds0, ds1;
-          f2unpack(fma2(f2pack(p0, p1),
+          f2unpack(fma2(f2pack(bf16lo(pb), bf16hi(pb)),
                         add2(f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
                              nd2),
                         0ull),
@@ -352,7 +380,9 @@ static_assert(kStageBytes % 1024 == 0, "stage alignment");
 struct KvBarriers {
   uint64_t kv_full;
   uint64_t qd_full[kKvStages], qd_empty[kKvStages];
-  uint64_t sd_full[2], ps_full[2], pt_free[2], dst_free[2];
+  uint64_t s_full[2], dp_full[2];        // S^T, dP^T landed [buffer]
+  uint64_t p_full[2], ds_full[2];        // P^T, dS^T written back [buffer]
+  uint64_t pt_free[2], dst_free[2];      // dV, dK products done with them [buffer]
   uint64_t acc_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -393,8 +423,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       mbar_init(&bars->qd_empty[s], 4);  // all four products read Q_r or dO_r
     }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&bars->sd_full[w], 2);  // S^T and dP^T, from their own issuers
-      mbar_init(&bars->ps_full[w], 128);
+      mbar_init(&bars->s_full[w], 1);
+      mbar_init(&bars->dp_full[w], 1);
+      mbar_init(&bars->p_full[w], 128);
+      mbar_init(&bars->ds_full[w], 128);
       mbar_init(&bars->pt_free[w], 1);
       mbar_init(&bars->dst_free[w], 1);
     }
@@ -491,7 +523,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                         smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
           }
-          tc_commit(&bars->sd_full[w]);
+          tc_commit(is_s ? &bars->s_full[w] : &bars->dp_full[w]);
           tc_commit(&bars->qd_empty[st]);
         }
       }
@@ -505,7 +537,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       bool first[2] = {true, true};
       for (int s = 0; s < n_steps; ++s) {
         const int st = s % kKvStages, w = s & 1, r = s & 1;
-        if (!mbar_wait(&bars->ps_full[w], (uint32_t)(s >> 1) & 1u, p.dev_status, &failed))
+        if (!mbar_wait(is_v ? &bars->p_full[w] : &bars->ds_full[w], (uint32_t)(s >> 1) & 1u,
+                       p.dev_status, &failed))
           break;
         tc_fence_after();
         const uint32_t sq = smem_u32(sStage) + st * kStageBytes, sdo = sq + kStageQ;
@@ -527,17 +560,22 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
   } else {
     // --------------------------------- softmax backward, steps of parity w
+    // Two passes per step.  P = 2^(s sc - lse) goes out as soon as S^T has
+    // landed, so the dV product starts (and frees the S^T buffer for step
+    // s + 2) while dP^T may still be in flight; dS = P (dP - D) follows from
+    // the same bf16 P, kept in registers.
     const int w = warp / 4;
     const int krow = (warp & 3) * 32 + lane;
     const int key = k0 + krow;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + 128 * w, t_dp = t_s + 64;
     const float sc = p.scale_log2;
     for (int s = w; s < n_steps; s += 2) {
       const int st = s % kKvStages;
+      const uint32_t ph = (uint32_t)(s >> 1) & 1u;
       const bool ok = mbar_wait(&bars->qd_full[st], (uint32_t)(s / kKvStages) & 1u,
                                 p.dev_status, &failed) &&
-                      mbar_wait(&bars->sd_full[w], (uint32_t)(s >> 1) & 1u, p.dev_status,
-                                &failed);
+                      mbar_wait(&bars->s_full[w], ph, p.dev_status, &failed);
       if (!__all_sync(0xffffffffu, ok)) {
         failed = true;
         break;
@@ -553,23 +591,20 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       if (kWindow) c_hi = min(c_hi, key + p.window - q0);
       const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == 64);
       const uint64_t sc2 = f2pack(sc, sc);
+      uint32_t pp[32];  // P row as packed bf16 pairs
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        uint32_t sv[32], dp[32], pp[16], pd[16];
-        tmem_ld32(tmem + lane_off + 128 * w + 32 * half, sv);
-        tmem_ld32(tmem + lane_off + 128 * w + 64 + 32 * half, dp);
+        uint32_t sv[32];
+        tmem_ld32(t_s + 32 * half, sv);
         tc_wait_ld();
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {  // 4 query columns: lse and D by broadcast loads
+        for (int e4 = 0; e4 < 8; ++e4) {  // 4 query columns: lse by a broadcast load
           const int c = 32 * half + 4 * e4;
           const float4 L = *reinterpret_cast<const float4*>(svec + c);
-          const float4 Dd = *reinterpret_cast<const float4*>(svec + 64 + c);
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int e = 2 * e4 + h2;
             const float l0 = h2 ? L.z : L.x, l1 = h2 ? L.w : L.y;
-            const float d0 = h2 ? Dd.z : Dd.x, d1 = h2 ? Dd.w : Dd.y;
-            // p = 2^(s sc - lse), ds = p (dP - D): packed pairs
             float x0, x1;
             f2unpack(fma2(f2pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
                           sc2, f2pack(-l0, -l1)),
@@ -580,22 +615,49 @@ __global__ void __launch_bounds__(kKvThreads, 1)
               p0 = (cc >= c_lo && cc < c_hi) ? p0 : 0.f;
               p1 = (cc + 1 >= c_lo && cc + 1 < c_hi) ? p1 : 0.f;
             }
-            const uint64_t pr = f2pack(p0, p1);
+            pp[16 * half + e] = pack_bf16(p0, p1);
+          }
+        }
+        // P^T over the first 32 columns of S^T (this half's S is already read)
+        tmem_st16(t_s + 16 * half, *reinterpret_cast<uint32_t(*)[16]>(pp + 16 * half));
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[w]);
+
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full[w], ph, p.dev_status, &failed))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dp[32], pd[16];
+        tmem_ld32(t_dp + 32 * half, dp);
+        tc_wait_ld();
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {  // D by a broadcast load
+          const int c = 32 * half + 4 * e4;
+          const float4 Dd = *reinterpret_cast<const float4*>(svec + 64 + c);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e4 + h2;
+            const float d0 = h2 ? Dd.z : Dd.x, d1 = h2 ? Dd.w : Dd.y;
+            const uint32_t pb = pp[16 * half + e];
+            const uint64_t pr = f2pack(bf16lo(pb), bf16hi(pb));
             const uint64_t dd = add2(
                 f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
                 f2pack(-d0, -d1));
             float ds0, ds1;
             f2unpack(fma2(pr, dd, 0ull), ds0, ds1);
-            pp[e] = pack_bf16(p0, p1);
             pd[e] = pack_bf16(ds0, ds1);
           }
         }
-        tmem_st16(tmem + lane_off + 128 * w + 16 * half, pp);
-        tmem_st16(tmem + lane_off + 128 * w + 64 + 16 * half, pd);
+        tmem_st16(t_dp + 16 * half, pd);
       }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->ps_full[w]);
+      mbar_arrive(&bars->ds_full[w]);
     }
     __syncwarp();
     if (failed) bars->abort_flag = 1;
