@@ -457,8 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float u = m_ref == -INFINITY ? 0.f : m_ref;
-        // p = 2^(s*sc - u): pairs on the f32x2 pipe; one pair in four takes the
-        // polynomial 2^x, the rest the multi-function unit.
+        // p = 2^(s*sc - u): pairs on the f32x2 pipe; some pairs take the
+        // polynomial 2^x on the FMA pipe, the rest the multi-function unit.
         const uint64_t sc2 = f2pack(sc, sc), nu2 = f2pack(-u, -u);
         uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -472,8 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             float x0, x1, p0, p1;
             f2unpack(x2, x0, x1);
             // Share of exponentials on the polynomial: V1's shorter Q.K^T leaves
-            // the softmax the critical path, so it offloads more (measured).
-            if (kForm == 1 ? (e & 3) == 3 : (e & 7) == 7) {
+            // the softmax the critical path, so it offloads more: three pairs in
+            // eight, spread over the row, against one in eight for V2 (both
+            // shares and positions measured).
+            if (kForm == 1 ? ((e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7) : (e & 7) == 7) {
               exp2_poly2(x0, x1, p0, p1);
             } else {
               p0 = ex2(x0);
