@@ -16,10 +16,13 @@
 // Two kernels:
 //   * dq kernel, one CTA per 128 query rows of a head (V1) or head pair
 //     (V2), walking 64-key tiles like the forward: per branch, S_r and dP_r
-//     into tensor memory (two SS MMAs), dS_r written back over S_r as bf16
-//     by the softmax-backward warps, then dQ_r += dS_r K_r (TS MMA) in
-//     tensor memory.  The softmax-backward warps form P as soon as S_r has
-//     landed and wait for dP_r only after that.  Warps: 0-3 / 4-7 branch 1 / 2 (thread = query row),
+//     into tensor memory (two SS MMAs), dS_r written as bf16 by the
+//     softmax-backward warps, then dQ_r += dS_r K_r in tensor memory.  V1
+//     writes dS_r back over S_r (TS MMA); V2, whose tensor memory has no
+//     second S buffer, writes it to swizzled shared memory (SS MMA) so that
+//     S_r(j+1) only waits for S_r(j) to be loaded.  The softmax-backward
+//     warps form P as soon as S_r has landed and wait for dP_r only after
+//     that.  Warps: 0-3 / 4-7 branch 1 / 2 (thread = query row),
 //     8 TMA producer, 9-12 the S_r and dP_r issuers (one thread per product
 //     stream, as in the forward), 13 / 14 dQ issuers.
 //   * dkdv kernel, one CTA per 128 keys of a head (V1) or KV head (V2),
@@ -80,6 +83,7 @@ struct DqBarriers {
   uint64_t dp_full[2];     // [branch]: dP_r landed
   uint64_t ds_full[2];     // [branch]: dS_r written back (and dP_r read)
   uint64_t dq_done[2][2];  // [branch][S buffer]: the dQ product of a tile has read its dS
+  uint64_t s_free[2];      // [branch], V2: the softmax backward has loaded S_r
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -99,7 +103,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   uint8_t* sdO = sQ + kQBytes;                     // 2 branches x 128 x 128
   uint8_t* sK = sdO + 2 * kTile128;                // stages x 64 x 128
   uint8_t* sV = sK + kDqStages * kTile64;
-  DqBarriers* bars = reinterpret_cast<DqBarriers*>(sV + kDqStages * kTile64);
+  // V2: dS_r (128 queries x 64 keys bf16, 128-byte swizzle, K-major) per branch
+  uint8_t* sDS = sV + kDqStages * kTile64;
+  DqBarriers* bars = reinterpret_cast<DqBarriers*>(sDS + (kForm == 2 ? 2 * kBox128 : 0));
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int mt = p.n_qtiles - 1 - (int)(blockIdx.x % p.n_qtiles);  // heavy tiles first
@@ -126,6 +132,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       mbar_init(&bars->ds_full[r], 128);
       mbar_init(&bars->dq_done[r][0], 1);
       mbar_init(&bars->dq_done[r][1], 1);
+      mbar_init(&bars->s_free[r], 128);
     }
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -138,9 +145,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  // tensor-memory columns: S_r, dP_r (64 each), dQ_r (D each); V1 leaves room
+  // tensor-memory columns: S_r, dP_r (64 each), dQ_r (D each).  V1 leaves room
   // for a second S buffer per branch at [384, 512), so S_r(j+1) can be computed
-  // while dS_r(j) still waits for its dQ product
+  // while dS_r(j), written back over S_r(j), still waits for its dQ product.  V2
+  // has no room for one; its dS_r goes to shared memory instead, so S_r(j+1)
+  // only waits for the softmax backward to have loaded S_r(j).
   constexpr int kSBufs = kForm == 1 ? 2 : 1;
   auto colS = [](int r, int j) {
     return (uint32_t)((kSBufs == 2 && (j & 1)) ? 384 + 64 * r : 128 * r);
@@ -198,9 +207,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           // S_r's buffer last held dS_r(j - kSBufs): its dQ product must have
           // read it; dP_r's buffer is free once the softmax backward has read
           // dP_r(j-1)
-          if (kind == 0 && j >= kSBufs &&
+          if (kForm == 1 && kind == 0 && j >= kSBufs &&
               !mbar_wait(&bars->dq_done[r][(j - kSBufs) & 1], (uint32_t)((j - kSBufs) >> 1) & 1u,
                          p.dev_status, &failed))
+            break;
+          if (kForm == 2 && kind == 0 && j >= 1 &&
+              !mbar_wait(&bars->s_free[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
             break;
           if (kind == 1 && j > 0 &&
               !mbar_wait(&bars->ds_full[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
@@ -247,10 +259,17 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           break;
         tc_fence_after();
         const uint32_t kt = smem_u32(sK) + s * kTile64 + (kForm == 1 ? r * kBox64 : 0);
-        for (int kk = 0; kk < 4; ++kk)  // 16 keys per step; B = K_r, MN-major
-          tc_mma_ts(tmem + colQ(r), tmem + colS(r, j) + kk * 8,
-                    smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
-                    (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {  // 16 keys per step; B = K_r, MN-major
+          if (kForm == 1)  // A = dS_r in tensor memory
+            tc_mma_ts(tmem + colQ(r), tmem + colS(r, j) + kk * 8,
+                      smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          else  // A = dS_r in shared memory, K-major
+            tc_mma_ss(tmem + colQ(r),
+                      smem_desc_sw128(smem_u32(sDS) + r * kBox128 + kk * 32, 16, 1024),
+                      smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        }
         tc_commit(&bars->dq_done[r][j & 1]);
         tc_commit(&bars->k_empty[s]);
       }
@@ -288,6 +307,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         uint32_t sv[32];
         tmem_ld32(tmem + lane_off + colS(r, j) + 32 * half, sv);
         tc_wait_ld();
+        if (kForm == 2 && half == 1) {  // S_r fully loaded: its buffer may take S_r(j+1)
+          tc_fence_before();
+          mbar_arrive(&bars->s_free[r]);
+        }
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           float x0, x1;
@@ -304,6 +327,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full[r], (uint32_t)j & 1u, p.dev_status,
+                                             &failed))) {
+        failed = true;
+        break;
+      }
+      // V2: the dQ product of the previous tile must have read dS_r out of
+      // shared memory before it is overwritten
+      if (kForm == 2 && j >= 1 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bars->dq_done[r][(j - 1) & 1],
+                                             (uint32_t)((j - 1) >> 1) & 1u, p.dev_status,
                                              &failed))) {
         failed = true;
         break;
@@ -325,8 +357,21 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                    ds0, ds1);
           pk[e] = pack_bf16(ds0, ds1);
         }
-        tmem_st16(tmem + lane_off + colS(r, j) + 16 * half, pk);
+        if (kForm == 1) {
+          tmem_st16(tmem + lane_off + colS(r, j) + 16 * half, pk);
+        } else {
+          // row `row` of the 128-byte-swizzled tile: 16-byte chunk c (8 keys)
+          // sits at chunk position c ^ (row & 7)
+          uint8_t* drow = sDS + r * kBox128 + row * 128;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int ch = 4 * half + c4;
+            *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
+                make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+          }
+        }
       }
+      if (kForm == 2) fence_proxy_async_smem();  // visible to the tensor core
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_full[r]);
@@ -905,7 +950,7 @@ cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
   {
     const int qbytes = a.fwd.form == 1 ? kTile128 : 2 * kTile128;
     const int smem = 1024 + qbytes + 2 * kTile128 + 2 * kDqStages * kTile64 +
-                     (int)sizeof(DqBarriers) + 64;
+                     (a.fwd.form == 2 ? 2 * kBox128 : 0) + (int)sizeof(DqBarriers) + 64;
     decltype(&diffattn_bwd_dq_kernel<1, false>) k =
         a.fwd.form == 1 ? (win ? diffattn_bwd_dq_kernel<1, true> : diffattn_bwd_dq_kernel<1, false>)
                         : (win ? diffattn_bwd_dq_kernel<2, true> : diffattn_bwd_dq_kernel<2, false>);
