@@ -23,6 +23,7 @@ DA_ERR_ALIGNMENT = -3
 DA_ERR_WORKSPACE = -4
 DA_ERR_CUDA = -5
 DA_ERR_DEVICE_TIMEOUT = -6
+DA_ERR_SCHEDULE = -7
 DA_BF16 = 0
 DA_FP32 = 1
 
@@ -49,6 +50,9 @@ EXPORTS = (
     "lambda_from_params_bwd",
     "diffattn_v2_prefill_oproj_workspace_size",
     "diffattn_v2_prefill_oproj",
+    "diffattn_reset_tile_counters",
+    "diffattn_selftest_hold_tile_counter",
+    "diffattn_selftest_keep_tile_counter",
     "diffattn_selftest_wait_timeout",
 )
 
@@ -133,6 +137,12 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.diffattn_v2_prefill_oproj.restype = _i
     lib.diffattn_v2_prefill_oproj.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                               _i, _i, _i, _i, _vp, _sz, _vp, _vp]
+    lib.diffattn_reset_tile_counters.restype = _i
+    lib.diffattn_reset_tile_counters.argtypes = [_vp]
+    lib.diffattn_selftest_hold_tile_counter.restype = _i
+    lib.diffattn_selftest_hold_tile_counter.argtypes = [_i, ctypes.c_uint, ctypes.c_uint, _vp]
+    lib.diffattn_selftest_keep_tile_counter.restype = _i
+    lib.diffattn_selftest_keep_tile_counter.argtypes = [_i, ctypes.c_uint, ctypes.c_uint, _vp]
     lib.diffattn_selftest_wait_timeout.restype = _i
     lib.diffattn_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp, _vp, _vp]
     _lib = lib
@@ -378,9 +388,10 @@ def diffattn_v1_bwd_workspace_size(batch, seqlen, n_heads, d_qk, d_v) -> int:
 
 def diffattn_v1_bwd(q, k, v, dout, lam, *, causal=True, window=0, apply_norm=False,
                     norm_weight=None, norm_eps=1e-5, lambda_init=0.0, workspace=None,
-                    dev_status=None, stream=None):
+                    out=None, dev_status=None, stream=None):
     """V1 gradients.  Returns dict of fp32 device tensors dq, dk (like q),
-    dv (like v), dlambda [H] and, with the norm, dnorm_weight [dv]."""
+    dv (like v), dlambda [H] and, with the norm, dnorm_weight [dv]; `out`
+    may supply any of them (caller-owned, written in place)."""
     _need_cuda(q, k, v, dout, lam, norm_weight)
     B, N, H, d2 = q.shape
     dvw = v.shape[-1]
@@ -391,6 +402,7 @@ def diffattn_v1_bwd(q, k, v, dout, lam, *, causal=True, window=0, apply_norm=Fal
     res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
            "dv": torch.empty(v.shape, **f32), "dlambda": torch.empty(H, **f32),
            "dnorm_weight": torch.empty(dvw, **f32) if apply_norm else None}
+    res.update(out or {})
     _check("diffattn_v1_bwd", load().diffattn_v1_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lam), _dtype_code(q), B, N, H, d2 // 2,
         dvw, int(bool(causal)), int(window), int(bool(apply_norm)), _ptr(norm_weight),
@@ -406,9 +418,9 @@ def diffattn_v2_bwd_workspace_size(batch, seqlen, n_q_heads, n_kv_heads, head_di
 
 
 def diffattn_v2_bwd(q, k, v, dout, lam, *, causal=True, window=0, workspace=None,
-                    dev_status=None, stream=None):
+                    out=None, dev_status=None, stream=None):
     """V2 gradients.  Returns dict of fp32 device tensors dq (like q), dk,
-    dv (like k) and dlambda [Hq/2]."""
+    dv (like k) and dlambda [Hq/2]; `out` may supply any of them."""
     _need_cuda(q, k, v, dout, lam)
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -418,6 +430,7 @@ def diffattn_v2_bwd(q, k, v, dout, lam, *, causal=True, window=0, workspace=None
     f32 = dict(dtype=torch.float32, device=q.device)
     res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
            "dv": torch.empty(v.shape, **f32), "dlambda": torch.empty(Hq // 2, **f32)}
+    res.update(out or {})
     _check("diffattn_v2_bwd", load().diffattn_v2_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lam), _dtype_code(q), B, N, Hq, Hkv, d,
         int(bool(causal)), int(window), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
@@ -470,3 +483,24 @@ def diffattn_selftest_wait_timeout(timeout_us, dev_status, waited_ns=None, strea
     _need_cuda(dev_status, waited_ns)
     _check("diffattn_selftest_wait_timeout", load().diffattn_selftest_wait_timeout(
         int(timeout_us), _ptr(dev_status), _ptr(waited_ns), _stream(stream)))
+
+
+def diffattn_reset_tile_counters(stream=None):
+    """Free every tile counter of the tensor-core prefill on the current
+    device (see the header)."""
+    _check("diffattn_reset_tile_counters",
+           load().diffattn_reset_tile_counters(_stream(stream)))
+
+
+def diffattn_selftest_hold_tile_counter(slot, tag, count, stream=None):
+    """Test hook: set tile counter `slot` to (tag, count) and make the next
+    tensor-core prefill launch take it (see the header)."""
+    _check("diffattn_selftest_hold_tile_counter", load().diffattn_selftest_hold_tile_counter(
+        int(slot), int(tag), int(count), _stream(stream)))
+
+
+def diffattn_selftest_keep_tile_counter(slot, tag, duration_ms, stream=None):
+    """Test hook: keep tile counter `slot` held by `tag`, as a launch in
+    flight would, for `duration_ms` (see the header)."""
+    _check("diffattn_selftest_keep_tile_counter", load().diffattn_selftest_keep_tile_counter(
+        int(slot), int(tag), int(duration_ms), _stream(stream)))

@@ -100,8 +100,26 @@ const char* diffattn_status_string(int status) {
     case DA_ERR_WORKSPACE: return "DA_ERR_WORKSPACE";
     case DA_ERR_CUDA: return "DA_ERR_CUDA";
     case DA_ERR_DEVICE_TIMEOUT: return "DA_ERR_DEVICE_TIMEOUT";
+    case DA_ERR_SCHEDULE: return "DA_ERR_SCHEDULE";
     default: return "DA_ERR_UNKNOWN";
   }
+}
+
+int diffattn_reset_tile_counters(void* stream) {
+  return cuda_status(da::reset_tile_counters(static_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_selftest_hold_tile_counter(int slot, unsigned int tag, unsigned int count,
+                                        void* stream) {
+  if (slot < 0 || slot >= 64) return DA_ERR_INVALID_ARG;
+  return cuda_status(da::hold_tile_counter(slot, tag, count, static_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_selftest_keep_tile_counter(int slot, unsigned int tag, unsigned int duration_ms,
+                                        void* stream) {
+  if (slot < 0 || slot >= 64 || duration_ms < 1 || duration_ms > 10000) return DA_ERR_INVALID_ARG;
+  return cuda_status(
+      da::keep_tile_counter(slot, tag, duration_ms, static_cast<cudaStream_t>(stream)));
 }
 
 double diffattn_lambda_init(int layer) {

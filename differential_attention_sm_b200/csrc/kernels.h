@@ -104,6 +104,11 @@ struct PrefillArgs {
 cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                               const CUtensorMap& tm_v, const PrefillArgs& a, int num_sms,
                               cudaStream_t stream);
+// Tile counters of the tensor-core prefill (64 per device): free them all, or
+// set one to (tag, count) and make the next launch of this process take it.
+cudaError_t reset_tile_counters(cudaStream_t stream);
+cudaError_t hold_tile_counter(int slot, unsigned tag, unsigned count, cudaStream_t stream);
+cudaError_t keep_tile_counter(int slot, unsigned tag, unsigned duration_ms, cudaStream_t stream);
 
 // ---- fused tcgen05 backward (bf16; V1 d_qk 64 / d_v 128, V2 head_dim 128) --
 struct FusedBwdArgs {

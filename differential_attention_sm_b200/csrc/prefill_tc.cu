@@ -162,22 +162,91 @@ __device__ __forceinline__ Tile tile_at(const Params& p, int id, int form, bool 
   return t;
 }
 
-// Tile counters.  A launch takes one of these slots in turn, so launches
-// that run at the same time (on different streams) count on different
-// counters as long as fewer than kTicketSlots are in flight together.
+// Tile counters.  The host hands each launch one of these slots in turn, so
+// launches that run at the same time on different streams normally count on
+// different slots.  A slot is one 64-bit word: the tag of the launch that
+// holds it in the high half and the tickets taken so far in the low half.
+//   * A launch claims a slot whose count is zero (free) with one
+//     compare-and-swap that writes its tag and count 1 (ticket 0); every later
+//     unit of work of the same launch takes the next ticket with a plain
+//     atomic add, so the CTAs that start together do not contend on a CAS.
+//   * A launch takes exactly one ticket per tile; the unit that takes the last
+//     one clears the count, so a finished launch leaves the slot free.
+//   * The first unit of a CTA that finds the slot held by another launch
+//     (two executions of one captured launch that overlap, or more launches
+//     in flight than slots) waits for that launch to hand out its last tile,
+//     then claims the slot.  The holder has a resident CTA that never waits
+//     on this one, so the wait ends; it is still bounded: after
+//     kScheduleWaitNs it gives up and DA_ERR_SCHEDULE is reported, so an
+//     incomplete output never comes with status 0.  A holder whose word has
+//     not changed for kStaleNs has stopped taking tickets (a launch that
+//     ended with DA_ERR_DEVICE_TIMEOUT); its slot is taken over.
+//   * Every later unit of a CTA finds its own launch's tag (the launch holds
+//     the slot until its last ticket); anything else is reported at once.
+// The tag is the grid's %gridid, which differs between launches that are in
+// flight at the same time (graph replays included).
 constexpr int kTicketSlots = 64;
-__device__ unsigned g_tickets[kTicketSlots];
+constexpr uint64_t kScheduleWaitNs = 2000000000ull;  // below the 4 s pipeline waits
+constexpr uint64_t kStaleNs = 250000000ull;
+__device__ unsigned long long g_tickets[kTicketSlots];
+__device__ unsigned g_gave_up[kTicketSlots];  // tag of the last launch that gave up waiting
 
-// One ticket per unit of work (a CTA that starts, or a CTA it cancels): the
-// counter runs modulo n_tiles, so a launch takes each tile number exactly
-// once and leaves the counter where it found it (zero).  A counter left
-// elsewhere by an aborted launch only rotates the next launch's order; a
-// value at or above n_tiles (left by a larger launch) wraps to zero on the
-// first ticket and is skipped.
-__device__ __forceinline__ int take_ticket(unsigned* ctr, int n_tiles) {
-  for (int i = 0; i < 4; ++i) {
-    const unsigned t = atomicInc(ctr, (unsigned)n_tiles - 1u);
-    if (t < (unsigned)n_tiles) return (int)t;
+__device__ __forceinline__ uint32_t launch_tag() {
+  uint64_t g;
+  asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
+  const uint32_t t = (uint32_t)(g ^ (g >> 32));
+  return t ? t : 1u;  // 0 marks a slot that no launch has used
+}
+
+// One ticket per unit of work (a CTA that starts, or a CTA it cancels):
+// returns the tile number, or -1 (the caller reports DA_ERR_SCHEDULE).
+// `first`: the CTA's own unit, the only one that may wait for or claim a slot.
+__device__ __noinline__ int take_ticket(int slot, int n_tiles, uint32_t tag, bool first) {
+  unsigned long long* ctr = g_tickets + slot;
+  volatile unsigned long long* vctr = ctr;
+  const unsigned long long claim =
+      ((unsigned long long)tag << 32) | (n_tiles == 1 ? 0ull : 1ull);
+  unsigned long long cur = *vctr, seen = 0ull;
+  uint64_t t0 = 0, t_seen = 0;
+  unsigned sleep_ns = 64;
+  for (uint32_t iter = 0; iter < (1u << 26); ++iter) {
+    if ((uint32_t)(cur >> 32) == tag) {
+      const unsigned long long old = atomicAdd(ctr, 1ull);
+      const uint32_t t = (uint32_t)old;
+      if ((uint32_t)(old >> 32) != tag || t >= (uint32_t)n_tiles) return -1;
+      if (t == (uint32_t)n_tiles - 1u) atomicAnd(ctr, 0xffffffff00000000ull);  // last: free
+      return (int)t;
+    }
+    if (!first) return -1;
+    // a CTA of this launch has already given up on the slot: so does this one
+    if (*reinterpret_cast<volatile unsigned*>(g_gave_up + slot) == tag) return -1;
+    if ((uint32_t)cur == 0u) {  // free: claim it
+      const unsigned long long prev = atomicCAS(ctr, cur, claim);
+      if (prev == cur) return 0;
+      cur = prev;  // lost the race (normally to a CTA of this launch): look again
+      continue;
+    }
+    // held by another launch: wait for it to hand out its last tile
+    const uint64_t now = global_ns();
+    if (t0 == 0) {
+      t0 = t_seen = now;
+      seen = cur;
+    } else if (cur != seen) {
+      seen = cur;
+      t_seen = now;
+    } else if (now - t_seen > kStaleNs) {  // the holder has stopped: take over
+      const unsigned long long prev = atomicCAS(ctr, cur, claim);
+      if (prev == cur) return 0;
+      cur = prev;
+      continue;
+    }
+    if (now - t0 > kScheduleWaitNs) {
+      g_gave_up[slot] = tag;
+      return -1;
+    }
+    __nanosleep(sleep_ns);
+    if (sleep_ns < 8192) sleep_ns *= 2;
+    cur = *vctr;
   }
   return -1;
 }
@@ -261,7 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       uint32_t J = 0;
-      int id = take_ticket(g_tickets + p.ticket_slot, p.n_tiles);
+      const uint32_t tag = launch_tag();
+      int id = take_ticket(p.ticket_slot, p.n_tiles, tag, true);
+      if (id < 0) report(p.dev_status, DA_ERR_SCHEDULE);
       for (int tc = 0;; ++tc) {
         // publish the tile number once every role has read the one before last
         const uint32_t u = (uint32_t)tc >> 1;
@@ -303,8 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bars->clc_full, 16);
         clc_try_cancel(bars->clc_resp, &bars->clc_full);
         if (!mbar_wait(&bars->clc_full, (uint32_t)tc & 1u, p.dev_status, &failed)) break;
-        id = clc_response(bars->clc_resp) >= 0 ? take_ticket(g_tickets + p.ticket_slot, p.n_tiles)
-                                                : -1;
+        if (clc_response(bars->clc_resp) < 0) {
+          id = -1;
+        } else {
+          id = take_ticket(p.ticket_slot, p.n_tiles, tag, false);
+          if (id < 0) report(p.dev_status, DA_ERR_SCHEDULE);
+        }
       }
     }
   } else if (warp == 9 || warp == 10) {
@@ -616,7 +691,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
 }
+// Host side of the tile counters: the slot the next launch takes.
+std::atomic<unsigned> g_next_slot{0};
+
+// Self-test: keeps counter `slot` held by `tag` with a count that changes
+// every ~20 us (a launch in flight, as another launch sees it) for
+// `duration_ns`, then frees it.
+__global__ void keep_ticket_word_kernel(int slot, unsigned tag, unsigned long long duration_ns) {
+  const uint64_t t0 = global_ns();
+  unsigned k = 1;
+  while (global_ns() - t0 < duration_ns) {
+    g_tickets[slot] = ((unsigned long long)tag << 32) | (unsigned long long)k;
+    k = k % 1000000u + 1u;
+    __nanosleep(20000);
+  }
+  g_tickets[slot] = (unsigned long long)tag << 32;
+}
+
+__global__ void set_ticket_word_kernel(int slot, unsigned long long value) {
+  if (slot < 0) {
+    for (int i = 0; i < kTicketSlots; ++i) {
+      g_tickets[i] = 0ull;
+      g_gave_up[i] = 0u;
+    }
+  } else {
+    g_tickets[slot] = value;
+  }
+}
 }  // namespace
+
+cudaError_t reset_tile_counters(cudaStream_t stream) {
+  set_ticket_word_kernel<<<1, 1, 0, stream>>>(-1, 0ull);
+  return cudaGetLastError();
+}
+
+cudaError_t hold_tile_counter(int slot, unsigned tag, unsigned count, cudaStream_t stream) {
+  if (slot < 0 || slot >= kTicketSlots) return cudaErrorInvalidValue;
+  set_ticket_word_kernel<<<1, 1, 0, stream>>>(
+      slot, ((unsigned long long)tag << 32) | (unsigned long long)count);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) g_next_slot.store((unsigned)slot, std::memory_order_relaxed);
+  return e;
+}
+
+cudaError_t keep_tile_counter(int slot, unsigned tag, unsigned duration_ms,
+                              cudaStream_t stream) {
+  if (slot < 0 || slot >= kTicketSlots || duration_ms == 0 || duration_ms > 10000)
+    return cudaErrorInvalidValue;
+  keep_ticket_word_kernel<<<1, 1, 0, stream>>>(slot, tag, 1000000ull * duration_ms);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) g_next_slot.store((unsigned)slot, std::memory_order_relaxed);
+  return e;
+}
 
 cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                               const CUtensorMap& tm_v, const PrefillArgs& a, int num_sms,
@@ -629,8 +755,7 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.heads = a.heads;
   p.pairs_per_kv = a.pairs_per_kv;
   p.n_qtiles = (a.seqlen + kBM - 1) / kBM;
-  static std::atomic<unsigned> next_slot{0};
-  p.ticket_slot = (int)(next_slot.fetch_add(1u, std::memory_order_relaxed) % kTicketSlots);
+  p.ticket_slot = (int)(g_next_slot.fetch_add(1u, std::memory_order_relaxed) % kTicketSlots);
   // Heads (V1) or pairs (V2) scheduled together: as many as keep their K and
   // V (2 x seqlen x 128 bf16 per KV head) within about half of the L2.
   const double kv_bytes = 2.0 * a.seqlen * 128 * 2;

@@ -29,14 +29,25 @@
  *  - Thread safety: concurrent calls on different streams are independent,
  *    with two exceptions: diffattn_v2_decode_noalloc's shared scratch array
  *    (see that entry point) and the prefill's tile counters (next).  Global
- *    state: a per-device cuBLAS handle for the backward and the output
- *    projection, created under a lock on first use, and, for the bf16
- *    tensor-core prefill (diffattn_v1_fwd / diffattn_v2_prefill and their
- *    window, training and projection variants), 64 tile counters per device
- *    in a statically allocated array.  Each such launch takes the next
- *    counter in turn and leaves it at zero when it completes, so at most 64
- *    of them may execute on one device at the same time (on several streams,
- *    or as replays of CUDA graphs).
+ *    state: a per-device cuBLAS handle for the materialising backward,
+ *    created under a lock on first use, and, for the bf16 tensor-core
+ *    prefill (diffattn_v1_fwd / diffattn_v2_prefill and their window,
+ *    training and projection variants), 64 tile counters per device in a
+ *    statically allocated array.  The host gives each such launch the next
+ *    counter in turn, fixed when the launch is enqueued (or captured into a
+ *    CUDA graph, whose every replay then uses that counter).  On the device
+ *    a launch claims its counter when it is free, hands out one tile per
+ *    ticket and frees it when its last tile is taken.  A launch that finds
+ *    its counter held by another launch still in flight (two graph
+ *    executions made from one capture that overlap, or more than 64 launches
+ *    in flight on one device) waits until that launch has taken its last
+ *    tile, then proceeds: overlapping launches stay correct.  That wait is
+ *    bounded: after 2 s the waiting CTAs compute nothing and store
+ *    DA_ERR_SCHEDULE in dev_status, so an incomplete output never comes with
+ *    status 0 (pass a status word to see it).  A counter whose holder has
+ *    stopped taking tickets for 250 ms (a launch that ended with
+ *    DA_ERR_DEVICE_TIMEOUT) is taken over; diffattn_reset_tile_counters
+ *    frees every counter at once.
  */
 #ifndef DIFFATTN_H_
 #define DIFFATTN_H_
@@ -60,7 +71,9 @@ typedef enum {
   DA_ERR_ALIGNMENT = -3,     /* a base address is not 16-byte aligned */
   DA_ERR_WORKSPACE = -4,     /* workspace missing or smaller than required */
   DA_ERR_CUDA = -5,          /* a CUDA runtime/driver call or launch failed */
-  DA_ERR_DEVICE_TIMEOUT = -6 /* written to dev_status by a kernel whose wait timed out */
+  DA_ERR_DEVICE_TIMEOUT = -6, /* written to dev_status by a kernel whose wait timed out */
+  DA_ERR_SCHEDULE = -7        /* written to dev_status by a prefill launch whose tile
+                                 counter another launch held for longer than 2 s */
 } da_status;
 
 typedef enum { DA_BF16 = 0, DA_FP32 = 1 } da_dtype;
@@ -174,8 +187,11 @@ DA_API int diffattn_v2_decode(const void* q, const void* k_cache, const void* v_
  *    scratch (batch * n_kv_heads above 2016) return DA_ERR_UNSUPPORTED
  *    before anything is enqueued.
  *  - Set-up: the first call on a device, with that device current, looks up
- *    the array's device address (cudaGetSymbolAddress) and caches it; make
- *    that first call before any stream capture.
+ *    the array's device address (cudaGetSymbolAddress) and caches it with
+ *    the device's current CUDA context; make that first call before any
+ *    stream capture.  A call under another context of that device (after
+ *    cudaDeviceReset, or under a context made with the driver API) looks the
+ *    address up again first, so make such a call outside capture too.
  *  - Every call on a device shares the one array, which keeps the last
  *    call's contents; nothing in it needs to start at zero.  Calls whose
  *    execution overlaps on the GPU (other streams, other host threads) race
@@ -330,6 +346,34 @@ DA_API int diffattn_v2_prefill_oproj(const void* q, const void* k, const void* v
                                      int n_kv_heads, int head_dim, int d_model, int causal,
                                      int window, void* workspace, size_t workspace_bytes,
                                      int* dev_status, void* stream);
+
+/* ---- Tile counters of the tensor-core prefill ------------------------------
+ * No counterpart on the pages (they are this library's scheduling state).
+ * diffattn_reset_tile_counters frees all 64 counters of the current device
+ * by a one-thread kernel enqueued on `stream`.  It is meant for recovery
+ * after a prefill launch reported DA_ERR_DEVICE_TIMEOUT (which can leave its
+ * counter held); no tensor-core prefill launch may be in flight on the
+ * device while it runs.  Returns DA_ERR_CUDA if the launch fails.
+ *
+ * diffattn_selftest_hold_tile_counter is a test hook: it enqueues a write of
+ * (tag, count) into counter `slot` (0 .. 63) and makes the next tensor-core
+ * prefill launch of this process take that counter.  With count > 0 and a
+ * tag no launch has, the counter looks held by a launch that stopped: the
+ * next launch takes it over after 250 ms.  With count = 0 it is free.
+ * Returns DA_ERR_INVALID_ARG for a slot out of range. */
+DA_API int diffattn_reset_tile_counters(void* stream);
+DA_API int diffattn_selftest_hold_tile_counter(int slot, unsigned int tag, unsigned int count,
+                                               void* stream);
+
+/* Test hook: enqueues a one-thread kernel that keeps counter `slot` held by
+ * `tag` with a count that changes every ~20 us (as a launch in flight would)
+ * for `duration_ms` (1 .. 10000), then frees it; the next tensor-core
+ * prefill launch of this process takes that counter.  A prefill launch that
+ * runs meanwhile on another stream waits for it and, if it is still held
+ * after 2 s, reports DA_ERR_SCHEDULE.  Returns DA_ERR_INVALID_ARG for a slot
+ * or duration out of range. */
+DA_API int diffattn_selftest_keep_tile_counter(int slot, unsigned int tag,
+                                               unsigned int duration_ms, void* stream);
 
 /* ---- Self-test of the failure report ----------------------------------------
  * No counterpart on the pages.  Launches one CTA whose thread waits on an

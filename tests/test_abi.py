@@ -49,6 +49,7 @@ def test_lambda_init_and_status_strings(lib):
         assert b.diffattn_lambda_init(l) == pytest.approx(oracle.lambda_init(l), abs=1e-15)
     assert b.status_string(b.DA_OK) == "DA_OK"
     assert b.status_string(b.DA_ERR_DEVICE_TIMEOUT) == "DA_ERR_DEVICE_TIMEOUT"
+    assert b.status_string(b.DA_ERR_SCHEDULE) == "DA_ERR_SCHEDULE"
     assert b.status_string(12345) == "DA_ERR_UNKNOWN"
 
 
@@ -226,3 +227,11 @@ def test_selftest_host_validation(lib):
     assert f(1000, None, None, None) == b.DA_ERR_INVALID_ARG
     assert f(0, A, None, None) == b.DA_ERR_INVALID_ARG
     assert f(2000000, A, None, None) == b.DA_ERR_INVALID_ARG
+    # the tile-counter hook checks its slot before enqueuing anything
+    g = lib.diffattn_selftest_hold_tile_counter
+    assert g(-1, 0, 0, None) == b.DA_ERR_INVALID_ARG
+    assert g(64, 0, 0, None) == b.DA_ERR_INVALID_ARG
+    k = lib.diffattn_selftest_keep_tile_counter
+    assert k(64, 1, 10, None) == b.DA_ERR_INVALID_ARG
+    assert k(0, 1, 0, None) == b.DA_ERR_INVALID_ARG
+    assert k(0, 1, 10001, None) == b.DA_ERR_INVALID_ARG
