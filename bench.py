@@ -31,6 +31,10 @@ if ROOT not in sys.path:
 
 METRIC = "DiffAttn fwd TFLOP/s (prefill), decode HBM GB/s; % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# The decode target (70 % of HBM bandwidth) is stated against about 8 TB/s of
+# nominal HBM3e bandwidth; the measured peak is a read+write copy, which a
+# pure read stream can exceed, so decode lines report both fractions.
+NOMINAL_HBM_GBS = 8000.0
 
 
 # ---------------------------------------------------------------------------
@@ -336,13 +340,59 @@ def time_call(fn, iters, warmup, stream):
     return a.elapsed_time(b) / iters
 
 
-def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
+def oracle_rate(run_once, target_s: float, unit_scale: float, what: str):
+    """Bounded CPU-baseline sample: calls ``run_once(n)`` (runs the oracle on
+    n units of the workload and returns the algorithmic work it covered)
+    with n doubling until about ``target_s`` seconds of host time are spent.
+    Returns the ``cpu_baseline`` object for one workload."""
+    import oracle as O
+    n, work, secs, units = 1, 0.0, 0.0, 0
+    while secs < target_s:
+        t0 = time.perf_counter()
+        work += run_once(n)
+        dt = time.perf_counter() - t0
+        secs += dt
+        units += n
+        if dt < target_s / 4:
+            n *= 2
+    return {"value": work / secs / unit_scale, "cores": O.n_threads(), "kind": "oracle",
+            "sample": "%d %s (%.1f s)" % (units, what, secs)}
+
+
+def _rows_sampler(fn, total_rows, per_row_work, seed):
+    """run_once(n) for row-wise oracle calls: n random output rows."""
+    rng = np.random.default_rng(seed)
+
+    def run_once(n):
+        rows = rng.integers(0, total_rows, n)
+        fn(rows)
+        return float(sum(per_row_work(int(r)) for r in rows))
+    return run_once
+
+
+def _decode_sampler(ref_entry, caches, B, per_entry_bytes, seed):
+    """run_once(n) for decode: n random batch entries, each entry's cache
+    slices copied to the host, all of its outputs by the oracle."""
+    rng = np.random.default_rng(seed)
+
+    def run_once(n):
+        for b in rng.integers(0, B, n):
+            k, v = caches[0][int(b)].cpu(), caches[1][int(b)].cpu()
+            ref_entry(int(b), k, v)
+        return float(n * per_entry_bytes)
+    return run_once
+
+
+def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None, cpu_s=2.0):
     """The other workloads, one GPU: V2 prefill, V1 long-context prefill,
     V2 decode and V1 decode (same kernels the parity tests check).
     `only` restricts the run to one of them and `decode_batch` shrinks the
-    decode batch (used for small profiling runs)."""
+    decode batch (used for small profiling runs).  Each entry carries the
+    oracle timed on a bounded sample of its workload (``cpu_baseline``,
+    about ``cpu_s`` seconds of host work; 0 skips it)."""
     import dataclasses
 
+    import oracle as O
     import torch
     from differential_attention_sm_b200 import binding as Bd
     from differential_attention_sm_b200 import inputs as I
@@ -371,6 +421,12 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         out["v2_prefill_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
                                   "frac": round(t / peaks["bf16_tflops"], 4),
                                   "peak": peaks["bf16_tflops"], "flop": fl}
+        if cpu_s > 0:
+            P_ = w.Hq // 2
+            out["v2_prefill_bf16"]["cpu_baseline"] = dict(oracle_rate(_rows_sampler(
+                lambda r: O.v2_rows(x["q"], x["k"], x["v"], x["lam"], r, causal=True),
+                w.B * w.N * P_, lambda r: ((r // P_) % w.N + 1) * v2_flops_per_pair(w.d), 11),
+                cpu_s, 1e12, "random output rows"), unit="TFLOP/s")
         del q, k, v, o, x
 
     if want("v1_long_bf16"):  # B1 H16 N32768, layer 24, planted signal
@@ -387,6 +443,13 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         t = fl / (ms * 1e-3) / 1e12
         out["v1_long_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
                                "frac": round(t / peaks["bf16_tflops"], 4), "flop": fl}
+        if cpu_s > 0:
+            lam_h = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+            out["v1_long_bf16"]["cpu_baseline"] = dict(oracle_rate(_rows_sampler(
+                lambda r: O.v1_rows(x["q"], x["k"], x["v"], lam_h, r, causal=True,
+                                    apply_norm=True, eps=w.eps, lambda_init_value=li),
+                w.B * w.N * w.H, lambda r: ((r // w.H) % w.N + 1) * v1_flops_per_pair(w.d, w.dv),
+                12), cpu_s, 1e12, "random output rows"), unit="TFLOP/s")
         del q, k, v, o, x
 
     if want("v2_decode_bf16"):  # B64 L32768 Hq64 Hkv8 d128
@@ -405,7 +468,16 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         gbs = by / (ms * 1e-3) / 1e9
         out["v2_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
                                  "frac": round(gbs / peaks["hbm_gbs"], 4),
-                                 "peak": peaks["hbm_gbs"], "bytes": by, "batch": w.B}
+                                 "peak": peaks["hbm_gbs"], "bytes": by, "batch": w.B,
+                                 "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4),
+                                 "target": ">= 0.70 of the nominal %.0f GB/s" % NOMINAL_HBM_GBS}
+        if cpu_s > 0:
+            P_ = w.Hq // 2
+            out["v2_decode_bf16"]["cpu_baseline"] = dict(oracle_rate(_decode_sampler(
+                lambda b, k_, v_: O.v2_decode_rows(x["q"][b:b + 1], k_[None], v_[None], x["lam"],
+                                                   np.arange(P_)),
+                (kc, vc), w.B, v2_decode_bytes(1, w.L, w.Hkv, w.d, w.Hq), 13),
+                cpu_s, 1e9, "batch entries, every output"), unit="GB/s")
         del kc, vc, ws
         torch.cuda.empty_cache()
 
@@ -430,7 +502,16 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         gbs = by / (ms * 1e-3) / 1e9
         out["v1_decode_bf16"] = {"value": round(gbs, 1), "unit": "GB/s", "ms": round(ms, 4),
                                  "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": by,
-                                 "batch": w.B}
+                                 "batch": w.B,
+                                 "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4)}
+        if cpu_s > 0:
+            lam_h = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+            out["v1_decode_bf16"]["cpu_baseline"] = dict(oracle_rate(_decode_sampler(
+                lambda b, k_, v_: O.v1_decode_rows(x["q"][b:b + 1], k_[None], v_[None], lam_h,
+                                                   np.arange(w.H), apply_norm=True, eps=w.eps,
+                                                   lambda_init_value=li),
+                (kc, vc), w.B, v1_decode_bytes(1, w.L, w.H, w.d, w.dv), 14),
+                cpu_s, 1e9, "batch entries, every output"), unit="GB/s")
         del kc, vc, ws
         torch.cuda.empty_cache()
 
@@ -449,6 +530,13 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
                                          "ms": round(ms, 4),
                                          "frac": round(t / peaks["bf16_tflops"], 4),
                                          "flop": flop, "window": W}
+        if cpu_s > 0:
+            P_ = w.Hq // 2
+            out["v2_prefill_window_bf16"]["cpu_baseline"] = dict(oracle_rate(_rows_sampler(
+                lambda r: O.v2_rows(x["q"], x["k"], x["v"], x["lam"], r, causal=True, window=W),
+                w.B * w.N * P_,
+                lambda r: min((r // P_) % w.N + 1, W) * v2_flops_per_pair(w.d), 15),
+                cpu_s, 1e12, "random output rows"), unit="TFLOP/s")
         del q, k, v, o
         torch.cuda.empty_cache()
 
@@ -472,7 +560,16 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         out["v2_decode_window_bf16"] = {"value": round(gbs, 1), "unit": "GB/s",
                                         "ms": round(ms, 4),
                                         "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": by,
-                                        "batch": w.B, "window": W}
+                                        "batch": w.B, "window": W,
+                                        "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4)}
+        if cpu_s > 0:  # the oracle reads the window's entries only: copy just those
+            P_ = w.Hq // 2
+            out["v2_decode_window_bf16"]["cpu_baseline"] = dict(oracle_rate(_decode_sampler(
+                lambda b, k_, v_: O.v2_decode_rows(x["q"][b:b + 1], k_[None], v_[None], x["lam"],
+                                                   np.arange(P_)),
+                (kc[:, w.L - span:], vc[:, w.L - span:]), w.B,
+                v2_decode_bytes(1, span, w.Hkv, w.d, w.Hq), 16),
+                cpu_s, 1e9, "batch entries, every output"), unit="GB/s")
         del kc, vc, ws
         torch.cuda.empty_cache()
 
@@ -494,6 +591,22 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         out["v1_backward_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
                                    "frac": round(t / peaks["bf16_tflops"], 4), "flop": flop,
                                    "workspace_bytes": ws.numel()}
+        if cpu_s > 0:  # the oracle's backward on (batch, head) slices of the first 512 tokens
+            lam_h = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+            g_h = dout.cpu()
+            rng = np.random.default_rng(17)
+            n_p = 512
+
+            def bwd_once(n):
+                for _ in range(n):
+                    b, h = int(rng.integers(w.B)), int(rng.integers(w.H))
+                    sl = (slice(b, b + 1), slice(0, n_p), slice(h, h + 1))
+                    O.v1_bwd(x["q"][sl], x["k"][sl], x["v"][sl], g_h[sl], lam_h[h:h + 1],
+                             causal=True, apply_norm=True, eps=w.eps, lambda_init_value=li)
+                return float(n * prefill_pairs(1, n_p, 1) * v1_bwd_flops_per_pair(w.d, w.dv))
+            out["v1_backward_bf16"]["cpu_baseline"] = dict(oracle_rate(
+                bwd_once, cpu_s, 1e12, "(batch, head) slices of the first 512 tokens"),
+                unit="TFLOP/s", cores=1)
         del q, k, v, dout, ws
         torch.cuda.empty_cache()
 
@@ -511,6 +624,23 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
         out["v2_backward_bf16"] = {"value": round(t, 2), "unit": "TFLOP/s", "ms": round(ms, 4),
                                    "frac": round(t / peaks["bf16_tflops"], 4), "flop": flop,
                                    "workspace_bytes": ws.numel()}
+        if cpu_s > 0:  # the oracle's backward on (batch, KV head) slices of 512 tokens
+            g_h = dout.cpu()
+            rng = np.random.default_rng(18)
+            n_p, grp = 512, w.Hq // w.Hkv
+
+            def bwd_once(n):
+                for _ in range(n):
+                    b, g = int(rng.integers(w.B)), int(rng.integers(w.Hkv))
+                    tq = (slice(b, b + 1), slice(0, n_p), slice(g * grp, (g + 1) * grp))
+                    tk = (slice(b, b + 1), slice(0, n_p), slice(g, g + 1))
+                    to = (slice(b, b + 1), slice(0, n_p), slice(g * grp // 2, (g + 1) * grp // 2))
+                    O.v2_bwd(x["q"][tq], x["k"][tk], x["v"][tk], g_h[to],
+                             x["lam"][g * grp // 2:(g + 1) * grp // 2], causal=True)
+                return float(n * prefill_pairs(1, n_p, grp // 2) * v1_bwd_flops_per_pair(w.d, w.d))
+            out["v2_backward_bf16"]["cpu_baseline"] = dict(oracle_rate(
+                bwd_once, cpu_s, 1e12, "(batch, KV head) slices of the first 512 tokens"),
+                unit="TFLOP/s", cores=1)
         del q, k, v, dout, ws
         torch.cuda.empty_cache()
 
@@ -533,6 +663,21 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None):
                                         "ms": round(ms, 4),
                                         "frac": round(t / peaks["bf16_tflops"], 4),
                                         "flop": flop_att + flop_gemm, "d_model": dm}
+        if cpu_s > 0:  # every pair of random tokens, then the projection, in float64
+            P_ = w.Hq // 2
+            W_h = W.double().cpu().numpy()
+            rng = np.random.default_rng(19)
+
+            def proj_once(n):
+                toks = rng.integers(0, w.B * w.N, n)
+                rows = (toks[:, None] * P_ + np.arange(P_)[None, :]).reshape(-1)
+                o_h = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], rows, causal=True)
+                _ = o_h.reshape(n, P_ * w.d) @ W_h
+                return float(sum((int(t) % w.N + 1) * P_ * v2_flops_per_pair(w.d) for t in toks)
+                             + n * 2 * P_ * w.d * dm)
+            out["v2_prefill_oproj_bf16"]["cpu_baseline"] = dict(oracle_rate(
+                proj_once, cpu_s, 1e12, "random tokens, every pair and the projection"),
+                unit="TFLOP/s")
         del q, k, v, W, ws, o
         torch.cuda.empty_cache()
 
@@ -644,6 +789,9 @@ def main():
                     help="skip the secondary workloads (V2 prefill, long V1, decode, SNR sweep)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded host time for the oracle CPU baseline")
+    ap.add_argument("--extras-cpu-seconds", type=float, default=2.0,
+                    help="bounded host time of each secondary workload's oracle sample "
+                         "(0 skips them)")
     ap.add_argument("--only", default=None,
                     choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
                              "v1_decode_bf16", "snr_v1_decode", "v2_prefill_window_bf16",
@@ -660,8 +808,8 @@ def main():
         import torch
         torch.cuda.set_device(local_rank)
         peaks, peak_src = load_peaks()
-        print(json.dumps(run_extras(local_rank, peaks, peak_src, args.only, args.decode_batch)),
-              flush=True)
+        print(json.dumps(run_extras(local_rank, peaks, peak_src, args.only, args.decode_batch,
+                                    cpu_s=args.extras_cpu_seconds)), flush=True)
         return 0
 
     import torch
@@ -677,7 +825,7 @@ def main():
     res, x = run_headline(args, rank, world, local_rank, peaks, peak_src)
     extras = None
     if world == 1 and not args.no_extras:
-        extras = run_extras(local_rank, peaks, peak_src)
+        extras = run_extras(local_rank, peaks, peak_src, cpu_s=args.extras_cpu_seconds)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -13,9 +13,13 @@
 //
 // Set-up: the device address of the array is looked up with
 // cudaGetSymbolAddress the first time the entry point runs on a device (with
-// that device current) and cached per device; that first call should come
-// before any stream capture.  In host code the array's name is only a
-// host-side stand-in, so the kernels always receive the looked-up address.
+// that device current) and cached for that device and its current CUDA
+// context; that first call should come before any stream capture.  A call
+// made under another context of the same device (after cudaDeviceReset has
+// replaced the primary context, or under a context the caller created with
+// the driver API) looks the address up again for that context.  In host
+// code the array's name is only a host-side stand-in, so the kernels always
+// receive the looked-up address.
 // Shared state: every call on a device uses the same array and leaves its
 // contents behind.  Nothing in it has to start at zero (each partial the
 // combine step reads is written earlier in the same call), but calls whose
@@ -24,7 +28,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -39,27 +42,51 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-std::atomic<void*> g_scratch_addr[kMaxDevices];
+// The looked-up address of g_decode_scratch per device, with the CUDA
+// context it belongs to.
+struct ScratchEntry {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+ScratchEntry g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of g_decode_scratch on the current device (looked up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  return fn;
+}
+
+// Device address of g_decode_scratch in the current device's current context
+// (looked up on the first call in each context).
 int scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return DA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DA_ERR_UNSUPPORTED;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    p = g_scratch_addr[dev].load(std::memory_order_relaxed);
-    if (p == nullptr) {
-      void* addr = nullptr;
-      if (cudaGetSymbolAddress(&addr, g_decode_scratch) != cudaSuccess || addr == nullptr)
-        return DA_ERR_CUDA;
-      g_scratch_addr[dev].store(addr, std::memory_order_release);
-      p = addr;
-    }
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (!get_ctx) return DA_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return DA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchEntry& e = g_scratch[dev];
+  if (ctx == nullptr || e.ctx != ctx || e.addr == nullptr) {
+    // the lookup also binds the runtime's context to this thread if none was
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_decode_scratch) != cudaSuccess || addr == nullptr)
+      return DA_ERR_CUDA;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return DA_ERR_CUDA;
+    e.ctx = ctx;
+    e.addr = addr;
   }
-  *out = p;
+  *out = e.addr;
   return DA_OK;
 }
 

@@ -7,6 +7,9 @@ Tolerances (the operator's accuracy bounds):
   * bf16 outputs without the norm (V2, and V1 with the norm off): the same
     two bounds on |gpu - oracle| / max|oracle|.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -50,3 +53,14 @@ def status_word(device="cuda"):
 def assert_status_ok(st):
     torch.cuda.synchronize()
     assert int(st.item()) == 0, "device status %d" % int(st.item())
+
+
+def record(name: str, **fields):
+    """Append one JSON line about a parity check to the file named by the
+    DA_PARITY_REPORT environment variable (nothing if it is unset)."""
+    path = os.environ.get("DA_PARITY_REPORT")
+    if not path:
+        return
+    fields["name"] = name
+    with open(path, "a") as f:
+        f.write(json.dumps(fields) + "\n")

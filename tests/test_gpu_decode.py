@@ -1,7 +1,7 @@
 """GPU parity of single-token decode (V2 split-KV tensor-core kernel, V1
 split-KV CUDA-core kernel, and the generic kernel) against the fp64 oracle,
-including ragged cache lengths, several GQA group sizes, the full-size
-workloads on sampled batch entries, and decode == last row of prefill."""
+including ragged cache lengths, several GQA group sizes and decode == last
+row of prefill.  The full-size workloads are in test_gpu_full_size.py."""
 import numpy as np
 import pytest
 import torch
@@ -101,61 +101,6 @@ def test_decode_equals_last_prefill_row(B):
     assert_bf16_close(pre[0, n - 1], ref, True, "prefill last row")
     assert_bf16_close(dec[0], ref, True, "decode")
     assert_bf16_close(dec[0], pre[0, n - 1].float().cpu().double().numpy(), True, "dec vs pre")
-
-
-def _full_cache(shape_k, shape_v, seed, sampled, slice_fn):
-    """Device caches filled from a device generator, with the batch entries
-    the oracle reads overwritten by their CPU-generated slices."""
-    kc = torch.empty(shape_k, dtype=torch.bfloat16, device="cuda")
-    vc = torch.empty(shape_v, dtype=torch.bfloat16, device="cuda")
-    I.fill_normal_on_device(kc, seed * 2 + 1)
-    I.fill_normal_on_device(vc, seed * 2 + 2)
-    host = {}
-    for b in sampled:
-        k, v = slice_fn(b)
-        kc[b].copy_(k)
-        vc[b].copy_(v)
-        host[b] = (k, v)
-    return kc, vc, host
-
-
-def test_v2_decode_full_size_sampled(B):
-    w = I.WORKLOADS["v2_decode_bf16"]
-    x = I.v2_decode_inputs(w.B, w.L, w.Hq, w.Hkv, w.d, w.seed, fill_caches=False)
-    sampled = [0, w.B - 1]
-    kc, vc, host = _full_cache((w.B, w.L, w.Hkv, w.d), (w.B, w.L, w.Hkv, w.d), w.seed, sampled,
-                               lambda b: I.decode_cache_slice(w.seed, b, w.L, w.Hkv, w.d, w.d))
-    st = status_word()
-    out = B.diffattn_v2_decode(cuda(x["q"]), kc, vc, cuda(x["lam"]), dev_status=st)
-    assert_status_ok(st)
-    P = w.Hq // 2
-    for b in sampled:
-        k, v = host[b]
-        ref = O.v2_decode_rows(x["q"][b:b + 1], k[None], v[None], x["lam"], np.arange(P))
-        assert_bf16_close(out[b], ref, True, "v2 decode full b=%d" % b)
-    del kc, vc
-    torch.cuda.empty_cache()
-
-
-def test_v1_decode_full_size_sampled(B):
-    w = I.WORKLOADS["v1_decode_bf16"]
-    x = I.v1_decode_inputs(w.B, w.L, w.H, w.d, w.dv, w.seed, fill_caches=False)
-    sampled = [w.B // 2]
-    kc, vc, host = _full_cache((w.B, w.L, w.H, 2 * w.d), (w.B, w.L, w.H, w.dv), w.seed + 1,
-                               sampled,
-                               lambda b: I.decode_cache_slice(w.seed, b, w.L, w.H, 2 * w.d, w.dv))
-    lam_dev = B.lambda_from_params(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")), w.layer)
-    lam_host = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
-    li = O.lambda_init(w.layer)
-    out = B.diffattn_v1_decode(cuda(x["q"]), kc, vc, lam_dev, apply_norm=True, norm_eps=w.eps,
-                               lambda_init=li)
-    for b in sampled:
-        k, v = host[b]
-        ref = O.v1_decode_rows(x["q"][b:b + 1], k[None], v[None], lam_host, np.arange(w.H),
-                               apply_norm=True, eps=w.eps, lambda_init_value=li)
-        assert_bf16_close(out[b], ref, False, "v1 decode full b=%d" % b)
-    del kc, vc
-    torch.cuda.empty_cache()
 
 
 def test_v2_decode_large_logits_and_negative_lambda(B):
