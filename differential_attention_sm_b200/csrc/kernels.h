@@ -110,6 +110,12 @@ cudaError_t reset_tile_counters(cudaStream_t stream);
 cudaError_t hold_tile_counter(int slot, unsigned tag, unsigned count, cudaStream_t stream);
 cudaError_t keep_tile_counter(int slot, unsigned tag, unsigned duration_ms, cudaStream_t stream);
 
+// ---- tcgen05 bf16 GEMM (row-major C[M][N] = A[M][K] . B[K][N]) -------------
+// K and N multiples of 8, base addresses 16-byte aligned (TMA).
+int gemm_bf16_tc_smem_bytes();
+cudaError_t launch_gemm_bf16_tc(const void* a, const void* b, void* c, int M, int N, int K,
+                                int num_sms, int* dev_status, cudaStream_t stream);
+
 // ---- fused tcgen05 backward (bf16; V1 d_qk 64 / d_v 128, V2 head_dim 128) --
 struct FusedBwdArgs {
   PrefillArgs fwd;  // the forward's problem (out/lse/obr are set internally)

@@ -5,24 +5,20 @@
 // width back to Hq/2 heads x d, and the result then goes through O_W.
 // This entry point runs the differential-attention prefill into a
 // workspace and multiplies the [B*N, Hq/2*d] result by O_W [Hq/2*d, d_model]
-// with one plain GEMM (bf16 operands, fp32 accumulation, bf16 output).
-// A fused epilogue would need every one of a row's Hq/2 head pairs in one
-// CTA, or cross-CTA reductions of Hq/2 partial products per output element;
-// the separate GEMM reads the 2 x B x N x Hq/2 x d bytes of the finished
-// attention output once, which on this part costs far less.
-#include <cublas_v2.h>
+// with the library's tcgen05 GEMM (gemm_tc.cu: bf16 operands, fp32
+// accumulation, bf16 output).  A fused epilogue would need every one of a
+// row's Hq/2 head pairs in one CTA, or cross-CTA reductions of Hq/2 partial
+// products per output element; the separate GEMM reads the
+// 2 x B x N x Hq/2 x d bytes of the finished attention output once, which
+// on this part costs far less.
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "diffattn.h"
+#include "kernels.h"
 
 namespace {
-
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex[kMaxDevices];
-cublasHandle_t g_handle[kMaxDevices] = {};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -45,36 +41,27 @@ int diffattn_v2_prefill_oproj(const void* q, const void* k, const void* v, const
   if (d_model < 1 || batch < 1 || seqlen < 1 || n_q_heads < 2 || head_dim < 1)
     return DA_ERR_INVALID_ARG;
   if (dtype != DA_BF16) return DA_ERR_UNSUPPORTED;
+  const long long rows = (long long)batch * seqlen;
+  const long long kdim = (long long)(n_q_heads / 2) * head_dim;
+  // the GEMM's TMA row pitches must be multiples of 16 bytes
+  if (d_model % 8 != 0 || kdim % 8 != 0) return DA_ERR_UNSUPPORTED;
+  if (rows > 0x7fffffffLL || kdim > 0x7fffffffLL) return DA_ERR_UNSUPPORTED;
   if (!aligned16(w_o) || !aligned16(out)) return DA_ERR_ALIGNMENT;
   const size_t need = diffattn_v2_prefill_oproj_workspace_size(batch, seqlen, n_q_heads, head_dim);
   if (!workspace || workspace_bytes < need) return DA_ERR_WORKSPACE;
-  const long long rows = (long long)batch * seqlen;
-  const long long kdim = (long long)(n_q_heads / 2) * head_dim;
-  if (rows > 0x7fffffffLL || kdim > 0x7fffffffLL) return DA_ERR_UNSUPPORTED;
   void* o = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(workspace) + 255) &
                                     ~uintptr_t(255));
   int st = diffattn_v2_prefill_window(q, k, v, o, dtype, batch, seqlen, n_q_heads, n_kv_heads,
                                       head_dim, lambda, causal, window, dev_status, stream);
   if (st != DA_OK) return st;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mutex[dev]);
-  if (!g_handle[dev] && cublasCreate(&g_handle[dev]) != CUBLAS_STATUS_SUCCESS) {
-    g_handle[dev] = nullptr;
-    return DA_ERR_CUDA;
-  }
-  cublasHandle_t h = g_handle[dev];
-  if (cublasSetStream(h, static_cast<cudaStream_t>(stream)) != CUBLAS_STATUS_SUCCESS ||
-      cublasSetPointerMode(h, CUBLAS_POINTER_MODE_HOST) != CUBLAS_STATUS_SUCCESS)
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
     return DA_ERR_CUDA;
   // row-major out[rows x d_model] = o[rows x kdim] . W_o[kdim x d_model]
-  // (cuBLAS is column-major: out^T = W_o^T o^T)
-  const float one = 1.f, zero = 0.f;
-  if (cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, d_model, (int)rows, (int)kdim, &one, w_o,
-                   CUDA_R_16BF, d_model, o, CUDA_R_16BF, (int)kdim, &zero, out, CUDA_R_16BF,
-                   d_model, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-    return DA_ERR_CUDA;
-  return DA_OK;
+  cudaError_t e = da::launch_gemm_bf16_tc(o, w_o, out, (int)rows, d_model, (int)kdim, sms,
+                                          dev_status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : DA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -335,9 +335,11 @@ DA_API int lambda_from_params_bwd(const float* lq1, const float* lk1, const floa
  *   w_o : device [n_q_heads/2 * head_dim, d_model] bf16 (row-major)
  *   out : device [batch, seqlen, d_model] bf16
  * The attention output goes to `workspace` (size from the query), then one
- * plain GEMM (cuBLAS; bf16 operands, fp32 accumulation) writes `out`.  The
- * first call on a device creates that device's cuBLAS handle.  bf16 only.
- * Errors as for diffattn_v2_prefill_window, plus DA_ERR_WORKSPACE. */
+ * GEMM on the tcgen05 tensor cores (bf16 operands, fp32 accumulation, bf16
+ * result) writes `out`.  bf16 only; d_model and n_q_heads/2 * head_dim must
+ * be multiples of 8 (DA_ERR_UNSUPPORTED otherwise).  Errors as for
+ * diffattn_v2_prefill_window, plus DA_ERR_WORKSPACE.  `dev_status` also
+ * receives DA_ERR_DEVICE_TIMEOUT from the GEMM's bounded waits. */
 DA_API size_t diffattn_v2_prefill_oproj_workspace_size(int batch, int seqlen, int n_q_heads,
                                                        int head_dim);
 DA_API int diffattn_v2_prefill_oproj(const void* q, const void* k, const void* v,

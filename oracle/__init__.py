@@ -10,6 +10,7 @@ from .oracle import (  # noqa: F401
     lambda_from_params,
     v1_rows,
     v2_rows,
+    v2_oproj_rows,
     v2_decode_rows,
     v1_decode_rows,
     n_threads,

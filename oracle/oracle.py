@@ -201,6 +201,26 @@ def v2_rows(q, k, v, lam, rows, *, causal: bool, return_weights: bool = False,
     return _run_rows(call, rows, d, N if return_weights else None, threads)
 
 
+def v2_oproj_rows(q, k, v, lam, w_o, tokens, *, causal: bool, window: int = 0,
+                  threads: int | None = None):
+    """Output projection of the V2 prefill (lesson "Atencion Diferencial
+    (V2)", "V1 vs V2: la diferencia" and step 5 of "Implementacion": the
+    paired heads, Hq/2 of width d, go through O_W).  For each token
+    t = b*N + i of ``tokens``: its Hq/2 pair rows from ``v2_rows``, laid end
+    to end in pair order ([Hq/2 * d]), times w_o [Hq/2 * d, d_model], in
+    float64 (numpy matrix product).  Returns [len(tokens), d_model]."""
+    qf = _f32(q)
+    P = qf.shape[2] // 2
+    d = qf.shape[3]
+    t = np.asarray(tokens, dtype=np.int64).reshape(-1)
+    rows = (t[:, None] * P + np.arange(P)[None, :]).reshape(-1)
+    o = v2_rows(qf, k, v, lam, rows, causal=causal, window=window, threads=threads)
+    w = np.asarray(_f32(w_o), dtype=np.float64)
+    if w.shape[0] != P * d:
+        raise ValueError("w_o must have Hq/2 * head_dim rows")
+    return o.reshape(t.size, P * d) @ w
+
+
 def v2_decode_rows(q, k_cache, v_cache, lam, rows, *, lens=None, window: int = 0,
                    threads: int | None = None):
     """V2 decode rows r = b*(Hq/2) + p of out [B, Hq/2, d] (double).

@@ -219,6 +219,10 @@ def test_oproj_host_validation(lib):
     assert f(*bad) == b.DA_ERR_UNSUPPORTED
     bad = list(ok); bad[5] = U
     assert f(*bad) == b.DA_ERR_ALIGNMENT
+    bad = list(ok); bad[12] = 2044   # row pitch of the output not a multiple of 16 bytes
+    assert f(*bad) == b.DA_ERR_UNSUPPORTED
+    bad = list(ok); bad[11] = 100; bad[9] = 2   # Hq/2 * head_dim = 100
+    assert f(*bad) == b.DA_ERR_UNSUPPORTED
 
 
 def test_selftest_host_validation(lib):

@@ -576,3 +576,27 @@ def test_lambda_params_backward_matches_autograd():
     (lam * torch.tensor(dl)).sum().backward()
     for name, t in zip(("dlq1", "dlk1", "dlq2", "dlk2"), ts):
         assert np.abs(res[name] - t.grad.numpy()).max() < 1e-14, name
+
+
+def test_oproj_is_the_flattened_pairs_times_o_w():
+    """Output projection ([L] "V1 vs V2", step 5).  With O_W the identity the
+    result is each token's pair rows laid end to end in pair order; with a
+    0/1 matrix that picks feature sel[j] into column j, column j holds that
+    feature (a transposed O_W or another flattening order fails both)."""
+    Bn, N, Hq, Hkv, d = 2, 9, 6, 1, 4
+    x = I.v2_inputs(Bn, N, Hq, Hkv, d, seed=41, dtype=torch.float32)
+    P = Hq // 2
+    toks = np.array([0, 5, 9, 17])
+    rows = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], np.arange(Bn * N * P), causal=True)
+    per_tok = rows.reshape(Bn * N, P * d)
+    ident = np.eye(P * d, dtype=np.float32)
+    got = O.v2_oproj_rows(x["q"], x["k"], x["v"], x["lam"], ident, toks, causal=True)
+    np.testing.assert_allclose(got, per_tok[toks], rtol=0, atol=1e-15)
+    sel = np.random.default_rng(42).integers(0, P * d, 7)   # 7 output columns
+    pick = np.zeros((P * d, sel.size), dtype=np.float32)
+    pick[sel, np.arange(sel.size)] = 1.0
+    got = O.v2_oproj_rows(x["q"], x["k"], x["v"], x["lam"], pick, toks, causal=True)
+    for j, f in enumerate(sel):
+        p_, c_ = divmod(int(f), d)   # feature f = pair p_, channel c_
+        want = rows.reshape(Bn * N, P, d)[toks, p_, c_]
+        np.testing.assert_allclose(got[:, j], want, rtol=0, atol=1e-15)
