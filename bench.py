@@ -610,6 +610,46 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None, cpu_s=
         del q, k, v, dout, ws
         torch.cuda.empty_cache()
 
+    if want("v1_backward_saved_bf16"):  # V1 headline shape: training forward + backward from saves
+        w = wl("v1_prefill_bf16")
+        x = I.v1_inputs(w.B, w.N, w.H, w.d, w.dv, w.seed)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        dout = torch.randn(w.B, w.N, w.H, w.dv, device=dev).to(torch.bfloat16)
+        lamt = Bd.lambda_from_params(*(x[n].to(dev) for n in ("lq1", "lk1", "lq2", "lk2")),
+                                     w.layer)
+        li = Bd.diffattn_lambda_init(w.layer)
+        kw = dict(causal=True, apply_norm=True, norm_eps=w.eps, lambda_init=li)
+        o = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+        _, saves = Bd.diffattn_v1_fwd_train(q, k, v, lamt, out=o, **kw)
+        ws = torch.empty(Bd.load().diffattn_v1_bwd_saved_workspace_size(w.B, w.N, w.H),
+                         dtype=torch.uint8, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
+                 "dv": torch.empty(v.shape, **f32), "dlambda": torch.empty(w.H, **f32),
+                 "dnorm_weight": torch.empty(w.dv, **f32)}
+        ms_b = time_call(lambda: Bd.diffattn_v1_bwd_saved(q, k, v, dout, lamt, saves, workspace=ws,
+                                                          out=grads, **kw), 5, 2, stream)
+
+        def train_step():
+            Bd.diffattn_v1_fwd_train(q, k, v, lamt, out=o, saves=saves, **kw)
+            Bd.diffattn_v1_bwd_saved(q, k, v, dout, lamt, saves, workspace=ws, out=grads, **kw)
+        ms_t = time_call(train_step, 5, 2, stream)
+        pairs = prefill_pairs(w.B, w.N, w.H)
+        fb = pairs * v1_bwd_flops_per_pair(w.d, w.dv)
+        ft = pairs * (v1_flops_per_pair(w.d, w.dv) + v1_bwd_flops_per_pair(w.d, w.dv))
+        tb, tt = fb / (ms_b * 1e-3) / 1e12, ft / (ms_t * 1e-3) / 1e12
+        out["v1_backward_saved_bf16"] = {
+            "value": round(tb, 2), "unit": "TFLOP/s", "ms": round(ms_b, 4),
+            "frac": round(tb / peaks["bf16_tflops"], 4), "flop": fb,
+            "what": "backward from the training forward's saves (row kernel, dQ, dK/dV)"}
+        out["v1_train_step_bf16"] = {
+            "value": round(tt, 2), "unit": "TFLOP/s", "ms": round(ms_t, 4),
+            "frac": round(tt / peaks["bf16_tflops"], 4), "flop": ft,
+            "what": "training forward with saves + backward from the saves "
+                    "(768 + 1792 flop per visible pair)"}
+        del q, k, v, dout, ws, saves, grads, o
+        torch.cuda.empty_cache()
+
     if want("v2_backward_bf16"):  # gradients at the V2 prefill shape (B2 Hq32 Hkv8 N8192)
         w = wl("v2_prefill_bf16")
         x = I.v2_inputs(w.B, w.N, w.Hq, w.Hkv, w.d, w.seed)
@@ -796,6 +836,7 @@ def main():
                     choices=["v2_prefill_bf16", "v1_long_bf16", "v2_decode_bf16",
                              "v1_decode_bf16", "snr_v1_decode", "v2_prefill_window_bf16",
                              "v2_decode_window_bf16", "v1_backward_bf16",
+                             "v1_backward_saved_bf16",
                              "v2_backward_bf16", "v2_prefill_oproj_bf16"],
                     help="run just this secondary workload (one GPU) and print its numbers")
     ap.add_argument("--decode-batch", type=int, default=None,

@@ -48,6 +48,14 @@ EXPORTS = (
     "diffattn_v2_bwd_workspace_size",
     "diffattn_v2_bwd",
     "lambda_from_params_bwd",
+    "diffattn_v1_fwd_train_saves_size",
+    "diffattn_v1_fwd_train",
+    "diffattn_v1_bwd_saved_workspace_size",
+    "diffattn_v1_bwd_saved",
+    "diffattn_v2_prefill_train_saves_size",
+    "diffattn_v2_prefill_train",
+    "diffattn_v2_bwd_saved_workspace_size",
+    "diffattn_v2_bwd_saved",
     "diffattn_v2_prefill_oproj_workspace_size",
     "diffattn_v2_prefill_oproj",
     "diffattn_reset_tile_counters",
@@ -132,6 +140,23 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.lambda_from_params_bwd.restype = _i
     lib.lambda_from_params_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp,
                                            _vp]
+    for name in ("diffattn_v1_fwd_train_saves_size", "diffattn_v1_bwd_saved_workspace_size",
+                 "diffattn_v2_prefill_train_saves_size", "diffattn_v2_bwd_saved_workspace_size"):
+        getattr(lib, name).restype = _sz
+        getattr(lib, name).argtypes = [_i, _i, _i]
+    lib.diffattn_v1_fwd_train.restype = _i
+    lib.diffattn_v1_fwd_train.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i,
+                                          _i, _i, _vp, _f, _f, _vp, _sz, _vp, _vp]
+    lib.diffattn_v1_bwd_saved.restype = _i
+    lib.diffattn_v1_bwd_saved.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                          _i, _i, _vp, _f, _f, _vp, _sz, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _sz, _vp, _vp]
+    lib.diffattn_v2_prefill_train.restype = _i
+    lib.diffattn_v2_prefill_train.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp,
+                                              _i, _i, _vp, _sz, _vp, _vp]
+    lib.diffattn_v2_bwd_saved.restype = _i
+    lib.diffattn_v2_bwd_saved.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                          _i, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
     lib.diffattn_v2_prefill_oproj_workspace_size.restype = _sz
     lib.diffattn_v2_prefill_oproj_workspace_size.argtypes = [_i, _i, _i, _i]
     lib.diffattn_v2_prefill_oproj.restype = _i
@@ -436,6 +461,98 @@ def diffattn_v2_bwd(q, k, v, dout, lam, *, causal=True, window=0, workspace=None
         int(bool(causal)), int(window), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
         _ptr(res["dlambda"]), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(dev_status), _stream(stream)))
+    return res
+
+
+# ---- training forward with saves, and the backward from the saves ----------
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def diffattn_v1_fwd_train(q, k, v, lam, *, causal=True, window=0, apply_norm=False,
+                          norm_weight=None, norm_eps=1e-5, lambda_init=0.0, out=None,
+                          saves=None, dev_status=None, stream=None):
+    """V1 forward that also writes the saves the backward reads.  Returns
+    (out, saves); saves is a uint8 device tensor (allocated here if None)."""
+    _need_cuda(q, k, v, lam, norm_weight, dev_status)
+    B, N, H, d2 = q.shape
+    dvw = v.shape[-1]
+    if saves is None:
+        saves = torch.empty(int(load().diffattn_v1_fwd_train_saves_size(B, N, H)),
+                            dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty(B, N, H, dvw, dtype=q.dtype, device=q.device)
+    _check("diffattn_v1_fwd_train", load().diffattn_v1_fwd_train(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, N, H, d2 // 2, dvw, _ptr(lam),
+        int(bool(causal)), int(window), int(bool(apply_norm)), _ptr(norm_weight),
+        float(norm_eps), float(lambda_init), _ptr(saves), _nbytes(saves), _ptr(dev_status),
+        _stream(stream)))
+    return out, saves
+
+
+def diffattn_v1_bwd_saved(q, k, v, dout, lam, saves, *, causal=True, window=0,
+                          apply_norm=False, norm_weight=None, norm_eps=1e-5, lambda_init=0.0,
+                          workspace=None, out=None, dev_status=None, stream=None):
+    """V1 gradients from the saves of diffattn_v1_fwd_train (same dict as
+    diffattn_v1_bwd)."""
+    _need_cuda(q, k, v, dout, lam, saves, norm_weight)
+    B, N, H, d2 = q.shape
+    dvw = v.shape[-1]
+    if workspace is None:
+        workspace = torch.empty(int(load().diffattn_v1_bwd_saved_workspace_size(B, N, H)),
+                                dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
+           "dv": torch.empty(v.shape, **f32), "dlambda": torch.empty(H, **f32),
+           "dnorm_weight": torch.empty(dvw, **f32) if apply_norm else None}
+    res.update(out or {})
+    _check("diffattn_v1_bwd_saved", load().diffattn_v1_bwd_saved(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lam), _dtype_code(q), B, N, H, d2 // 2,
+        dvw, int(bool(causal)), int(window), int(bool(apply_norm)), _ptr(norm_weight),
+        float(norm_eps), float(lambda_init), _ptr(saves), _nbytes(saves), _ptr(res["dq"]),
+        _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dlambda"]), _ptr(res["dnorm_weight"]),
+        _ptr(workspace), _nbytes(workspace), _ptr(dev_status), _stream(stream)))
+    return res
+
+
+def diffattn_v2_prefill_train(q, k, v, lam, *, causal=True, window=0, out=None, saves=None,
+                              dev_status=None, stream=None):
+    """V2 prefill that also writes the saves the backward reads.  Returns
+    (out, saves)."""
+    _need_cuda(q, k, v, lam, dev_status)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if saves is None:
+        saves = torch.empty(int(load().diffattn_v2_prefill_train_saves_size(B, N, Hq)),
+                            dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty(B, N, Hq // 2, d, dtype=q.dtype, device=q.device)
+    _check("diffattn_v2_prefill_train", load().diffattn_v2_prefill_train(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, N, Hq, Hkv, d, _ptr(lam),
+        int(bool(causal)), int(window), _ptr(saves), _nbytes(saves), _ptr(dev_status),
+        _stream(stream)))
+    return out, saves
+
+
+def diffattn_v2_bwd_saved(q, k, v, dout, lam, saves, *, causal=True, window=0, workspace=None,
+                          out=None, dev_status=None, stream=None):
+    """V2 gradients from the saves of diffattn_v2_prefill_train (same dict
+    as diffattn_v2_bwd)."""
+    _need_cuda(q, k, v, dout, lam, saves)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if workspace is None:
+        workspace = torch.empty(int(load().diffattn_v2_bwd_saved_workspace_size(B, N, Hq)),
+                                dtype=torch.uint8, device=q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    res = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
+           "dv": torch.empty(v.shape, **f32), "dlambda": torch.empty(Hq // 2, **f32)}
+    res.update(out or {})
+    _check("diffattn_v2_bwd_saved", load().diffattn_v2_bwd_saved(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lam), _dtype_code(q), B, N, Hq, Hkv, d,
+        int(bool(causal)), int(window), _ptr(saves), _nbytes(saves), _ptr(res["dq"]),
+        _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dlambda"]), _ptr(workspace),
+        _nbytes(workspace), _ptr(dev_status), _stream(stream)))
     return res
 
 

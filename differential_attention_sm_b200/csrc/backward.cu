@@ -29,6 +29,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <initializer_list>
 #include <mutex>
 
 #include "diffattn.h"
@@ -610,6 +611,202 @@ int diffattn_v2_bwd(const void* q, const void* k, const void* v, const void* dou
                      static_cast<const __nv_bfloat16*>(dout), lambda, causal ? 1 : 0, window, 0,
                      nullptr, 0.f, 1.f, dq, dk, dv, dlambda, nullptr, workspace,
                      workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// ---- training forward with saves, and the backward from those saves -------
+namespace {
+
+da::PrefillArgs v1_fwd_args(int batch, int seqlen, int n_heads, int causal, int window,
+                            const float* lambda, int apply_norm, const float* norm_weight,
+                            float norm_eps, float lambda_init, int* dev_status) {
+  da::PrefillArgs f{};
+  f.form = 1;
+  f.batch = batch;
+  f.seqlen = seqlen;
+  f.heads = n_heads;
+  f.kv_heads = n_heads;
+  f.pairs_per_kv = 1;
+  f.causal = causal ? 1 : 0;
+  f.window = window;
+  f.lambda = lambda;
+  f.apply_norm = apply_norm ? 1 : 0;
+  f.norm_weight = norm_weight;
+  f.eps = norm_eps;
+  f.post_scale = 1.0f - lambda_init;
+  f.dev_status = dev_status;
+  return f;
+}
+
+da::PrefillArgs v2_fwd_args(int batch, int seqlen, int n_q_heads, int n_kv_heads, int causal,
+                            int window, const float* lambda, int* dev_status) {
+  da::PrefillArgs f{};
+  f.form = 2;
+  f.batch = batch;
+  f.seqlen = seqlen;
+  f.heads = n_q_heads / 2;
+  f.kv_heads = n_kv_heads;
+  f.pairs_per_kv = (n_q_heads / n_kv_heads) / 2;
+  f.causal = causal ? 1 : 0;
+  f.window = window;
+  f.lambda = lambda;
+  f.apply_norm = 0;
+  f.post_scale = 1.f;
+  f.dev_status = dev_status;
+  return f;
+}
+
+// Shared checks of the saved-state calls: sizes, masks, the tensor-core
+// widths, alignment.  Returns DA_OK or the status to return.
+int check_train(int batch, int seqlen, int units, int causal, int window, bool widths_ok,
+                std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs)
+    if (!q) return DA_ERR_INVALID_ARG;
+  if (batch < 1 || seqlen < 1 || units < 1) return DA_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && !causal)) return DA_ERR_INVALID_ARG;
+  if (!widths_ok) return DA_ERR_UNSUPPORTED;
+  if (!da::fits_int((long long)batch * seqlen) || (long long)seqlen * seqlen > (1LL << 31))
+    return DA_ERR_UNSUPPORTED;
+  for (const void* q : ptrs)
+    if (!da::aligned16(q)) return DA_ERR_ALIGNMENT;
+  return DA_OK;
+}
+
+}  // namespace
+
+size_t diffattn_v1_fwd_train_saves_size(int batch, int seqlen, int n_heads) {
+  if (batch < 1 || seqlen < 1 || n_heads < 1) return 0;
+  return da::train_saves_bytes(batch, seqlen, n_heads);
+}
+
+int diffattn_v1_fwd_train(const void* q, const void* k, const void* v, void* out,
+                          da_dtype dtype, int batch, int seqlen, int n_heads, int d_qk, int d_v,
+                          const float* lambda, int causal, int window, int apply_norm,
+                          const float* norm_weight, float norm_eps, float lambda_init,
+                          void* saves, size_t saves_bytes, int* dev_status, void* stream) {
+  if (apply_norm && !(norm_eps >= 0.f)) return DA_ERR_INVALID_ARG;
+  if (dtype != DA_BF16) return DA_ERR_UNSUPPORTED;
+  int rc = check_train(batch, seqlen, n_heads, causal, window, d_qk == 64 && d_v == 128,
+                       {q, k, v, out, lambda, saves});
+  if (rc != DA_OK) return rc;
+  if (saves_bytes < da::train_saves_bytes(batch, seqlen, n_heads)) return DA_ERR_WORKSPACE;
+  const int sms = da::sm_count();
+  if (sms < 1) return DA_ERR_CUDA;
+  return da::launch_fwd_train(v1_fwd_args(batch, seqlen, n_heads, causal, window, lambda,
+                                          apply_norm, norm_weight, norm_eps, lambda_init,
+                                          dev_status),
+                              q, k, v, out, saves, sms, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? DA_OK
+             : DA_ERR_CUDA;
+}
+
+size_t diffattn_v1_bwd_saved_workspace_size(int batch, int seqlen, int n_heads) {
+  if (batch < 1 || seqlen < 1 || n_heads < 1) return 0;
+  return da::saved_bwd_workspace_bytes(batch, seqlen, n_heads);
+}
+
+int diffattn_v1_bwd_saved(const void* q, const void* k, const void* v, const void* dout,
+                          const float* lambda, da_dtype dtype, int batch, int seqlen,
+                          int n_heads, int d_qk, int d_v, int causal, int window, int apply_norm,
+                          const float* norm_weight, float norm_eps, float lambda_init,
+                          const void* saves, size_t saves_bytes, float* dq, float* dk,
+                          float* dv, float* dlambda, float* dnorm_weight, void* workspace,
+                          size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!dq || !dk || !dv || !dlambda) return DA_ERR_INVALID_ARG;
+  if (apply_norm && !(norm_eps >= 0.f)) return DA_ERR_INVALID_ARG;
+  if (dtype != DA_BF16) return DA_ERR_UNSUPPORTED;
+  int rc = check_train(batch, seqlen, n_heads, causal, window, d_qk == 64 && d_v == 128,
+                       {q, k, v, dout, lambda, saves, workspace});
+  if (rc != DA_OK) return rc;
+  if (saves_bytes < da::train_saves_bytes(batch, seqlen, n_heads) ||
+      workspace_bytes < da::saved_bwd_workspace_bytes(batch, seqlen, n_heads))
+    return DA_ERR_WORKSPACE;
+  da::FusedBwdArgs a{};
+  a.fwd = v1_fwd_args(batch, seqlen, n_heads, causal, window, lambda, apply_norm, norm_weight,
+                      norm_eps, lambda_init, dev_status);
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dlambda = dlambda;
+  a.dg = apply_norm ? dnorm_weight : nullptr;
+  a.workspace = workspace;
+  a.num_sms = da::sm_count();
+  if (a.num_sms < 1) return DA_ERR_CUDA;
+  return da::launch_bwd_from_saves(a, saves, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DA_OK
+             : DA_ERR_CUDA;
+}
+
+size_t diffattn_v2_prefill_train_saves_size(int batch, int seqlen, int n_q_heads) {
+  if (batch < 1 || seqlen < 1 || n_q_heads < 2) return 0;
+  return da::train_saves_bytes(batch, seqlen, n_q_heads / 2);
+}
+
+int diffattn_v2_prefill_train(const void* q, const void* k, const void* v, void* out,
+                              da_dtype dtype, int batch, int seqlen, int n_q_heads,
+                              int n_kv_heads, int head_dim, const float* lambda, int causal,
+                              int window, void* saves, size_t saves_bytes, int* dev_status,
+                              void* stream) {
+  if (n_q_heads < 2 || n_kv_heads < 1 || n_q_heads % n_kv_heads != 0 ||
+      (n_q_heads / n_kv_heads) % 2 != 0)
+    return DA_ERR_INVALID_ARG;
+  if (dtype != DA_BF16) return DA_ERR_UNSUPPORTED;
+  int rc = check_train(batch, seqlen, n_q_heads / 2, causal, window, head_dim == 128,
+                       {q, k, v, out, lambda, saves});
+  if (rc != DA_OK) return rc;
+  if (saves_bytes < da::train_saves_bytes(batch, seqlen, n_q_heads / 2)) return DA_ERR_WORKSPACE;
+  const int sms = da::sm_count();
+  if (sms < 1) return DA_ERR_CUDA;
+  return da::launch_fwd_train(
+             v2_fwd_args(batch, seqlen, n_q_heads, n_kv_heads, causal, window, lambda,
+                         dev_status),
+             q, k, v, out, saves, sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DA_OK
+             : DA_ERR_CUDA;
+}
+
+size_t diffattn_v2_bwd_saved_workspace_size(int batch, int seqlen, int n_q_heads) {
+  if (batch < 1 || seqlen < 1 || n_q_heads < 2) return 0;
+  return da::saved_bwd_workspace_bytes(batch, seqlen, n_q_heads / 2);
+}
+
+int diffattn_v2_bwd_saved(const void* q, const void* k, const void* v, const void* dout,
+                          const float* lambda, da_dtype dtype, int batch, int seqlen,
+                          int n_q_heads, int n_kv_heads, int head_dim, int causal, int window,
+                          const void* saves, size_t saves_bytes, float* dq, float* dk,
+                          float* dv, float* dlambda, void* workspace, size_t workspace_bytes,
+                          int* dev_status, void* stream) {
+  if (!dq || !dk || !dv || !dlambda) return DA_ERR_INVALID_ARG;
+  if (n_q_heads < 2 || n_kv_heads < 1 || n_q_heads % n_kv_heads != 0 ||
+      (n_q_heads / n_kv_heads) % 2 != 0)
+    return DA_ERR_INVALID_ARG;
+  if (dtype != DA_BF16) return DA_ERR_UNSUPPORTED;
+  int rc = check_train(batch, seqlen, n_q_heads / 2, causal, window, head_dim == 128,
+                       {q, k, v, dout, lambda, saves, workspace});
+  if (rc != DA_OK) return rc;
+  if (saves_bytes < da::train_saves_bytes(batch, seqlen, n_q_heads / 2) ||
+      workspace_bytes < da::saved_bwd_workspace_bytes(batch, seqlen, n_q_heads / 2))
+    return DA_ERR_WORKSPACE;
+  da::FusedBwdArgs a{};
+  a.fwd = v2_fwd_args(batch, seqlen, n_q_heads, n_kv_heads, causal, window, lambda, dev_status);
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dlambda = dlambda;
+  a.workspace = workspace;
+  a.num_sms = da::sm_count();
+  if (a.num_sms < 1) return DA_ERR_CUDA;
+  return da::launch_bwd_from_saves(a, saves, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DA_OK
+             : DA_ERR_CUDA;
 }
 
 int lambda_from_params_bwd(const float* lq1, const float* lk1, const float* lq2,

@@ -22,9 +22,10 @@
 //     second S buffer, writes it to swizzled shared memory (SS MMA) so that
 //     S_r(j+1) only waits for S_r(j) to be loaded.  The softmax-backward
 //     warps form P as soon as S_r has landed and wait for dP_r only after
-//     that.  Warps: 0-3 / 4-7 branch 1 / 2 (thread = query row),
-//     8 TMA producer, 9-12 the S_r and dP_r issuers (one thread per product
-//     stream, as in the forward), 13 / 14 dQ issuers.
+//     that.  Warps: 0-15 softmax backward (thread = query row; two
+//     warpgroups per branch, one per half of the tile's 64 key columns),
+//     16 TMA producer, 17-20 the S_r and dP_r issuers (one thread per product
+//     stream, as in the forward), 21 / 22 dQ issuers.
 //   * dkdv kernel, one CTA per 128 keys of a head (V1) or KV head (V2),
 //     walking 64-query tiles (and, for V2, every pair that reads the KV
 //     head): S^T = K_r Q_r^T and dP^T = V do_r^T (SS), P^T and dS^T written
@@ -34,8 +35,9 @@
 //     halves of each step's handshake are separate: P^T is written (and the
 //     dV product released) as soon as S^T lands, dS^T once dP^T has; the
 //     next S^T into a buffer waits only for dV, the next dP^T only for dK.
-//     Warps: 0-3 / 4-7 alternate steps (= branches), 8 producer,
-//     9 S^T issuer, 10 dP^T issuer, 11 dV issuer, 12 dK issuer.
+//     Warps: 0-15 softmax backward (two warpgroups per step parity, one per
+//     half of the step's 64 query columns), 16 producer, 17 S^T issuer,
+//     18 dP^T issuer, 19 dV issuer, 20 dK issuer.
 // Every wait is bounded (DA_ERR_DEVICE_TIMEOUT in the status word).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -72,7 +74,11 @@ struct BwdParams {
 };
 
 // ===================================================================== dQ
-constexpr int kDqThreads = 480;
+// warps 0-15: softmax backward (branch r = (warp >> 2) & 1, key-column half
+// h = warp >> 3); 16 producer; 17-20 the S_r and dP_r issuers (17 owns tensor
+// memory); 21 / 22 the dQ_1 / dQ_2 issuers
+constexpr int kDqThreads = 736;
+constexpr int kDqProducer = 16;
 constexpr int kDqStages = 2;
 
 struct DqBarriers {
@@ -129,15 +135,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       mbar_init(&bars->s_full[r][0], 1);
       mbar_init(&bars->s_full[r][1], 1);
       mbar_init(&bars->dp_full[r], 1);
-      mbar_init(&bars->ds_full[r], 128);
+      mbar_init(&bars->ds_full[r], 256);  // both column halves
       mbar_init(&bars->dq_done[r][0], 1);
       mbar_init(&bars->dq_done[r][1], 1);
-      mbar_init(&bars->s_free[r], 128);
+      mbar_init(&bars->s_free[r], 256);
     }
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == kDqProducer + 1) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   auto colQ = [](int r) { return (uint32_t)(256 + D * r); };
   bool failed = false;
 
-  if (warp == 8) {
+  if (warp == kDqProducer) {
     if (lane == 0) {  // ---------------------------------------------- producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
@@ -192,9 +198,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tma_load_4d(sV + s * kTile64 + kBox64, &tm_v, &bars->v_full[s], 64, kvh, row, b);
       }
     }
-  } else if (warp >= 9 && warp <= 12) {
-    if (lane == 0) {  // ---- S_r issuer (kind 0) or dP_r issuer (kind 1): warp 9 + 2r + kind
-      const int r = (warp - 9) >> 1, kind = (warp - 9) & 1;
+  } else if (warp >= kDqProducer + 1 && warp <= kDqProducer + 4) {
+    if (lane == 0) {  // ---- S_r issuer (kind 0) or dP_r issuer (kind 1): warp 17 + 2r + kind
+      const int r = (warp - kDqProducer - 1) >> 1, kind = (warp - kDqProducer - 1) & 1;
       const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO) + r * kTile128;
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
@@ -248,9 +254,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
       }
     }
-  } else if (warp == 13 || warp == 14) {
-    if (lane == 0) {  // ------------------------------------ dQ_r issuer, r = warp - 13
-      const int r = warp - 13;
+  } else if (warp == kDqProducer + 5 || warp == kDqProducer + 6) {
+    if (lane == 0) {  // ------------------------------------ dQ_r issuer, r = warp - 21
+      const int r = warp - kDqProducer - 5;
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kDqStages;
@@ -260,8 +266,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tc_fence_after();
         const uint32_t kt = smem_u32(sK) + s * kTile64 + (kForm == 1 ? r * kBox64 : 0);
         for (int kk = 0; kk < 4; ++kk) {  // 16 keys per step; B = K_r, MN-major
+          // keys [32h, 32h + 32) of a tile are packed into columns [32h, 32h + 16)
+          // of the S buffer (each column half writes inside the columns it read)
           if (kForm == 1)  // A = dS_r in tensor memory
-            tc_mma_ts(tmem + colQ(r), tmem + colS(r, j) + kk * 8,
+            tc_mma_ts(tmem + colQ(r), tmem + colS(r, j) + 32 * (kk >> 1) + 8 * (kk & 1),
                       smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
                       (j > 0 || kk > 0) ? 1u : 0u);
           else  // A = dS_r in shared memory, K-major
@@ -275,8 +283,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------- softmax backward, branch r
-    const int r = warp / 4;
+    // ------------------------- softmax backward, branch r, key columns of half h
+    // Each tile's 64 key columns are split between two warpgroups per branch,
+    // which halves every thread's serial chain and gives each sub-partition
+    // four softmax warps to interleave.
+    const int r = (warp >> 2) & 1;
+    const int h = warp >> 3;
     const int row = (warp & 3) * 32 + lane;
     const int qrow = q0 + row;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -298,16 +310,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         break;
       }
       tc_fence_after();
-      const int k0 = (kv0 + j) * 64;
-      // tiles fully inside every row's visible range skip the masks
-      const bool full = __all_sync(0xffffffffu, k0 + 64 <= lim && (!kWindow || k0 >= lo));
-      uint32_t pp[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      const int k0 = (kv0 + j) * 64 + 32 * h;  // first key of this half
+      // halves fully inside every row's visible range skip the masks
+      const bool full = __all_sync(0xffffffffu, k0 + 32 <= lim && (!kWindow || k0 >= lo));
+      uint32_t pp[16];
+      {
         uint32_t sv[32];
-        tmem_ld32(tmem + lane_off + colS(r, j) + 32 * half, sv);
+        tmem_ld32(tmem + lane_off + colS(r, j) + 32 * h, sv);
         tc_wait_ld();
-        if (kForm == 2 && half == 1) {  // S_r fully loaded: its buffer may take S_r(j+1)
+        if (kForm == 2) {  // S_r fully loaded: its buffer may take S_r(j+1)
           tc_fence_before();
           mbar_arrive(&bars->s_free[r]);
         }
@@ -319,11 +330,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                    x0, x1);
           float p0 = ex2(x0), p1 = ex2(x1);
           if (!full) {
-            const int key = k0 + 32 * half + 2 * e;
+            const int key = k0 + 2 * e;
             p0 = (key < lim && (!kWindow || key >= lo)) ? p0 : 0.f;
             p1 = (key + 1 < lim && (!kWindow || key + 1 >= lo)) ? p1 : 0.f;
           }
-          pp[16 * half + e] = pack_bf16(p0, p1);
+          pp[e] = pack_bf16(p0, p1);
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full[r], (uint32_t)j & 1u, p.dev_status,
@@ -341,14 +352,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t dp[32], pk[16];
-        tmem_ld32(tmem + lane_off + colP(r) + 32 * half, dp);
+        tmem_ld32(tmem + lane_off + colP(r) + 32 * h, dp);
         tc_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const uint32_t pb = pp[16 * half + e];
+          const uint32_t pb = pp[e];
           float ds0, ds1;
           f2unpack(fma2(f2pack(bf16lo(pb), bf16hi(pb)),
                         add2(f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
@@ -358,14 +368,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           pk[e] = pack_bf16(ds0, ds1);
         }
         if (kForm == 1) {
-          tmem_st16(tmem + lane_off + colS(r, j) + 16 * half, pk);
+          tmem_st16(tmem + lane_off + colS(r, j) + 32 * h, pk);
         } else {
           // row `row` of the 128-byte-swizzled tile: 16-byte chunk c (8 keys)
           // sits at chunk position c ^ (row & 7)
           uint8_t* drow = sDS + r * kBox128 + row * 128;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
-            const int ch = 4 * half + c4;
+            const int ch = 4 * h + c4;
             *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
                 make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
           }
@@ -383,13 +393,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 p.dev_status, &failed);
     tc_fence_after();
     const bool store = qrow < p.seqlen;
-    float* dst = kForm == 1
-                     ? p.dq + (((size_t)b * p.seqlen + qrow) * p.q_heads + hh) * 128 + 64 * r
-                     : p.dq + (((size_t)b * p.seqlen + qrow) * p.q_heads + 2 * hh + r) * 128;
+    // each half writes half of this branch's dQ_r columns
+    float* dst = (kForm == 1
+                      ? p.dq + (((size_t)b * p.seqlen + qrow) * p.q_heads + hh) * 128 + 64 * r
+                      : p.dq + (((size_t)b * p.seqlen + qrow) * p.q_heads + 2 * hh + r) * 128) +
+                 (D / 2) * h;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       uint32_t v[32];
-      tmem_ld32(tmem + lane_off + colQ(r) + 32 * c, v);
+      tmem_ld32(tmem + lane_off + colQ(r) + (D / 2) * h + 32 * c, v);
       tc_wait_ld();
       if (store && !bars->abort_flag) {
 #pragma unroll
@@ -407,14 +419,18 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kDqProducer + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
 // =================================================================== dK, dV
-constexpr int kKvThreads = 416;
+// warps 0-15: softmax backward (step parity w = (warp >> 2) & 1, query-column
+// half h = warp >> 3); 16 producer; 17 S^T issuer (owns tensor memory);
+// 18 dP^T issuer; 19 dV issuer; 20 dK issuer
+constexpr int kKvThreads = 672;
+constexpr int kKvProducer = 16;
 constexpr int kKvStages = 3;
 constexpr int kStageQ = kTile64;                       // Q_r tile (V1 uses one box)
 // + dO_r tile + lse/D vectors; a multiple of 1 KB keeps every stage's
@@ -470,8 +486,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
       mbar_init(&bars->dp_full[w], 1);
-      mbar_init(&bars->p_full[w], 128);
-      mbar_init(&bars->ds_full[w], 128);
+      mbar_init(&bars->p_full[w], 256);   // both column halves
+      mbar_init(&bars->ds_full[w], 256);
       mbar_init(&bars->pt_free[w], 1);
       mbar_init(&bars->dst_free[w], 1);
     }
@@ -479,7 +495,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == kKvProducer + 1) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -496,7 +512,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     return kForm == 1 ? g : g * p.pairs_per_kv + (s >> 1) % members;
   };
 
-  if (warp == 8) {
+  if (warp == kKvProducer) {
     if (lane == 0) {  // ---------------------------------------------- producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
@@ -529,9 +545,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         bulk_load(svec + 64, p.Dv + vrow, 256, &bars->qd_full[st]);
       }
     }
-  } else if (warp == 9 || warp == 10) {
-    if (lane == 0) {  // ------------------ S^T issuer (warp 9) and dP^T issuer (warp 10)
-      const bool is_s = warp == 9;
+  } else if (warp == kKvProducer + 1 || warp == kKvProducer + 2) {
+    if (lane == 0) {  // -------------------------------------- S^T issuer and dP^T issuer
+      const bool is_s = warp == kKvProducer + 1;
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       if (mbar_wait(&bars->kv_full, 0, p.dev_status, &failed)) {
@@ -573,10 +589,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
       }
     }
-  } else if (warp == 11 || warp == 12) {
-    if (lane == 0) {  // -------------- dV issuer (warp 11) and dK issuer (warp 12)
+  } else if (warp == kKvProducer + 3 || warp == kKvProducer + 4) {
+    if (lane == 0) {  // ---------------------------------------- dV issuer and dK issuer
       // each accumulator has one issuing thread, so its order is fixed
-      const bool is_v = warp == 11;
+      const bool is_v = warp == kKvProducer + 3;
       constexpr uint32_t idV = idesc_bf16_f32(128, 128, false, true);
       constexpr uint32_t idK = idesc_bf16_f32(128, D, false, true);
       bool first[2] = {true, true};
@@ -590,11 +606,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const int fb = (is_v || kForm == 2) ? 0 : r;  // accumulator of this step
         for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step; B operands MN-major
           const uint32_t acc = (first[fb] && kk == 0) ? 0u : 1u;
+          // queries [32h, 32h + 32) of a step are packed into columns [32h, 32h + 16)
+          // of their buffer (each column half writes inside the columns it read)
+          const uint32_t pc = 32u * (uint32_t)(kk >> 1) + 8u * (uint32_t)(kk & 1);
           if (is_v)
-            tc_mma_ts(tmem + kColDV, tmem + 128 * w + kk * 8,
+            tc_mma_ts(tmem + kColDV, tmem + 128 * w + pc,
                       smem_desc_sw128(sdo + kk * 2048, kBox64, 1024), idV, acc);
           else
-            tc_mma_ts(tmem + kColDK + (kForm == 1 ? 64 * r : 0), tmem + 128 * w + 64 + kk * 8,
+            tc_mma_ts(tmem + kColDK + (kForm == 1 ? 64 * r : 0), tmem + 128 * w + 64 + pc,
                       smem_desc_sw128(sq + kk * 2048, kBox64, 1024), idK, acc);
         }
         first[fb] = false;
@@ -604,16 +623,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc_commit(&bars->acc_done);
     }
   } else {
-    // --------------------------------- softmax backward, steps of parity w
+    // ------------------ softmax backward, steps of parity w, query columns of half h
     // Two passes per step.  P = 2^(s sc - lse) goes out as soon as S^T has
     // landed, so the dV product starts (and frees the S^T buffer for step
     // s + 2) while dP^T may still be in flight; dS = P (dP - D) follows from
-    // the same bf16 P, kept in registers.
-    const int w = warp / 4;
+    // the same bf16 P, kept in registers.  Each step's 64 query columns are
+    // split between two warpgroups, which halves every thread's serial chain
+    // and gives each sub-partition four softmax warps to interleave.
+    const int w = (warp >> 2) & 1;
+    const int h = warp >> 3;
     const int krow = (warp & 3) * 32 + lane;
     const int key = k0 + krow;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + 128 * w, t_dp = t_s + 64;
+    const uint32_t t_s = tmem + lane_off + 128 * w + 32 * h, t_dp = t_s + 64;
     const float sc = p.scale_log2;
     for (int s = w; s < n_steps; s += 2) {
       const int st = s % kKvStages;
@@ -628,23 +650,25 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       tc_fence_after();
       const int q0 = step_q0(s);
       const float* svec =
-          reinterpret_cast<const float*>(sStage + st * kStageBytes + kStageQ + kTile64);
-      // query columns this key row sees in the step: [c_lo, c_hi)
+          reinterpret_cast<const float*>(sStage + st * kStageBytes + kStageQ + kTile64) + 32 * h;
+      // query columns this key row sees in the step: [c_lo, c_hi), relative
+      // to this half's first column
       int c_lo = 0, c_hi = min(64, p.seqlen - q0);
       if (key >= p.seqlen) c_hi = 0;
       if (p.causal) c_lo = max(0, key - q0);
       if (kWindow) c_hi = min(c_hi, key + p.window - q0);
-      const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == 64);
+      c_lo -= 32 * h;
+      c_hi -= 32 * h;
+      const bool full = __all_sync(0xffffffffu, c_lo <= 0 && c_hi >= 32);
       const uint64_t sc2 = f2pack(sc, sc);
-      uint32_t pp[32];  // P row as packed bf16 pairs
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      uint32_t pp[16];  // P row (32 queries) as packed bf16 pairs
+      {
         uint32_t sv[32];
-        tmem_ld32(t_s + 32 * half, sv);
+        tmem_ld32(t_s, sv);
         tc_wait_ld();
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {  // 4 query columns: lse by a broadcast load
-          const int c = 32 * half + 4 * e4;
+          const int c = 4 * e4;
           const float4 L = *reinterpret_cast<const float4*>(svec + c);
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
@@ -660,11 +684,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
               p0 = (cc >= c_lo && cc < c_hi) ? p0 : 0.f;
               p1 = (cc + 1 >= c_lo && cc + 1 < c_hi) ? p1 : 0.f;
             }
-            pp[16 * half + e] = pack_bf16(p0, p1);
+            pp[e] = pack_bf16(p0, p1);
           }
         }
-        // P^T over the first 32 columns of S^T (this half's S is already read)
-        tmem_st16(t_s + 16 * half, *reinterpret_cast<uint32_t(*)[16]>(pp + 16 * half));
+        // P^T over the first 16 of the 32 columns this half has read
+        tmem_st16(t_s, pp);
       }
       tc_wait_st();
       tc_fence_before();
@@ -675,20 +699,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t dp[32], pd[16];
-        tmem_ld32(t_dp + 32 * half, dp);
+        tmem_ld32(t_dp, dp);
         tc_wait_ld();
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {  // D by a broadcast load
-          const int c = 32 * half + 4 * e4;
+          const int c = 4 * e4;
           const float4 Dd = *reinterpret_cast<const float4*>(svec + 64 + c);
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int e = 2 * e4 + h2;
             const float d0 = h2 ? Dd.z : Dd.x, d1 = h2 ? Dd.w : Dd.y;
-            const uint32_t pb = pp[16 * half + e];
+            const uint32_t pb = pp[e];
             const uint64_t pr = f2pack(bf16lo(pb), bf16hi(pb));
             const uint64_t dd = add2(
                 f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
@@ -698,7 +721,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             pd[e] = pack_bf16(ds0, ds1);
           }
         }
-        tmem_st16(t_dp + 16 * half, pd);
+        tmem_st16(t_dp, pd);
       }
       tc_wait_st();
       tc_fence_before();
@@ -708,14 +731,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (failed) bars->abort_flag = 1;
     mbar_wait(&bars->acc_done, 0, p.dev_status, &failed);
     tc_fence_after();
-    asm volatile("bar.sync 2, 256;" ::: "memory");
+    asm volatile("bar.sync 2, 512;" ::: "memory");
     const bool store = key < p.seqlen && !bars->abort_flag;
-    // warpgroup 0 writes dV, warpgroup 1 writes dK (scaled by 1/sqrt(d))
-    float* dst = (w == 0 ? p.dv : p.dk) + (((size_t)b * p.seqlen + key) * p.kv_heads + g) * 128;
-    const uint32_t col = w == 0 ? kColDV : kColDK;
+    // warpgroups of w = 0 write dV, of w = 1 dK (scaled by 1/sqrt(d)), columns [64h, 64h + 64)
+    float* dst = (w == 0 ? p.dv : p.dk) + (((size_t)b * p.seqlen + key) * p.kv_heads + g) * 128 +
+                 64 * h;
+    const uint32_t col = (w == 0 ? kColDV : kColDK) + 64u * (uint32_t)h;
     const float mul = w == 0 ? 1.f : p.scale;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       uint32_t v[32];
       tmem_ld32(tmem + lane_off + col + 32 * c, v);
       tc_wait_ld();
@@ -735,7 +759,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kKvProducer + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -852,33 +876,83 @@ __global__ void __launch_bounds__(32 * kPreWarps) bwd_pre2_kernel(Pre2Args a) {
 
 }  // namespace
 
-size_t fused_bwd_workspace_bytes(int batch, int seqlen, int units) {
+// Saves of the training forward: per-row log2-sum-exp of each branch
+// (fp32 [B][units][2][npad], padding zero) and each branch's normalised output
+// O_r / l_r (bf16 [B][N][units][2][128]).
+struct SavesLayout {
+  size_t lse_bytes, obr_bytes;
+};
+
+SavesLayout saves_layout(int batch, int seqlen, int units) {
   const size_t npad = (size_t)((seqlen + 63) / 64) * 64;
-  const size_t vec = (size_t)batch * units * 2 * npad * 4;
-  const size_t big = (size_t)batch * seqlen * units * 256 * 2;
+  SavesLayout L;
+  L.lse_bytes = ((size_t)batch * units * 2 * npad * 4 + 255) & ~size_t(255);
+  L.obr_bytes = ((size_t)batch * seqlen * units * 256 * 2 + 255) & ~size_t(255);
+  return L;
+}
+
+size_t train_saves_bytes(int batch, int seqlen, int units) {
+  const SavesLayout L = saves_layout(batch, seqlen, units);
+  return L.lse_bytes + L.obr_bytes + 256;
+}
+
+size_t saved_bwd_workspace_bytes(int batch, int seqlen, int units) {
+  // D_r (as lse) and the per-branch upstream gradients (as the branch outputs)
+  return train_saves_bytes(batch, seqlen, units);
+}
+
+size_t fused_bwd_workspace_bytes(int batch, int seqlen, int units) {
   const size_t out = (size_t)batch * seqlen * units * 128 * 2;
-  return 2 * ((vec + 255) & ~size_t(255)) + 2 * ((big + 255) & ~size_t(255)) +
+  // + 256: the workspace's own start is rounded up to 256 bytes
+  return train_saves_bytes(batch, seqlen, units) + saved_bwd_workspace_bytes(batch, seqlen, units) +
          ((out + 255) & ~size_t(255)) + 256;
 }
 
-cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
+namespace {
+uint8_t* align256(void* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 255) & ~uintptr_t(255));
+}
+}  // namespace
+
+cudaError_t launch_fwd_train(const PrefillArgs& fwd, const void* q, const void* k,
+                             const void* v, void* out, void* saves, int num_sms,
+                             cudaStream_t st) {
+  const int B = fwd.batch, N = fwd.seqlen, U = fwd.heads;
+  const int npad = (N + 63) / 64 * 64;
+  const SavesLayout L = saves_layout(B, N, U);
+  uint8_t* base = align256(saves);
+  float* lse = reinterpret_cast<float*>(base);
+  void* obr = base + L.lse_bytes;
+  const int qh = fwd.form == 1 ? U : 2 * U, kvh = fwd.kv_heads;
+  CUtensorMap tq128, tk64, tv64;
+  if (make_tmap_bf16_4d(&tq128, q, 128, qh, N, B, 64, 1, 128, 1) ||
+      make_tmap_bf16_4d(&tk64, k, 128, kvh, N, B, 64, 1, 64, 1) ||
+      make_tmap_bf16_4d(&tv64, v, 128, kvh, N, B, 64, 1, 64, 1))
+    return cudaErrorInvalidValue;
+  // lse rows are read in 64-entry blocks, so the padding is zeroed first
+  cudaError_t e = cudaMemsetAsync(lse, 0, (size_t)B * U * 2 * npad * 4, st);
+  if (e != cudaSuccess) return e;
+  PrefillArgs fa = fwd;
+  fa.out = out;
+  fa.lse = lse;
+  fa.lse_stride = npad;
+  fa.obr = obr;
+  return launch_prefill_tc(tq128, tk64, tv64, fa, num_sms, st);
+}
+
+cudaError_t launch_bwd_from_saves(const FusedBwdArgs& a, const void* saves, cudaStream_t st) {
   const int B = a.fwd.batch, N = a.fwd.seqlen, U = a.fwd.heads;
   const int npad = (N + 63) / 64 * 64;
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(a.workspace) + 255) & ~uintptr_t(255));
-  auto take = [&](size_t bytes) {
-    uint8_t* p = base;
-    base += (bytes + 255) & ~size_t(255);
-    return p;
-  };
-  float* lse = reinterpret_cast<float*>(take((size_t)B * U * 2 * npad * 4));
-  float* Dv = reinterpret_cast<float*>(take((size_t)B * U * 2 * npad * 4));
-  __nv_bfloat16* obr = reinterpret_cast<__nv_bfloat16*>(take((size_t)B * N * U * 256 * 2));
-  __nv_bfloat16* dob = reinterpret_cast<__nv_bfloat16*>(take((size_t)B * N * U * 256 * 2));
-  void* fwd_out = take((size_t)B * N * U * 128 * 2);
+  const SavesLayout L = saves_layout(B, N, U);
+  const uint8_t* sv = align256(const_cast<void*>(saves));
+  const float* lse = reinterpret_cast<const float*>(sv);
+  const __nv_bfloat16* obr = reinterpret_cast<const __nv_bfloat16*>(sv + L.lse_bytes);
+  uint8_t* wb = align256(a.workspace);
+  float* Dv = reinterpret_cast<float*>(wb);
+  __nv_bfloat16* dob = reinterpret_cast<__nv_bfloat16*>(wb + L.lse_bytes);
 
   // tensor maps: inputs as [B][N][heads][128] with 64-column boxes of 128
-  // or 64 rows, and the saved upstream gradients [B][N][2U][128]
+  // or 64 rows, and the per-branch upstream gradients [B][N][2U][128]
   const int qh = a.fwd.form == 1 ? U : 2 * U, kvh = a.fwd.kv_heads;
   CUtensorMap tq128, tq64, tk64, tk128, tv64, tv128, tdo128, tdo64;
   if (make_tmap_bf16_4d(&tq128, a.q, 128, qh, N, B, 64, 1, 128, 1) ||
@@ -890,18 +964,8 @@ cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
       make_tmap_bf16_4d(&tdo128, dob, 128, 2 * U, N, B, 64, 1, 128, 1) ||
       make_tmap_bf16_4d(&tdo64, dob, 128, 2 * U, N, B, 64, 1, 64, 1))
     return cudaErrorInvalidValue;
-  // 1. training forward: lse and the normalised branch outputs (lse rows are
-  // read in 64-entry blocks, so the padding is zeroed first)
-  cudaError_t e = cudaMemsetAsync(lse, 0, (size_t)B * U * 2 * npad * 4, st);
-  if (e != cudaSuccess) return e;
-  PrefillArgs fa = a.fwd;
-  fa.out = fwd_out;
-  fa.lse = lse;
-  fa.lse_stride = npad;
-  fa.obr = obr;
-  e = launch_prefill_tc(tq128, tk64, tv64, fa, a.num_sms, st);
-  if (e != cudaSuccess) return e;
-  // 2. upstream gradients per branch, D, dlambda, gain gradient
+  // upstream gradients per branch, D, dlambda, gain gradient
+  cudaError_t e;
   if ((e = cudaMemsetAsync(Dv, 0, (size_t)B * U * 2 * npad * 4, st)) != cudaSuccess ||
       (e = cudaMemsetAsync(a.dlambda, 0, (size_t)U * 4, st)) != cudaSuccess ||
       (a.dg && (e = cudaMemsetAsync(a.dg, 0, 128 * 4, st)) != cudaSuccess))
@@ -946,7 +1010,7 @@ cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
   p.n_ktiles = (N + 127) / 128;
   p.dev_status = a.fwd.dev_status;
   const bool win = a.fwd.window > 0;
-  // 4. dQ
+  // dQ
   {
     const int qbytes = a.fwd.form == 1 ? kTile128 : 2 * kTile128;
     const int smem = 1024 + qbytes + 2 * kTile128 + 2 * kDqStages * kTile64 +
@@ -960,7 +1024,7 @@ cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
     k<<<p.n_qtiles * B * U, kDqThreads, smem, st>>>(tq128, tdo128, tk64, tv64, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // 5. dK, dV
+  // dK, dV
   {
     const int smem = 1024 + 2 * kTile128 + kKvStages * kStageBytes + (int)sizeof(KvBarriers) + 64;
     decltype(&diffattn_bwd_dkdv_kernel<1, false>) k =
@@ -974,6 +1038,19 @@ cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t st) {
+  // workspace: [saves of the training forward][backward workspace][forward output]
+  const int B = a.fwd.batch, N = a.fwd.seqlen, U = a.fwd.heads;
+  uint8_t* base = align256(a.workspace);
+  const size_t saves = train_saves_bytes(B, N, U), bwd = saved_bwd_workspace_bytes(B, N, U);
+  void* fwd_out = base + saves + bwd;
+  cudaError_t e = launch_fwd_train(a.fwd, a.q, a.k, a.v, fwd_out, base, a.num_sms, st);
+  if (e != cudaSuccess) return e;
+  FusedBwdArgs b = a;
+  b.workspace = base + saves;
+  return launch_bwd_from_saves(b, base, st);
 }
 
 }  // namespace da

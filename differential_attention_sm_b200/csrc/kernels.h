@@ -133,5 +133,15 @@ struct FusedBwdArgs {
 };
 size_t fused_bwd_workspace_bytes(int batch, int seqlen, int units);
 cudaError_t launch_fused_bwd(const FusedBwdArgs& a, cudaStream_t stream);
+// The same split in two: the training forward (the prefill kernel writing
+// `out` and the saves) and the backward from those saves (a.workspace holds
+// saved_bwd_workspace_bytes).  units = heads (V1) or pairs (V2).
+size_t train_saves_bytes(int batch, int seqlen, int units);
+size_t saved_bwd_workspace_bytes(int batch, int seqlen, int units);
+cudaError_t launch_fwd_train(const PrefillArgs& fwd, const void* q, const void* k,
+                             const void* v, void* out, void* saves, int num_sms,
+                             cudaStream_t stream);
+cudaError_t launch_bwd_from_saves(const FusedBwdArgs& a, const void* saves,
+                                  cudaStream_t stream);
 
 }  // namespace da

@@ -317,6 +317,56 @@ DA_API int diffattn_v2_bwd(const void* q, const void* k, const void* v, const vo
                            float* dq, float* dk, float* dv, float* dlambda, void* workspace,
                            size_t workspace_bytes, int* dev_status, void* stream);
 
+/* ---- Training forward with saves, and the backward from the saves --------
+ * A training step runs the forward once for its output and then the
+ * backward.  diffattn_v1_bwd / diffattn_v2_bwd above take no forward state
+ * and so run the training forward again internally.  These calls split that
+ * work: the *_train forward writes the output exactly as diffattn_v1_fwd /
+ * diffattn_v2_prefill_window do, plus the saves the backward reads; the
+ * *_bwd_saved backward takes those saves and computes the same gradients as
+ * diffattn_v1_bwd / diffattn_v2_bwd.  (The pages give the forward only; the
+ * gradients are its chain rule, as above.)
+ *  - Supported: bf16 with the tensor-core widths (V1 d_qk 64, d_v 128; V2
+ *    head_dim 128); else DA_ERR_UNSUPPORTED.
+ *  - saves: caller-owned device memory of at least the *_saves_size bytes
+ *    (contents: per-row log2-sum-exp of each branch, fp32, and each branch's
+ *    normalised output O_r / l_r, bf16; any alignment).  The backward must
+ *    get the same q, k, v, lambda, causal, window and norm arguments as the
+ *    forward that wrote the saves; the saves are only read by it.
+ *  - workspace of the backward: at least the *_bwd_saved_workspace_size
+ *    bytes, scratch (contents undefined after the call).
+ *  - Errors as for the forward and backward above, plus DA_ERR_WORKSPACE for
+ *    short saves or workspace. */
+DA_API size_t diffattn_v1_fwd_train_saves_size(int batch, int seqlen, int n_heads);
+DA_API int diffattn_v1_fwd_train(const void* q, const void* k, const void* v, void* out,
+                                 da_dtype dtype, int batch, int seqlen, int n_heads, int d_qk,
+                                 int d_v, const float* lambda, int causal, int window,
+                                 int apply_norm, const float* norm_weight, float norm_eps,
+                                 float lambda_init, void* saves, size_t saves_bytes,
+                                 int* dev_status, void* stream);
+DA_API size_t diffattn_v1_bwd_saved_workspace_size(int batch, int seqlen, int n_heads);
+DA_API int diffattn_v1_bwd_saved(const void* q, const void* k, const void* v, const void* dout,
+                                 const float* lambda, da_dtype dtype, int batch, int seqlen,
+                                 int n_heads, int d_qk, int d_v, int causal, int window,
+                                 int apply_norm, const float* norm_weight, float norm_eps,
+                                 float lambda_init, const void* saves, size_t saves_bytes,
+                                 float* dq, float* dk, float* dv, float* dlambda,
+                                 float* dnorm_weight, void* workspace, size_t workspace_bytes,
+                                 int* dev_status, void* stream);
+DA_API size_t diffattn_v2_prefill_train_saves_size(int batch, int seqlen, int n_q_heads);
+DA_API int diffattn_v2_prefill_train(const void* q, const void* k, const void* v, void* out,
+                                     da_dtype dtype, int batch, int seqlen, int n_q_heads,
+                                     int n_kv_heads, int head_dim, const float* lambda,
+                                     int causal, int window, void* saves, size_t saves_bytes,
+                                     int* dev_status, void* stream);
+DA_API size_t diffattn_v2_bwd_saved_workspace_size(int batch, int seqlen, int n_q_heads);
+DA_API int diffattn_v2_bwd_saved(const void* q, const void* k, const void* v, const void* dout,
+                                 const float* lambda, da_dtype dtype, int batch, int seqlen,
+                                 int n_q_heads, int n_kv_heads, int head_dim, int causal,
+                                 int window, const void* saves, size_t saves_bytes, float* dq,
+                                 float* dk, float* dv, float* dlambda, void* workspace,
+                                 size_t workspace_bytes, int* dev_status, void* stream);
+
 /* Gradients of the four lambda vectors (device fp32 [n_heads, dim]) of
  * lambda_from_params, from dlambda [n_heads]:
  *   dlq1 = dlambda e^{lq1.lk1} lk1,  dlk1 = dlambda e^{lq1.lk1} lq1,

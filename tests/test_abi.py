@@ -225,6 +225,47 @@ def test_oproj_host_validation(lib):
     assert f(*bad) == b.DA_ERR_UNSUPPORTED
 
 
+def test_saved_state_host_validation(lib):
+    from differential_attention_sm_b200 import binding as b
+    sz = b.load().diffattn_v1_fwd_train_saves_size(2, 300, 3)
+    assert sz >= 2 * 3 * 2 * 320 * 4 + 2 * 300 * 3 * 256 * 2
+    assert b.load().diffattn_v1_fwd_train_saves_size(0, 300, 3) == 0
+    f = lib.diffattn_v1_fwd_train
+    ok = [A, A, A, A, b.DA_BF16, 2, 300, 3, 64, 128, A, 1, 0, 1, None, 1e-5, 0.2, A, sz, None,
+          None]
+    bad = list(ok); bad[18] = sz - 1
+    assert f(*bad) == b.DA_ERR_WORKSPACE
+    bad = list(ok); bad[8] = 32                     # not the tensor-core widths
+    assert f(*bad) == b.DA_ERR_UNSUPPORTED
+    bad = list(ok); bad[17] = U
+    assert f(*bad) == b.DA_ERR_ALIGNMENT
+    bad = list(ok); bad[12] = 5; bad[11] = 0        # window without causal
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    ws = b.load().diffattn_v1_bwd_saved_workspace_size(2, 300, 3)
+    g = lib.diffattn_v1_bwd_saved
+    ok = [A, A, A, A, A, b.DA_BF16, 2, 300, 3, 64, 128, 1, 0, 1, None, 1e-5, 0.2, A, sz, A, A, A,
+          A, A, A, ws, None, None]
+    bad = list(ok); bad[25] = ws - 1
+    assert g(*bad) == b.DA_ERR_WORKSPACE
+    bad = list(ok); bad[19] = None
+    assert g(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(ok); bad[5] = b.DA_FP32
+    assert g(*bad) == b.DA_ERR_UNSUPPORTED
+    sz2 = b.load().diffattn_v2_prefill_train_saves_size(1, 300, 8)
+    h = lib.diffattn_v2_prefill_train
+    ok = [A, A, A, A, b.DA_BF16, 1, 300, 8, 2, 128, A, 1, 0, A, sz2, None, None]
+    bad = list(ok); bad[9] = 64
+    assert h(*bad) == b.DA_ERR_UNSUPPORTED
+    bad = list(ok); bad[8] = 3                      # 8 query heads over 3 KV heads
+    assert h(*bad) == b.DA_ERR_INVALID_ARG
+    ws2 = b.load().diffattn_v2_bwd_saved_workspace_size(1, 300, 8)
+    k = lib.diffattn_v2_bwd_saved
+    ok = [A, A, A, A, A, b.DA_BF16, 1, 300, 8, 2, 128, 1, 0, A, sz2, A, A, A, A, A, ws2, None,
+          None]
+    bad = list(ok); bad[14] = sz2 - 1
+    assert k(*bad) == b.DA_ERR_WORKSPACE
+
+
 def test_selftest_host_validation(lib):
     from differential_attention_sm_b200 import binding as b
     f = lib.diffattn_selftest_wait_timeout

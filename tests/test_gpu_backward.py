@@ -151,3 +151,69 @@ def test_v2_backward_full_size_one_pair(B):
     ds = dout[b:b + 1, :n, 2 * g:2 * g + 2].contiguous()
     ref = O.v2_bwd(qs, ks, vs, ds, x["lam"][2 * g:2 * g + 2], causal=True)
     close(res["dq"][b:b + 1, :n, 4 * g:4 * g + 4], ref["dq"], "v2 full dq")
+
+
+# ---------------------------------------------------------------------------
+# training forward with saves, and the backward from the saves
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,causal,window,norm", [(300, True, 0, True), (200, False, 0, False),
+                                                  (333, True, 70, True)])
+def test_v1_train_forward_and_saved_backward(B, N, causal, window, norm):
+    """The training forward's output equals the plain forward's (and the
+    oracle's); the backward from its saves equals the self-contained backward
+    (and the oracle backward).  dq, dk, dv come from the same kernels on the
+    same saves, so they are compared bit for bit; dlambda and the gain
+    gradient are block reductions with atomic adds, so within rounding."""
+    Bn, H, d, dv, layer = 2, 3, 64, 128, 12
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=1400 + N)
+    dout = cuda(I.v1_inputs(Bn, N, H, d, dv, seed=1500 + N)["v"])
+    q, k, v = cuda(x["q"]), cuda(x["k"]), cuda(x["v"])
+    lam_dev = B.lambda_from_params(*(cuda(x[n]) for n in ("lq1", "lk1", "lq2", "lk2")), layer)
+    lam = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], layer)
+    li = O.lambda_init(layer)
+    g = (1.0 + 0.2 * torch.randn(dv, generator=torch.Generator().manual_seed(6))).float()
+    kw = dict(causal=causal, window=window, apply_norm=norm,
+              norm_weight=cuda(g) if norm else None, lambda_init=li)
+    st = status_word()
+    out, saves = B.diffattn_v1_fwd_train(q, k, v, lam_dev, dev_status=st, **kw)
+    assert_status_ok(st)
+    plain = B.diffattn_v1_fwd_window(q, k, v, lam_dev, window, **kw)
+    assert torch.equal(out, plain), "training forward output differs from the forward"
+    ref_o = O.v1_rows(x["q"], x["k"], x["v"], lam, np.arange(Bn * N * H), causal=causal,
+                      window=window, apply_norm=norm, norm_weight=g if norm else None,
+                      lambda_init_value=li)
+    close(out.reshape(-1, dv), ref_o, "v1 training forward")
+    res = B.diffattn_v1_bwd_saved(q, k, v, dout, lam_dev, saves, dev_status=st, **kw)
+    assert_status_ok(st)
+    full = B.diffattn_v1_bwd(q, k, v, dout, lam_dev, **kw)
+    for name in ("dq", "dk", "dv"):
+        assert torch.equal(res[name], full[name]), name
+    ref = O.v1_bwd(x["q"], x["k"], x["v"], dout.cpu(), lam, causal=causal, window=window,
+                   apply_norm=norm, norm_weight=g if norm else None, lambda_init_value=li)
+    for name in ("dq", "dk", "dv", "dlambda") + (("dnorm_weight",) if norm else ()):
+        close(res[name], ref[name], "v1 saved %s N=%d" % (name, N))
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,causal,window", [(520, 8, 2, True, 0), (300, 8, 4, False, 0),
+                                                     (400, 16, 2, True, 100)])
+def test_v2_train_forward_and_saved_backward(B, N, Hq, Hkv, causal, window):
+    Bn, d = 1, 128
+    x = I.v2_inputs(Bn, N, Hq, Hkv, d, seed=1600 + N)
+    dout = torch.randn(Bn, N, Hq // 2, d, generator=torch.Generator().manual_seed(N)).to(
+        torch.bfloat16)
+    q, k, v, lam = (cuda(x[n]) for n in ("q", "k", "v", "lam"))
+    st = status_word()
+    out, saves = B.diffattn_v2_prefill_train(q, k, v, lam, causal=causal, window=window,
+                                             dev_status=st)
+    assert_status_ok(st)
+    plain = B.diffattn_v2_prefill_window(q, k, v, lam, window, causal=causal)
+    assert torch.equal(out, plain), "training forward output differs from the forward"
+    res = B.diffattn_v2_bwd_saved(q, k, v, cuda(dout), lam, saves, causal=causal, window=window,
+                                  dev_status=st)
+    assert_status_ok(st)
+    full = B.diffattn_v2_bwd(q, k, v, cuda(dout), lam, causal=causal, window=window)
+    for name in ("dq", "dk", "dv"):
+        assert torch.equal(res[name], full[name]), name
+    ref = O.v2_bwd(x["q"], x["k"], x["v"], dout, x["lam"], causal=causal, window=window)
+    for name in ("dq", "dk", "dv", "dlambda"):
+        close(res[name], ref[name], "v2 saved %s N=%d" % (name, N))
