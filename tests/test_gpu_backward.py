@@ -177,7 +177,8 @@ def test_v1_train_forward_and_saved_backward(B, N, causal, window, norm):
     st = status_word()
     out, saves = B.diffattn_v1_fwd_train(q, k, v, lam_dev, dev_status=st, **kw)
     assert_status_ok(st)
-    plain = B.diffattn_v1_fwd_window(q, k, v, lam_dev, window, **kw)
+    plain = B.diffattn_v1_fwd_window(q, k, v, lam_dev, window,
+                                     **{n: a for n, a in kw.items() if n != "window"})
     assert torch.equal(out, plain), "training forward output differs from the forward"
     ref_o = O.v1_rows(x["q"], x["k"], x["v"], lam, np.arange(Bn * N * H), causal=causal,
                       window=window, apply_norm=norm, norm_weight=g if norm else None,
