@@ -635,24 +635,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv2 = inv2_raw * p.lambda[T.hh];
       float o[64];
       {
-        uint32_t a[32], c2[32];
+        // accumulator columns read at a time: the training saves keep fewer in
+        // flight, so that O1, O2 and the 64 outputs fit in registers together
+        constexpr int kEC = kSave ? 8 : 32;
+        uint32_t a[kEC], c2[kEC];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tmem_ld32(tmem + lane_off + kColO1 + 64 * r + 32 * half, a);
-          tmem_ld32(tmem + lane_off + kColO2 + 64 * r + 32 * half, c2);
+        for (int ch = 0; ch < 64 / kEC; ++ch) {
+          if constexpr (kEC == 32) {
+            tmem_ld32(tmem + lane_off + kColO1 + 64 * r + kEC * ch, a);
+            tmem_ld32(tmem + lane_off + kColO2 + 64 * r + kEC * ch, c2);
+          } else if constexpr (kEC == 16) {
+            tmem_ld16(tmem + lane_off + kColO1 + 64 * r + kEC * ch, a);
+            tmem_ld16(tmem + lane_off + kColO2 + 64 * r + kEC * ch, c2);
+          } else {
+            tmem_ld8(tmem + lane_off + kColO1 + 64 * r + kEC * ch, a);
+            tmem_ld8(tmem + lane_off + kColO2 + 64 * r + kEC * ch, c2);
+          }
           tc_wait_ld();
-          if (half == 1) {  // O fully read: the next tile's first P.V may overwrite it
+          if (ch == 64 / kEC - 1) {  // O fully read: the next tile's first P.V may overwrite it
             tc_fence_before();
             mbar_arrive(&bars->o_free);
           }
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            o[half * 32 + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
+          for (int e = 0; e < kEC; ++e)
+            o[ch * kEC + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
           if (kSave && qrow < p.seqlen) {
             __nv_bfloat16* ob = p.obr + (((size_t)T.b * p.seqlen + qrow) * p.heads + T.hh) * 256 +
-                                64 * r + 32 * half;
+                                64 * r + kEC * ch;
 #pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8) {
+            for (int v8 = 0; v8 < kEC / 8; ++v8) {
               uint4 w1, w2;
               w1.x = pack_bf16(__uint_as_float(a[8 * v8 + 0]) * inv1, __uint_as_float(a[8 * v8 + 1]) * inv1);
               w1.y = pack_bf16(__uint_as_float(a[8 * v8 + 2]) * inv1, __uint_as_float(a[8 * v8 + 3]) * inv1);
