@@ -792,27 +792,33 @@ __global__ void __launch_bounds__(32 * kPreWarps) bwd_pre2_kernel(Pre2Args a) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int u = blockIdx.y % a.units, b = blockIdx.y / a.units;
   const float lam = a.lambda[u];
+  // lane l owns channels 4l .. 4l + 3: every row moves as 8-byte vectors
+  const int c0 = 4 * lane;
+  float gc[4] = {1.f, 1.f, 1.f, 1.f};
+  if (a.apply_norm && a.g) {  // the gain has no alignment guarantee: scalar loads
+#pragma unroll
+    for (int t = 0; t < 4; ++t) gc[t] = a.g[c0 + t];
+  }
   float dg[4] = {0.f, 0.f, 0.f, 0.f};
   float dl = 0.f;
   const int r0 = blockIdx.x * kPreRows;
   for (int i = r0 + warp; i < min(r0 + kPreRows, a.N); i += kPreWarps) {
     const size_t tok = ((size_t)b * a.N + i) * a.units + u;
-    float o1[4], o2[4], o[4], dy[4], d_o[4];
+    const uint2 w1 = *reinterpret_cast<const uint2*>(a.obr + tok * 256 + c0);
+    const uint2 w2 = *reinterpret_cast<const uint2*>(a.obr + tok * 256 + 128 + c0);
+    const uint2 wy = *reinterpret_cast<const uint2*>(a.dout + tok * 128 + c0);
+    const float o1[4] = {bf16lo(w1.x), bf16hi(w1.x), bf16lo(w1.y), bf16hi(w1.y)};
+    const float o2[4] = {bf16lo(w2.x), bf16hi(w2.x), bf16lo(w2.y), bf16hi(w2.y)};
+    const float dy[4] = {bf16lo(wy.x), bf16hi(wy.x), bf16lo(wy.y), bf16hi(wy.y)};
+    float o[4], d_o[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int c = lane + 32 * t;
-      o1[t] = __bfloat162float(a.obr[tok * 256 + c]);
-      o2[t] = __bfloat162float(a.obr[tok * 256 + 128 + c]);
-      o[t] = o1[t] - lam * o2[t];
-      dy[t] = __bfloat162float(a.dout[tok * 128 + c]);
-    }
+    for (int t = 0; t < 4; ++t) o[t] = o1[t] - lam * o2[t];
     if (a.apply_norm) {
       float ss = 0.f, gdo = 0.f;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const float gc = a.g ? a.g[lane + 32 * t] : 1.f;
         ss = fmaf(o[t], o[t], ss);
-        gdo = fmaf(gc * dy[t], o[t], gdo);
+        gdo = fmaf(gc[t] * dy[t], o[t], gdo);
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
@@ -823,24 +829,28 @@ __global__ void __launch_bounds__(32 * kPreWarps) bwd_pre2_kernel(Pre2Args a) {
       const float cr = a.post / rr, k2 = gdo / (128.f * rr * rr);
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const float gc = a.g ? a.g[lane + 32 * t] : 1.f;
-        d_o[t] = cr * (gc * dy[t] - o[t] * k2);
+        d_o[t] = cr * (gc[t] * dy[t] - o[t] * k2);
         dg[t] = fmaf(dy[t] * o[t], cr, dg[t]);
       }
     } else {
 #pragma unroll
       for (int t = 0; t < 4; ++t) d_o[t] = dy[t];
     }
+    // bf16 upstream gradients of each branch; D_r from the same rounded values
+    uint2 b1, b2;
+    b1.x = pack_bf16(d_o[0], d_o[1]);
+    b1.y = pack_bf16(d_o[2], d_o[3]);
+    b2.x = pack_bf16(-lam * d_o[0], -lam * d_o[1]);
+    b2.y = pack_bf16(-lam * d_o[2], -lam * d_o[3]);
+    *reinterpret_cast<uint2*>(a.dob + tok * 256 + c0) = b1;
+    *reinterpret_cast<uint2*>(a.dob + tok * 256 + 128 + c0) = b2;
+    const float r1[4] = {bf16lo(b1.x), bf16hi(b1.x), bf16lo(b1.y), bf16hi(b1.y)};
+    const float r2[4] = {bf16lo(b2.x), bf16hi(b2.x), bf16lo(b2.y), bf16hi(b2.y)};
     float s1 = 0.f, s2 = 0.f, sl = 0.f;
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      const int c = lane + 32 * t;
-      const __nv_bfloat16 b1 = __float2bfloat16_rn(d_o[t]);
-      const __nv_bfloat16 b2 = __float2bfloat16_rn(-lam * d_o[t]);
-      a.dob[tok * 256 + c] = b1;
-      a.dob[tok * 256 + 128 + c] = b2;
-      s1 = fmaf(__bfloat162float(b1), o1[t], s1);
-      s2 = fmaf(__bfloat162float(b2), o2[t], s2);
+      s1 = fmaf(r1[t], o1[t], s1);
+      s2 = fmaf(r2[t], o2[t], s2);
       sl = fmaf(d_o[t], o2[t], sl);
     }
 #pragma unroll
@@ -857,7 +867,7 @@ __global__ void __launch_bounds__(32 * kPreWarps) bwd_pre2_kernel(Pre2Args a) {
     dl -= sl;
   }
 #pragma unroll
-  for (int t = 0; t < 4; ++t) sh_dg[warp][lane + 32 * t] = dg[t];
+  for (int t = 0; t < 4; ++t) sh_dg[warp][c0 + t] = dg[t];
   if (lane == 0) sh_dl[warp] = dl;
   __syncthreads();
   if (threadIdx.x < 128 && a.dg) {
