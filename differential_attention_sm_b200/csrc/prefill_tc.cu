@@ -258,57 +258,6 @@ __device__ __forceinline__ int read_tile(Barriers* bars, int tc, int* dev_status
   return *(volatile int*)&bars->t_id[tc & 1];
 }
 
-// p = 2^(s * sc - u) for the 64 scores of one row of a key tile: packed bf16
-// pairs into pk, their sum into psum.  Pairs run on the f32x2 pipe; some take
-// the polynomial 2^x on the FMA pipe, the rest the multi-function unit.  V1's
-// shorter Q.K^T leaves the softmax the critical path, so it offloads more:
-// five pairs in sixteen, spread over the row, against one in eight for V2
-// (both shares and positions measured).  kMax: also fold the raw scores into
-// the 8 running maxima m8 in the same pass.
-template <int kForm, bool kMax>
-__device__ __forceinline__ void tile_exps(const uint32_t (&sr)[64], float sc, float u,
-                                          uint32_t (&pk)[32], float& psum, float (&m8)[8]) {
-  const uint64_t sc2 = f2pack(sc, sc), nu2 = f2pack(-u, -u);
-  uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const float s0 = __uint_as_float(sr[2 * e]), s1 = __uint_as_float(sr[2 * e + 1]);
-    if (kMax) m8[e & 7] = max3(m8[e & 7], s0, s1);
-    float x0, x1, p0, p1;
-    f2unpack(fma2(f2pack(s0, s1), sc2, nu2), x0, x1);
-    const int ei = e & 15;
-    if (kForm == 1 ? (ei == 2 || ei == 5 || ei == 7 || ei == 10 || ei == 13) : (ei & 7) == 7) {
-      exp2_poly2(x0, x1, p0, p1);
-    } else {
-      p0 = ex2(x0);
-      p1 = ex2(x1);
-    }
-    ps2[e & 3] = add2(ps2[e & 3], f2pack(p0, p1));
-    pk[e] = pack_bf16(p0, p1);
-  }
-  float lo, hi;
-  f2unpack(add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3])), lo, hi);
-  psum = lo + hi;
-}
-
-// One row of a key tile from tensor memory, masked entries set to -inf.
-__device__ __forceinline__ void load_scores(uint32_t t_s, int k0, int lim, int lo, bool window,
-                                            uint32_t (&sr)[64]) {
-  tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
-  tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-  tc_wait_ld();
-  if (k0 + kBN > lim) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c)
-      if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
-  }
-  if (window && k0 < lo) {  // window start (a row may see none of this tile)
-#pragma unroll
-    for (int c = 0; c < 64; ++c)
-      if (k0 + c < lo) sr[c] = __float_as_uint(-INFINITY);
-  }
-}
-
 // kForm: 1 = V1 (d_qk 64 per branch, one head), 2 = V2 (d 128 per branch, a head pair).
 // kWindow: sliding-window masking compiled in (p.window > 0) or out.
 // kSave: also write the training saves p.lse and p.obr.
@@ -543,50 +492,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t t_s = tmem + lane_off + s_col(r, buf);
-        const int k0 = (T.kv0 + j) * kBN;
         uint32_t sr[64];  // raw S row of this tile (masked entries set to -inf)
-        load_scores(t_s, k0, lim, lo, kWindow, sr);
+        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+        tc_wait_ld();
+        const int k0 = (T.kv0 + j) * kBN;
+        if (k0 + kBN > lim) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        if (kWindow && k0 < lo) {  // window start (a row may see none of this tile)
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (k0 + c < lo) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // row maximum: 3-input max over 8 independent chains
         float m8[8];
-        uint32_t pk[32];
-        float psum, alpha = 1.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float m = max3(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]),
+                         __uint_as_float(sr[16 + i]));
+          m = max3(m, __uint_as_float(sr[24 + i]), __uint_as_float(sr[32 + i]));
+          m = max3(m, __uint_as_float(sr[40 + i]), __uint_as_float(sr[48 + i]));
+          m8[i] = fmaxf(m, __uint_as_float(sr[56 + i]));
+        }
+        const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
+                              fmaxf(m8[6], m8[7])) * sc;  // sc > 0 commutes with max
+        float alpha = 1.f;
         bool resc = false;
         if (j == 0) {
-          // no reference yet: the row maximum (3-input max over 8 independent
-          // chains) first, then the exponentials against it
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float m = max3(__uint_as_float(sr[i]), __uint_as_float(sr[8 + i]),
-                           __uint_as_float(sr[16 + i]));
-            m = max3(m, __uint_as_float(sr[24 + i]), __uint_as_float(sr[32 + i]));
-            m = max3(m, __uint_as_float(sr[40 + i]), __uint_as_float(sr[48 + i]));
-            m8[i] = fmaxf(m, __uint_as_float(sr[56 + i]));
-          }
-          m_ref = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
-                       fmaxf(m8[6], m8[7])) * sc;  // sc > 0 commutes with max
-          tile_exps<kForm, false>(sr, sc, m_ref == -INFINITY ? 0.f : m_ref, pk, psum, m8);
+          m_ref = mx;
         } else {
-          // exponentials against the current reference, with the tile's row
-          // maximum reduced in the same pass; the reference only moves when
-          // that maximum outgrows it by more than 2^kLazyTau
-#pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
-          tile_exps<kForm, true>(sr, sc, m_ref == -INFINITY ? 0.f : m_ref, pk, psum, m8);
-          const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
-                                fmaxf(m8[6], m8[7])) * sc;
-          resc = mx > m_ref + kLazyTau;
-          if (__any_sync(0xffffffffu, resc)) {
-            // rare: new reference for those rows, and the exponentials again
-            // from S, which is still in tensor memory (P is stored below)
-            if (resc) {
-              alpha = ex2(m_ref - mx);
-              m_ref = mx;
-            }
-            load_scores(t_s, k0, lim, lo, kWindow, sr);
-            tile_exps<kForm, false>(sr, sc, m_ref == -INFINITY ? 0.f : m_ref, pk, psum, m8);
+          const float m_new = fmaxf(m_ref, mx);
+          resc = m_new > m_ref + kLazyTau;
+          if (resc) {
+            alpha = ex2(m_ref - m_new);
+            m_ref = m_new;
           }
         }
-        tmem_st16(t_s, *reinterpret_cast<uint32_t(*)[16]>(pk));
-        tmem_st16(t_s + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+        const float u = m_ref == -INFINITY ? 0.f : m_ref;
+        // p = 2^(s*sc - u): pairs on the f32x2 pipe; some pairs take the
+        // polynomial 2^x on the FMA pipe, the rest the multi-function unit.
+        const uint64_t sc2 = f2pack(sc, sc), nu2 = f2pack(-u, -u);
+        uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int qt = 0; qt < 2; ++qt) {  // 32 logits -> 16 packed bf16 pairs per store
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = qt * 32 + 2 * e;
+            const uint64_t x2 = fma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                     sc2, nu2);
+            float x0, x1, p0, p1;
+            f2unpack(x2, x0, x1);
+            // Share of exponentials on the polynomial: V1's shorter Q.K^T leaves
+            // the softmax the critical path, so it offloads more: five pairs in
+            // sixteen, spread over the row, against one in eight for V2 (both
+            // shares and positions measured).
+            if (kForm == 1 ? (e == 2 || e == 5 || e == 7 || e == 10 || e == 13) : (e & 7) == 7) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            ps2[e & 3] = add2(ps2[e & 3], f2pack(p0, p1));
+            pk[e] = pack_bf16(p0, p1);
+          }
+          tmem_st16(t_s + 16 * qt, pk);
+        }
+        float psum, psum_hi;
+        f2unpack(add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3])), psum, psum_hi);
+        psum += psum_hi;
         if (__any_sync(0xffffffffu, resc)) {
           // O_r must be quiescent (the previous tile's P.V into O_r done) before
           // it is rescaled in place; rows that keep their reference use alpha 1.
@@ -644,9 +621,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (kEC == 32) {
             tmem_ld32(tmem + lane_off + kColO1 + 64 * r + kEC * ch, a);
             tmem_ld32(tmem + lane_off + kColO2 + 64 * r + kEC * ch, c2);
-          } else if constexpr (kEC == 16) {
-            tmem_ld16(tmem + lane_off + kColO1 + 64 * r + kEC * ch, a);
-            tmem_ld16(tmem + lane_off + kColO2 + 64 * r + kEC * ch, c2);
           } else {
             tmem_ld8(tmem + lane_off + kColO1 + 64 * r + kEC * ch, a);
             tmem_ld8(tmem + lane_off + kColO2 + 64 * r + kEC * ch, c2);

@@ -156,12 +156,19 @@ def test_v2_backward_full_size_one_pair(B):
 # ---------------------------------------------------------------------------
 # training forward with saves, and the backward from the saves
 # ---------------------------------------------------------------------------
+def same_up_to_rounding(a, b, what):
+    """The training forward is a separate instantiation of the forward kernel
+    (it also writes the saves), compiled on its own, so its bf16 output may
+    differ from the plain forward's by a rounding step: within one bf16 unit
+    in the last place of the largest output, everywhere."""
+    d = (a.float() - b.float()).abs().max().item()
+    assert d <= b.float().abs().max().item() * 2.0 ** -7, (what, d)
 @pytest.mark.parametrize("N,causal,window,norm", [(300, True, 0, True), (200, False, 0, False),
                                                   (333, True, 70, True)])
 def test_v1_train_forward_and_saved_backward(B, N, causal, window, norm):
-    """The training forward's output equals the plain forward's (and the
-    oracle's); the backward from its saves equals the self-contained backward
-    (and the oracle backward).  dq, dk, dv come from the same kernels on the
+    """The training forward's output matches the plain forward's (up to a
+    bf16 rounding step) and the oracle's; the backward from its saves equals
+    the self-contained backward (and the oracle backward).  dq, dk, dv come from the same kernels on the
     same saves, so they are compared bit for bit; dlambda and the gain
     gradient are block reductions with atomic adds, so within rounding."""
     Bn, H, d, dv, layer = 2, 3, 64, 128, 12
@@ -179,7 +186,7 @@ def test_v1_train_forward_and_saved_backward(B, N, causal, window, norm):
     assert_status_ok(st)
     plain = B.diffattn_v1_fwd_window(q, k, v, lam_dev, window,
                                      **{n: a for n, a in kw.items() if n != "window"})
-    assert torch.equal(out, plain), "training forward output differs from the forward"
+    same_up_to_rounding(out, plain, "v1 training forward vs forward")
     ref_o = O.v1_rows(x["q"], x["k"], x["v"], lam, np.arange(Bn * N * H), causal=causal,
                       window=window, apply_norm=norm, norm_weight=g if norm else None,
                       lambda_init_value=li)
@@ -208,7 +215,10 @@ def test_v2_train_forward_and_saved_backward(B, N, Hq, Hkv, causal, window):
                                              dev_status=st)
     assert_status_ok(st)
     plain = B.diffattn_v2_prefill_window(q, k, v, lam, window, causal=causal)
-    assert torch.equal(out, plain), "training forward output differs from the forward"
+    same_up_to_rounding(out, plain, "v2 training forward vs forward")
+    ref_o = O.v2_rows(x["q"], x["k"], x["v"], x["lam"], np.arange(Bn * N * Hq // 2),
+                      causal=causal, window=window)
+    close(out.reshape(-1, d), ref_o, "v2 training forward")
     res = B.diffattn_v2_bwd_saved(q, k, v, cuda(dout), lam, saves, causal=causal, window=window,
                                   dev_status=st)
     assert_status_ok(st)
