@@ -87,7 +87,7 @@ struct DqBarriers {
   uint64_t v_full[kDqStages], v_empty[kDqStages];
   uint64_t s_full[2][2];   // [branch][S buffer]: S_r landed
   uint64_t dp_full[2];     // [branch]: dP_r landed
-  uint64_t ds_full[2];     // [branch]: dS_r written back (and dP_r read)
+  uint64_t ds_full[2][2];  // [branch][column half]: dS_r written back (and dP_r read)
   uint64_t dq_done[2][2];  // [branch][S buffer]: the dQ product of a tile has read its dS
   uint64_t s_free[2];      // [branch], V2: the softmax backward has loaded S_r
   uint32_t tmem_base;
@@ -135,7 +135,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       mbar_init(&bars->s_full[r][0], 1);
       mbar_init(&bars->s_full[r][1], 1);
       mbar_init(&bars->dp_full[r], 1);
-      mbar_init(&bars->ds_full[r], 256);  // both column halves
+      mbar_init(&bars->ds_full[r][0], 128);
+      mbar_init(&bars->ds_full[r][1], 128);
       mbar_init(&bars->dq_done[r][0], 1);
       mbar_init(&bars->dq_done[r][1], 1);
       mbar_init(&bars->s_free[r], 256);
@@ -221,7 +222,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
               !mbar_wait(&bars->s_free[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
             break;
           if (kind == 1 && j > 0 &&
-              !mbar_wait(&bars->ds_full[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
+              !(mbar_wait(&bars->ds_full[r][0], (uint32_t)(j - 1) & 1u, p.dev_status, &failed) &&
+                mbar_wait(&bars->ds_full[r][1], (uint32_t)(j - 1) & 1u, p.dev_status, &failed)))
             break;
           tc_fence_after();
           if (kind == 0) {
@@ -260,24 +262,28 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kDqStages;
-        if (!mbar_wait(&bars->ds_full[r], (uint32_t)j & 1u, p.dev_status, &failed)) break;
         if (!mbar_wait(&bars->k_full[s], (uint32_t)(j / kDqStages) & 1u, p.dev_status, &failed))
           break;
-        tc_fence_after();
         const uint32_t kt = smem_u32(sK) + s * kTile64 + (kForm == 1 ? r * kBox64 : 0);
-        for (int kk = 0; kk < 4; ++kk) {  // 16 keys per step; B = K_r, MN-major
-          // keys [32h, 32h + 32) of a tile are packed into columns [32h, 32h + 16)
-          // of the S buffer (each column half writes inside the columns it read)
-          if (kForm == 1)  // A = dS_r in tensor memory
-            tc_mma_ts(tmem + colQ(r), tmem + colS(r, j) + 32 * (kk >> 1) + 8 * (kk & 1),
-                      smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-          else  // A = dS_r in shared memory, K-major
-            tc_mma_ss(tmem + colQ(r),
-                      smem_desc_sw128(smem_u32(sDS) + r * kBox128 + kk * 32, 16, 1024),
-                      smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+        // each column half's products go out as soon as that half's dS_r is written
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(&bars->ds_full[r][h], (uint32_t)j & 1u, p.dev_status, &failed)) break;
+          tc_fence_after();
+          for (int kk = 2 * h; kk < 2 * h + 2; ++kk) {  // 16 keys each; B = K_r, MN-major
+            // keys [32h, 32h + 32) of a tile are packed into columns [32h, 32h + 16)
+            // of the S buffer (each column half writes inside the columns it read)
+            if (kForm == 1)  // A = dS_r in tensor memory
+              tc_mma_ts(tmem + colQ(r), tmem + colS(r, j) + 32 * h + 8 * (kk & 1),
+                        smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+            else  // A = dS_r in shared memory, K-major
+              tc_mma_ss(tmem + colQ(r),
+                        smem_desc_sw128(smem_u32(sDS) + r * kBox128 + kk * 32, 16, 1024),
+                        smem_desc_sw128(kt + kk * 2048, kBox64, 1024), idQ,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          }
         }
+        if (failed) break;
         tc_commit(&bars->dq_done[r][j & 1]);
         tc_commit(&bars->k_empty[s]);
       }
@@ -384,7 +390,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       if (kForm == 2) fence_proxy_async_smem();  // visible to the tensor core
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->ds_full[r]);
+      mbar_arrive(&bars->ds_full[r][h]);
     }
     __syncwarp();
     if (failed) bars->abort_flag = 1;
@@ -442,7 +448,7 @@ struct KvBarriers {
   uint64_t kv_full;
   uint64_t qd_full[kKvStages], qd_empty[kKvStages];
   uint64_t s_full[2], dp_full[2];        // S^T, dP^T landed [buffer]
-  uint64_t p_full[2], ds_full[2];        // P^T, dS^T written back [buffer]
+  uint64_t p_full[2][2], ds_full[2][2];  // P^T, dS^T written back [buffer][column half]
   uint64_t pt_free[2], dst_free[2];      // dV, dK products done with them [buffer]
   uint64_t acc_done;
   uint32_t tmem_base;
@@ -486,8 +492,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
       mbar_init(&bars->dp_full[w], 1);
-      mbar_init(&bars->p_full[w], 256);   // both column halves
-      mbar_init(&bars->ds_full[w], 256);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(&bars->p_full[w][h], 128);
+        mbar_init(&bars->ds_full[w][h], 128);
+      }
       mbar_init(&bars->pt_free[w], 1);
       mbar_init(&bars->dst_free[w], 1);
     }
@@ -598,24 +606,28 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       bool first[2] = {true, true};
       for (int s = 0; s < n_steps; ++s) {
         const int st = s % kKvStages, w = s & 1, r = s & 1;
-        if (!mbar_wait(is_v ? &bars->p_full[w] : &bars->ds_full[w], (uint32_t)(s >> 1) & 1u,
-                       p.dev_status, &failed))
-          break;
-        tc_fence_after();
         const uint32_t sq = smem_u32(sStage) + st * kStageBytes, sdo = sq + kStageQ;
         const int fb = (is_v || kForm == 2) ? 0 : r;  // accumulator of this step
-        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step; B operands MN-major
-          const uint32_t acc = (first[fb] && kk == 0) ? 0u : 1u;
-          // queries [32h, 32h + 32) of a step are packed into columns [32h, 32h + 16)
-          // of their buffer (each column half writes inside the columns it read)
-          const uint32_t pc = 32u * (uint32_t)(kk >> 1) + 8u * (uint32_t)(kk & 1);
-          if (is_v)
-            tc_mma_ts(tmem + kColDV, tmem + 128 * w + pc,
-                      smem_desc_sw128(sdo + kk * 2048, kBox64, 1024), idV, acc);
-          else
-            tc_mma_ts(tmem + kColDK + (kForm == 1 ? 64 * r : 0), tmem + 128 * w + 64 + pc,
-                      smem_desc_sw128(sq + kk * 2048, kBox64, 1024), idK, acc);
+        // each column half's products go out as soon as that half's P^T / dS^T is written
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(is_v ? &bars->p_full[w][h] : &bars->ds_full[w][h],
+                         (uint32_t)(s >> 1) & 1u, p.dev_status, &failed))
+            break;
+          tc_fence_after();
+          for (int kk = 2 * h; kk < 2 * h + 2; ++kk) {  // 16 queries each; B operands MN-major
+            const uint32_t acc = (first[fb] && kk == 0) ? 0u : 1u;
+            // queries [32h, 32h + 32) of a step are packed into columns [32h, 32h + 16)
+            // of their buffer (each column half writes inside the columns it read)
+            const uint32_t pc = 32u * (uint32_t)h + 8u * (uint32_t)(kk & 1);
+            if (is_v)
+              tc_mma_ts(tmem + kColDV, tmem + 128 * w + pc,
+                        smem_desc_sw128(sdo + kk * 2048, kBox64, 1024), idV, acc);
+            else
+              tc_mma_ts(tmem + kColDK + (kForm == 1 ? 64 * r : 0), tmem + 128 * w + 64 + pc,
+                        smem_desc_sw128(sq + kk * 2048, kBox64, 1024), idK, acc);
+          }
         }
+        if (failed) break;
         first[fb] = false;
         tc_commit(is_v ? &bars->pt_free[w] : &bars->dst_free[w]);
         tc_commit(&bars->qd_empty[st]);
@@ -692,7 +704,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[w]);
+      mbar_arrive(&bars->p_full[w][h]);
 
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full[w], ph, p.dev_status, &failed))) {
         failed = true;
@@ -725,7 +737,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
       }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->ds_full[w]);
+      mbar_arrive(&bars->ds_full[w][h]);
     }
     __syncwarp();
     if (failed) bars->abort_flag = 1;
