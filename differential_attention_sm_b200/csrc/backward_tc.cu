@@ -785,7 +785,7 @@ constexpr int kPreWarps = 8;
 constexpr int kPreRows = 64;
 
 struct Pre2Args {
-  const __nv_bfloat16* obr;  // [B][N][units][2][128]
+  const float* obr;          // [B][N][units][2][128]
   const __nv_bfloat16* dout; // [B][N][units][128]
   __nv_bfloat16* dob;        // [B][N][units][2][128]
   float* Dv;                 // [B][units][2][npad]
@@ -816,11 +816,11 @@ __global__ void __launch_bounds__(32 * kPreWarps) bwd_pre2_kernel(Pre2Args a) {
   const int r0 = blockIdx.x * kPreRows;
   for (int i = r0 + warp; i < min(r0 + kPreRows, a.N); i += kPreWarps) {
     const size_t tok = ((size_t)b * a.N + i) * a.units + u;
-    const uint2 w1 = *reinterpret_cast<const uint2*>(a.obr + tok * 256 + c0);
-    const uint2 w2 = *reinterpret_cast<const uint2*>(a.obr + tok * 256 + 128 + c0);
+    const float4 w1 = *reinterpret_cast<const float4*>(a.obr + tok * 256 + c0);
+    const float4 w2 = *reinterpret_cast<const float4*>(a.obr + tok * 256 + 128 + c0);
     const uint2 wy = *reinterpret_cast<const uint2*>(a.dout + tok * 128 + c0);
-    const float o1[4] = {bf16lo(w1.x), bf16hi(w1.x), bf16lo(w1.y), bf16hi(w1.y)};
-    const float o2[4] = {bf16lo(w2.x), bf16hi(w2.x), bf16lo(w2.y), bf16hi(w2.y)};
+    const float o1[4] = {w1.x, w1.y, w1.z, w1.w};
+    const float o2[4] = {w2.x, w2.y, w2.z, w2.w};
     const float dy[4] = {bf16lo(wy.x), bf16hi(wy.x), bf16lo(wy.y), bf16hi(wy.y)};
     float o[4], d_o[4];
 #pragma unroll
@@ -900,16 +900,20 @@ __global__ void __launch_bounds__(32 * kPreWarps) bwd_pre2_kernel(Pre2Args a) {
 
 // Saves of the training forward: per-row log2-sum-exp of each branch
 // (fp32 [B][units][2][npad], padding zero) and each branch's normalised output
-// O_r / l_r (bf16 [B][N][units][2][128]).
+// O_r / l_r (fp32 [B][N][units][2][128]: dlambda and the gain gradient are
+// sums of N x 128 products of them with heavy cancellation, which bf16 saves
+// would leave a few percent off).  The backward's workspace holds D_r (as lse)
+// and the per-branch upstream gradients (bf16, the MMA operands).
 struct SavesLayout {
-  size_t lse_bytes, obr_bytes;
+  size_t lse_bytes, obr_bytes, dob_bytes;
 };
 
 SavesLayout saves_layout(int batch, int seqlen, int units) {
   const size_t npad = (size_t)((seqlen + 63) / 64) * 64;
   SavesLayout L;
   L.lse_bytes = ((size_t)batch * units * 2 * npad * 4 + 255) & ~size_t(255);
-  L.obr_bytes = ((size_t)batch * seqlen * units * 256 * 2 + 255) & ~size_t(255);
+  L.obr_bytes = ((size_t)batch * seqlen * units * 256 * 4 + 255) & ~size_t(255);
+  L.dob_bytes = ((size_t)batch * seqlen * units * 256 * 2 + 255) & ~size_t(255);
   return L;
 }
 
@@ -919,8 +923,8 @@ size_t train_saves_bytes(int batch, int seqlen, int units) {
 }
 
 size_t saved_bwd_workspace_bytes(int batch, int seqlen, int units) {
-  // D_r (as lse) and the per-branch upstream gradients (as the branch outputs)
-  return train_saves_bytes(batch, seqlen, units);
+  const SavesLayout L = saves_layout(batch, seqlen, units);
+  return L.lse_bytes + L.dob_bytes + 256;
 }
 
 size_t fused_bwd_workspace_bytes(int batch, int seqlen, int units) {
@@ -968,7 +972,7 @@ cudaError_t launch_bwd_from_saves(const FusedBwdArgs& a, const void* saves, cuda
   const SavesLayout L = saves_layout(B, N, U);
   const uint8_t* sv = align256(const_cast<void*>(saves));
   const float* lse = reinterpret_cast<const float*>(sv);
-  const __nv_bfloat16* obr = reinterpret_cast<const __nv_bfloat16*>(sv + L.lse_bytes);
+  const float* obr = reinterpret_cast<const float*>(sv + L.lse_bytes);
   uint8_t* wb = align256(a.workspace);
   float* Dv = reinterpret_cast<float*>(wb);
   __nv_bfloat16* dob = reinterpret_cast<__nv_bfloat16*>(wb + L.lse_bytes);

@@ -122,10 +122,10 @@ struct Params {
   __nv_bfloat16* out;
   // training saves (nullptr when not wanted): per-row log2-sum-exp of each
   // branch [B][units][2][lse_stride], and each branch's normalised output
-  // O_r / l_r as bf16 [B][N][units][2][128]
+  // O_r / l_r as fp32 [B][N][units][2][128]
   float* lse;
   int lse_stride;  // row stride of lse (>= seqlen)
-  __nv_bfloat16* obr;
+  float* obr;
   int* dev_status;
 };
 
@@ -633,22 +633,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < kEC; ++e)
             o[ch * kEC + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
-          if (kSave && qrow < p.seqlen) {
-            __nv_bfloat16* ob = p.obr + (((size_t)T.b * p.seqlen + qrow) * p.heads + T.hh) * 256 +
-                                64 * r + kEC * ch;
+          if (kSave && qrow < p.seqlen) {  // normalised branch outputs, fp32
+            float* ob = p.obr + (((size_t)T.b * p.seqlen + qrow) * p.heads + T.hh) * 256 +
+                        64 * r + kEC * ch;
 #pragma unroll
-            for (int v8 = 0; v8 < kEC / 8; ++v8) {
-              uint4 w1, w2;
-              w1.x = pack_bf16(__uint_as_float(a[8 * v8 + 0]) * inv1, __uint_as_float(a[8 * v8 + 1]) * inv1);
-              w1.y = pack_bf16(__uint_as_float(a[8 * v8 + 2]) * inv1, __uint_as_float(a[8 * v8 + 3]) * inv1);
-              w1.z = pack_bf16(__uint_as_float(a[8 * v8 + 4]) * inv1, __uint_as_float(a[8 * v8 + 5]) * inv1);
-              w1.w = pack_bf16(__uint_as_float(a[8 * v8 + 6]) * inv1, __uint_as_float(a[8 * v8 + 7]) * inv1);
-              w2.x = pack_bf16(__uint_as_float(c2[8 * v8 + 0]) * inv2_raw, __uint_as_float(c2[8 * v8 + 1]) * inv2_raw);
-              w2.y = pack_bf16(__uint_as_float(c2[8 * v8 + 2]) * inv2_raw, __uint_as_float(c2[8 * v8 + 3]) * inv2_raw);
-              w2.z = pack_bf16(__uint_as_float(c2[8 * v8 + 4]) * inv2_raw, __uint_as_float(c2[8 * v8 + 5]) * inv2_raw);
-              w2.w = pack_bf16(__uint_as_float(c2[8 * v8 + 6]) * inv2_raw, __uint_as_float(c2[8 * v8 + 7]) * inv2_raw);
-              *reinterpret_cast<uint4*>(ob + 8 * v8) = w1;
-              *reinterpret_cast<uint4*>(ob + 128 + 8 * v8) = w2;
+            for (int v4 = 0; v4 < kEC / 4; ++v4) {
+              *reinterpret_cast<float4*>(ob + 4 * v4) =
+                  make_float4(__uint_as_float(a[4 * v4]) * inv1, __uint_as_float(a[4 * v4 + 1]) * inv1,
+                              __uint_as_float(a[4 * v4 + 2]) * inv1,
+                              __uint_as_float(a[4 * v4 + 3]) * inv1);
+              *reinterpret_cast<float4*>(ob + 128 + 4 * v4) = make_float4(
+                  __uint_as_float(c2[4 * v4]) * inv2_raw, __uint_as_float(c2[4 * v4 + 1]) * inv2_raw,
+                  __uint_as_float(c2[4 * v4 + 2]) * inv2_raw,
+                  __uint_as_float(c2[4 * v4 + 3]) * inv2_raw);
             }
           }
         }
@@ -783,7 +780,7 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   p.lse_stride = a.lse_stride;
-  p.obr = static_cast<__nv_bfloat16*>(a.obr);
+  p.obr = static_cast<float*>(a.obr);
   p.dev_status = a.dev_status;
   const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
   const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +

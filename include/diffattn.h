@@ -284,8 +284,8 @@ DA_API int diffattn_v1_decode_window(const void* q, const void* k_cache, const v
  * (per-row log-sum-exp and normalised branch outputs), then one kernel
  * accumulates dQ per query tile and one accumulates dK and dV per key tile
  * in tensor memory, recomputing the maps tile by tile; no N x N buffer
- * exists and the workspace is about (8 units + 2 units) x N x 128 bf16 per
- * batch entry.  `dev_status` (optional) receives DA_ERR_DEVICE_TIMEOUT if
+ * exists and the workspace is about 1.8 KB per token and head (V1) or head
+ * pair (V2).  `dev_status` (optional) receives DA_ERR_DEVICE_TIMEOUT if
  * one of its bounded waits ever times out. */
 
 /* V1.  q, k: device [batch, seqlen, n_heads, 2*d_qk]; v, dout: device
@@ -329,8 +329,8 @@ DA_API int diffattn_v2_bwd(const void* q, const void* k, const void* v, const vo
  *  - Supported: bf16 with the tensor-core widths (V1 d_qk 64, d_v 128; V2
  *    head_dim 128); else DA_ERR_UNSUPPORTED.
  *  - saves: caller-owned device memory of at least the *_saves_size bytes
- *    (contents: per-row log2-sum-exp of each branch, fp32, and each branch's
- *    normalised output O_r / l_r, bf16; any alignment).  The backward must
+ *    (contents: per-row log2-sum-exp of each branch and each branch's
+ *    normalised output O_r / l_r, both fp32; any alignment).  The backward must
  *    get the same q, k, v, lambda, causal, window and norm arguments as the
  *    forward that wrote the saves; the saves are only read by it.
  *  - workspace of the backward: at least the *_bwd_saved_workspace_size
