@@ -6,7 +6,7 @@
 // glossary page re-parameterises it by four vectors), so its gradient and,
 // in V1, that of the per-head norm gain are produced too.
 //
-// This first implementation materialises the two attention maps of one head
+// The general implementation materialises the two attention maps of one head
 // (V1) or head pair (V2) for a chunk of batch entries at a time:
 //   for each branch r:  S_r = Q_r K_r^T / sqrt(d)           (GEMM)
 //                       P_r = masked softmax(S_r)            (kernel, bf16)
@@ -19,18 +19,18 @@
 //                       dQ_r = dS_r K_r / sqrt(d)            (GEMM)
 //                       dK_r += dS_r^T Q_r / sqrt(d)         (GEMM)
 //                       dV  += P_r^T do_r                    (GEMM)
-// The six products are plain strided-batched GEMMs (bf16 operands, fp32
-// accumulation) issued to cuBLAS; every other step is a kernel here.  The
-// masked-out part of each map is zero, so the GEMMs run over the full N x N
-// square (twice the causal work).  Gradients are written in fp32.
-#include <cublas_v2.h>
+// The six products are strided-batched GEMMs (bf16 operands, fp32
+// accumulation) on a CUDA-core kernel of this file; every other step is a
+// kernel here too.  This path only serves the widths the fused tensor-core
+// backward (backward_tc.cu) does not cover.  The masked-out part of each map
+// is zero, so the GEMMs run over the full N x N square (twice the causal
+// work).  Gradients are written in fp32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
 #include <initializer_list>
-#include <mutex>
 
 #include "diffattn.h"
 #include "kernels.h"
@@ -38,12 +38,8 @@
 namespace da {
 namespace {
 
-constexpr int kMaxDevices = 64;
 constexpr size_t kChunkCap = size_t(4) << 30;  // workspace bound per chunk of batch entries
 constexpr int kMaxDv = 128;
-
-std::mutex g_mutex[kMaxDevices];
-cublasHandle_t g_handle[kMaxDevices] = {};
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -249,15 +245,91 @@ __global__ void lambda_params_bwd_kernel(const float* lq1, const float* lk1, con
 // Row-major C[M x N] (ldc) = alpha op(A) op(B) + beta C, batched with strides.
 // A is row-major [M x K] (lda), or [K x M] read transposed when ta; B is
 // [K x N] (ldb), or [N x K] read transposed when tb.  bf16 operands, fp32 C.
-// (cuBLAS is column-major: it computes C^T = op(B)^T op(A)^T.)
-cublasStatus_t gemm_rm(cublasHandle_t h, bool ta, bool tb, int M, int N, int K, float alpha,
-                       const void* A, int lda, long long sA, const void* B, int ldb,
-                       long long sB, float beta, float* C, int ldc, long long sC, int batch) {
-  return cublasGemmStridedBatchedEx(h, tb ? CUBLAS_OP_T : CUBLAS_OP_N,
-                                    ta ? CUBLAS_OP_T : CUBLAS_OP_N, N, M, K, &alpha, B,
-                                    CUDA_R_16BF, ldb, sB, A, CUDA_R_16BF, lda, sA, &beta, C,
-                                    CUDA_R_32F, ldc, sC, batch, CUBLAS_COMPUTE_32F,
-                                    CUBLAS_GEMM_DEFAULT);
+// A plain CUDA-core kernel: this path serves only the widths the fused
+// tensor-core backward does not cover.  64 x 64 output tiles, K in steps of
+// 16 staged in shared memory as fp32, a 4 x 4 block of outputs per thread;
+// out-of-range operand elements read as zero.
+constexpr int kGT = 64, kGK = 16;
+
+template <bool kTA, bool kTB>
+__global__ void __launch_bounds__(256) gemm_bf16_simt_kernel(
+    int M, int N, int K, float alpha, const __nv_bfloat16* A, int lda, long long sA,
+    const __nv_bfloat16* Bm, int ldb, long long sB, float beta, float* C, int ldc, long long sC) {
+  __shared__ float As[kGK][kGT + 4];
+  __shared__ float Bs[kGK][kGT + 4];
+  const int z = blockIdx.z;
+  A += z * sA;
+  Bm += z * sB;
+  C += z * sC;
+  const int m0 = blockIdx.y * kGT, n0 = blockIdx.x * kGT;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += kGK) {
+    for (int e = threadIdx.x; e < kGT * kGK; e += 256) {
+      // element (row i of the tile, column kk of the K step), both operands
+      const int i = kTA ? e % kGT : e / kGK, kk = kTA ? e / kGT : e % kGK;
+      const int m = m0 + i, k = k0 + kk;
+      float va = 0.f;
+      if (m < M && k < K)
+        va = __bfloat162float(kTA ? A[(long long)k * lda + m] : A[(long long)m * lda + k]);
+      As[kk][i] = va;
+      const int j = kTB ? e / kGK : e % kGT, kb = kTB ? e % kGK : e / kGT;
+      const int n = n0 + j, kn = k0 + kb;
+      float vb = 0.f;
+      if (n < N && kn < K)
+        vb = __bfloat162float(kTB ? Bm[(long long)n * ldb + kn] : Bm[(long long)kn * ldb + n]);
+      Bs[kb][j] = vb;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kGK; ++kk) {
+      float a4[4], b4[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        a4[t] = As[kk][ty * 4 + t];
+        b4[t] = Bs[kk][tx * 4 + t];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n >= N) continue;
+      float* c = C + (long long)m * ldc + n;
+      *c = alpha * acc[i][j] + (beta != 0.f ? beta * *c : 0.f);
+    }
+  }
+}
+
+cudaError_t gemm_rm(cudaStream_t st, bool ta, bool tb, int M, int N, int K, float alpha,
+                    const void* A, int lda, long long sA, const void* B, int ldb, long long sB,
+                    float beta, float* C, int ldc, long long sC, int batch) {
+  const dim3 grid((unsigned)((N + kGT - 1) / kGT), (unsigned)((M + kGT - 1) / kGT),
+                  (unsigned)batch);
+  const auto* a = static_cast<const __nv_bfloat16*>(A);
+  const auto* b = static_cast<const __nv_bfloat16*>(B);
+  if (ta && tb)
+    gemm_bf16_simt_kernel<true, true><<<grid, 256, 0, st>>>(M, N, K, alpha, a, lda, sA, b, ldb, sB,
+                                                          beta, C, ldc, sC);
+  else if (ta)
+    gemm_bf16_simt_kernel<true, false><<<grid, 256, 0, st>>>(M, N, K, alpha, a, lda, sA, b, ldb,
+                                                           sB, beta, C, ldc, sC);
+  else if (tb)
+    gemm_bf16_simt_kernel<false, true><<<grid, 256, 0, st>>>(M, N, K, alpha, a, lda, sA, b, ldb,
+                                                           sB, beta, C, ldc, sC);
+  else
+    gemm_bf16_simt_kernel<false, false><<<grid, 256, 0, st>>>(M, N, K, alpha, a, lda, sA, b, ldb,
+                                                            sB, beta, C, ldc, sC);
+  return cudaGetLastError();
 }
 
 // Geometry of one backward problem, in elements.  A "unit" is one head (V1)
@@ -293,20 +365,6 @@ size_t bwd_workspace_bytes(int B, int N, int dv) {
   return (size_t)chunk_units(B, N, dv) * unit_bytes(N, dv) + 256;
 }
 
-int get_handle(cublasHandle_t* out, int* dev_out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DA_ERR_CUDA;
-  *dev_out = dev;
-  if (!g_handle[dev]) {
-    if (cublasCreate(&g_handle[dev]) != CUBLAS_STATUS_SUCCESS) {
-      g_handle[dev] = nullptr;
-      return DA_ERR_CUDA;
-    }
-  }
-  *out = g_handle[dev];
-  return DA_OK;
-}
-
 // The whole backward for one problem (device pointers; fp32 gradients).
 int run_bwd(const Geo& G, const __nv_bfloat16* q, const __nv_bfloat16* k,
             const __nv_bfloat16* v, const __nv_bfloat16* dout, const float* lambda, int causal,
@@ -316,18 +374,6 @@ int run_bwd(const Geo& G, const __nv_bfloat16* q, const __nv_bfloat16* k,
   const int N = G.N, dvw = G.dv;
   const int cu = chunk_units(G.B, N, dvw);
   if (!ws || ws_bytes < bwd_workspace_bytes(G.B, N, dvw)) return DA_ERR_WORKSPACE;
-  int dev = 0;
-  cublasHandle_t h = nullptr;
-  {
-    int dd = 0;
-    if (cudaGetDevice(&dd) != cudaSuccess || dd < 0 || dd >= kMaxDevices) return DA_ERR_CUDA;
-    dev = dd;
-  }
-  std::lock_guard<std::mutex> lock(g_mutex[dev]);
-  if (get_handle(&h, &dev) != DA_OK) return DA_ERR_CUDA;
-  if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return DA_ERR_CUDA;
-  if (cublasSetPointerMode(h, CUBLAS_POINTER_MODE_HOST) != CUBLAS_STATUS_SUCCESS)
-    return DA_ERR_CUDA;
 
   // carve the workspace
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
@@ -372,13 +418,13 @@ int run_bwd(const Geo& G, const __nv_bfloat16* q, const __nv_bfloat16* k,
       for (int r = 0; r < 2; ++r) {
         const __nv_bfloat16* qr = q + b0 * G.q_b + hh * G.q_unit + r * G.q_br;
         const __nv_bfloat16* kr = k + b0 * G.k_b + kvh * G.k_unit + r * G.k_br;
-        if (gemm_rm(h, false, true, N, N, G.d, scale, qr, (int)G.q_row, G.q_b, kr,
-                    (int)G.k_row, G.k_b, 0.f, X, N, (long long)n2, nb) != CUBLAS_STATUS_SUCCESS)
+        if (gemm_rm(st, false, true, N, N, G.d, scale, qr, (int)G.q_row, G.q_b, kr,
+                    (int)G.k_row, G.k_b, 0.f, X, N, (long long)n2, nb) != cudaSuccess)
           return DA_ERR_CUDA;
         bwd_softmax_kernel<<<grid_rows, 32 * rows_per_blk, 0, st>>>(X, P[r], N, nb, causal,
                                                                     window);
-        if (gemm_rm(h, false, false, N, dvw, N, 1.f, P[r], N, (long long)n2, vb, (int)G.v_row,
-                    G.v_b, 0.f, O[r], dvw, (long long)N * dvw, nb) != CUBLAS_STATUS_SUCCESS)
+        if (gemm_rm(st, false, false, N, dvw, N, 1.f, P[r], N, (long long)n2, vb, (int)G.v_row,
+                    G.v_b, 0.f, O[r], dvw, (long long)N * dvw, nb) != cudaSuccess)
           return DA_ERR_CUDA;
       }
       PreArgs pa;
@@ -409,17 +455,16 @@ int run_bwd(const Geo& G, const __nv_bfloat16* q, const __nv_bfloat16* k,
         float* dqr = dq + b0 * G.q_b + hh * G.q_unit + r * G.q_br;
         float* dkr = dk + b0 * G.k_b + kvh * G.k_unit + r * G.k_br;
         float* dvb = dv + b0 * G.v_b + kvh * G.v_unit;
-        if (gemm_rm(h, false, true, N, N, dvw, 1.f, dO[r], dvw, (long long)N * dvw, vb,
-                    (int)G.v_row, G.v_b, 0.f, X, N, (long long)n2, nb) != CUBLAS_STATUS_SUCCESS)
+        if (gemm_rm(st, false, true, N, N, dvw, 1.f, dO[r], dvw, (long long)N * dvw, vb,
+                    (int)G.v_row, G.v_b, 0.f, X, N, (long long)n2, nb) != cudaSuccess)
           return DA_ERR_CUDA;
         bwd_ds_kernel<<<grid_rows, 32 * rows_per_blk, 0, st>>>(P[r], X, D[r], dS, N, nb);
-        if (gemm_rm(h, false, false, N, G.d, N, scale, dS, N, (long long)n2, kr, (int)G.k_row,
-                    G.k_b, 0.f, dqr, (int)G.q_row, G.q_b, nb) != CUBLAS_STATUS_SUCCESS ||
-            gemm_rm(h, true, false, N, G.d, N, scale, dS, N, (long long)n2, qr, (int)G.q_row,
-                    G.q_b, 1.f, dkr, (int)G.k_row, G.k_b, nb) != CUBLAS_STATUS_SUCCESS ||
-            gemm_rm(h, true, false, N, dvw, N, 1.f, P[r], N, (long long)n2, dO[r], dvw,
-                    (long long)N * dvw, 1.f, dvb, (int)G.v_row, G.v_b, nb) !=
-                CUBLAS_STATUS_SUCCESS)
+        if (gemm_rm(st, false, false, N, G.d, N, scale, dS, N, (long long)n2, kr, (int)G.k_row,
+                    G.k_b, 0.f, dqr, (int)G.q_row, G.q_b, nb) != cudaSuccess ||
+            gemm_rm(st, true, false, N, G.d, N, scale, dS, N, (long long)n2, qr, (int)G.q_row,
+                    G.q_b, 1.f, dkr, (int)G.k_row, G.k_b, nb) != cudaSuccess ||
+            gemm_rm(st, true, false, N, dvw, N, 1.f, P[r], N, (long long)n2, dO[r], dvw,
+                    (long long)N * dvw, 1.f, dvb, (int)G.v_row, G.v_b, nb) != cudaSuccess)
           return DA_ERR_CUDA;
       }
     }

@@ -28,10 +28,9 @@
  *    it beforehand) and returns early, leaving the output undefined.
  *  - Thread safety: concurrent calls on different streams are independent,
  *    with two exceptions: diffattn_v2_decode_noalloc's shared scratch array
- *    (see that entry point) and the prefill's tile counters (next).  Global
- *    state: a per-device cuBLAS handle for the materialising backward,
- *    created under a lock on first use, and, for the bf16 tensor-core
- *    prefill (diffattn_v1_fwd / diffattn_v2_prefill and their window,
+ *    (see that entry point) and the prefill's tile counters (next).  The
+ *    library calls no other library that keeps state.  Global state: for the
+ *    bf16 tensor-core prefill (diffattn_v1_fwd / diffattn_v2_prefill and their window,
  *    training and projection variants), 64 tile counters per device in a
  *    statically allocated array.  The host gives each such launch the next
  *    counter in turn, fixed when the launch is enqueued (or captured into a
@@ -269,15 +268,14 @@ DA_API int diffattn_v1_decode_window(const void* q, const void* k_cache, const v
  * fp32, written (not accumulated) in the layout of the matching input.
  * Outputs must not overlap inputs or each other.
  *
- * For widths outside the tensor-core forward the implementation materialises the two attention maps of one head (V1)
- * or head pair (V2) for a chunk of batch entries at a time in `workspace`
- * (size from the *_workspace_size query; about 10 N^2 bytes per batch entry
- * of a chunk) and issues its six matrix products per branch as
- * strided-batched cuBLAS GEMMs (bf16 operands, fp32 accumulation).  The
- * first call on a device creates that device's cuBLAS handle, which
- * allocates cuBLAS's own workspace; calls on one device are serialised on
- * the host while they enqueue.  Errors: as for the forward, plus
- * DA_ERR_WORKSPACE for a missing or short workspace.
+ * For widths outside the tensor-core forward the implementation
+ * materialises the two attention maps of one head (V1) or head pair (V2)
+ * for a chunk of batch entries at a time in `workspace` (size from the
+ * *_workspace_size query; about 10 N^2 bytes per batch entry of a chunk)
+ * and runs its six matrix products per branch as strided-batched GEMMs on
+ * a CUDA-core kernel of this library (bf16 operands, fp32 accumulation).
+ * Errors: as for the forward, plus DA_ERR_WORKSPACE for a missing or short
+ * workspace.
  *
  * The shapes of the tensor-core forward (V1 d_qk 64 / d_v 128, V2 head_dim
  * 128) take a fused path instead: the forward kernel re-runs with saves
