@@ -647,6 +647,29 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None, cpu_s=
             "frac": round(tt / peaks["bf16_tflops"], 4), "flop": ft,
             "what": "training forward with saves + backward from the saves "
                     "(768 + 1792 flop per visible pair)"}
+        if cpu_s > 0:  # the oracle's backward (it runs the forward too) on head slices
+            lam_h = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
+            g_h = dout.cpu()
+            rng = np.random.default_rng(20)
+            n_p, n_run = 512, [0]
+
+            def slices_once(n):
+                for _ in range(n):
+                    b, h = int(rng.integers(w.B)), int(rng.integers(w.H))
+                    sl = (slice(b, b + 1), slice(0, n_p), slice(h, h + 1))
+                    O.v1_bwd(x["q"][sl], x["k"][sl], x["v"][sl], g_h[sl], lam_h[h:h + 1],
+                             causal=True, apply_norm=True, eps=w.eps, lambda_init_value=li)
+                n_run[0] += n
+                return float(n * prefill_pairs(1, n_p, 1) * v1_bwd_flops_per_pair(w.d, w.dv))
+            cb = dict(oracle_rate(slices_once, cpu_s, 1e12,
+                                  "(batch, head) slices of the first 512 tokens"),
+                      unit="TFLOP/s", cores=1)
+            out["v1_backward_saved_bf16"]["cpu_baseline"] = cb
+            # the same oracle calls, counted with the forward's flops as well
+            ct = dict(cb)
+            ct["value"] = cb["value"] * (v1_flops_per_pair(w.d, w.dv) + v1_bwd_flops_per_pair(
+                w.d, w.dv)) / v1_bwd_flops_per_pair(w.d, w.dv)
+            out["v1_train_step_bf16"]["cpu_baseline"] = ct
         del q, k, v, dout, ws, saves, grads, o
         torch.cuda.empty_cache()
 
