@@ -651,7 +651,7 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None, cpu_s=
             lam_h = O.lambda_from_params(x["lq1"], x["lk1"], x["lq2"], x["lk2"], w.layer)
             g_h = dout.cpu()
             rng = np.random.default_rng(20)
-            n_p, n_run = 512, [0]
+            n_p = 512
 
             def slices_once(n):
                 for _ in range(n):
@@ -659,7 +659,6 @@ def run_extras(local_rank, peaks, peak_src, only=None, decode_batch=None, cpu_s=
                     sl = (slice(b, b + 1), slice(0, n_p), slice(h, h + 1))
                     O.v1_bwd(x["q"][sl], x["k"][sl], x["v"][sl], g_h[sl], lam_h[h:h + 1],
                              causal=True, apply_norm=True, eps=w.eps, lambda_init_value=li)
-                n_run[0] += n
                 return float(n * prefill_pairs(1, n_p, 1) * v1_bwd_flops_per_pair(w.d, w.dv))
             cb = dict(oracle_rate(slices_once, cpu_s, 1e12,
                                   "(batch, head) slices of the first 512 tokens"),
