@@ -89,7 +89,8 @@ struct Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2][2], p_full[2][2];   // [branch][buffer]
+  uint64_t s_full[2][2];                  // [branch][buffer]
+  uint64_t p_full[2][2][2];               // [branch][buffer][key half]
   uint64_t o_done[2][2];                  // [branch][buffer]: P_r(j).V complete
   uint64_t o_free;                        // the epilogue has read O out of tensor memory
   uint64_t t_full[2], t_empty[2];         // tile numbers handed to the roles [buffer]
@@ -292,7 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int r = 0; r < 2; ++r) {
       for (int u = 0; u < 2; ++u) {
         mbar_init(&bars->s_full[r][u], 1);
-        mbar_init(&bars->p_full[r][u], 128);
+        mbar_init(&bars->p_full[r][u][0], 128);
+        mbar_init(&bars->p_full[r][u][1], 128);
         mbar_init(&bars->o_done[r][u], 1);
       }
     }
@@ -440,20 +442,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < T.n_kv; ++j, ++J) {
           const int s = J % kStages;
           if (!mbar_wait(&bars->v_full[s], (J / kStages) & 1u, p.dev_status, &failed)) break;
-          if (!mbar_wait(&bars->p_full[r][J & 1], (J >> 1) & 1u, p.dev_status, &failed)) break;
           // the first P.V of a tile overwrites O: the previous tile's
           // epilogue must have read it out
           if (j == 0 && tc > 0 &&
               !mbar_wait(&bars->o_free, (uint32_t)(tc - 1) & 1u, p.dev_status, &failed))
             break;
-          tc_fence_after();
           const uint32_t vt = v_addr + s * kKVTile;
           const uint32_t pcol = pcol0 + 64u * (J & 1u);
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
-            tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
-                      kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          // each half of the keys goes out once its P is in tensor memory (V2
+          // releases the halves one after the other, V1 both at the end)
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(&bars->p_full[r][J & 1][h], (J >> 1) & 1u, p.dev_status, &failed))
+              break;
+            tc_fence_after();
+            for (int kk = 2 * h; kk < 2 * h + 2; ++kk) {
+              // B = V tile, MN-major: 64-column halves kKVBox apart, 8-key groups 1 KB apart
+              tc_mma_ts(ocol, pcol + kk * 8, smem_desc_sw128(vt + kk * 2048, kKVBox, 1024),
+                        kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+            }
           }
+          if (failed) break;
           tc_commit(&bars->o_done[r][J & 1]);
           tc_commit(&bars->v_empty[s]);
         }
@@ -532,6 +540,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float u = m_ref == -INFINITY ? 0.f : m_ref;
+        // O_r rescaled in place when a row's reference moved: O_r must be
+        // quiescent first (the previous tile's P.V into O_r done); rows that
+        // keep their reference use alpha 1.  V2 does it before any P of this
+        // tile is released to its P.V, V1 after computing P (both orders put
+        // the rescale before this tile's P.V).
+        auto rescale_o = [&]() -> bool {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[r][(J - 1) & 1],
+                                                  ((J - 1) >> 1) & 1u, p.dev_status,
+                                                  &failed)))
+            return false;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t ov[16];
+            tmem_ld16(t_o + 16 * c, ov);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st16(t_o + 16 * c, ov);
+          }
+          return true;
+        };
+        if (kForm == 2 && __any_sync(0xffffffffu, resc) && !rescale_o()) {
+          failed = true;
+          break;
+        }
         // p = 2^(s*sc - u): pairs on the f32x2 pipe; some pairs take the
         // polynomial 2^x on the FMA pipe, the rest the multi-function unit.
         const uint64_t sc2 = f2pack(sc, sc), nu2 = f2pack(-u, -u);
@@ -560,34 +594,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[e] = pack_bf16(p0, p1);
           }
           tmem_st16(t_s + 16 * qt, pk);
+          if (kForm == 2) {  // this half of P is ready for its P.V
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[r][buf][qt]);
+          }
         }
         float psum, psum_hi;
         f2unpack(add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3])), psum, psum_hi);
         psum += psum_hi;
-        if (__any_sync(0xffffffffu, resc)) {
-          // O_r must be quiescent (the previous tile's P.V into O_r done) before
-          // it is rescaled in place; rows that keep their reference use alpha 1.
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[r][(J - 1) & 1],
-                                                  ((J - 1) >> 1) & 1u, p.dev_status,
-                                                  &failed))) {
-            failed = true;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t ov[16];
-            tmem_ld16(t_o + 16 * c, ov);
-            tc_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st16(t_o + 16 * c, ov);
-          }
+        if (kForm == 1 && __any_sync(0xffffffffu, resc) && !rescale_o()) {
+          failed = true;
+          break;
         }
         l_run = l_run * alpha + psum;
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[r][buf]);
+        if (kForm == 1) {
+          tc_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars->p_full[r][buf][0]);
+          mbar_arrive(&bars->p_full[r][buf][1]);
+        }
       }
 
       // ---- epilogue: o = O1/l1 - lambda O2/l2 (+ V1 norm), channels [64 r, 64 r + 64) ----
