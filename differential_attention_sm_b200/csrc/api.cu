@@ -408,8 +408,9 @@ size_t diffattn_v1_decode_workspace_size(int batch, int n_heads, int d_qk, int d
                                          int max_cache_len) {
   if (batch < 1 || n_heads < 1 || d_qk < 1 || d_v < 1 || max_cache_len < 1) return 0;
   if (!v1_decode_fast(d_qk, d_v)) return 0;
-  da::V1DecodePlan plan = da::plan_v1_decode(batch, n_heads, max_cache_len, kPlanSMs);
-  return da::v1_decode_workspace_bytes(plan);
+  // the V1 fast path runs on the split-KV tensor-core kernel, one KV head per head
+  da::V2DecodePlan plan = da::plan_v2_decode(batch, n_heads, max_cache_len, kPlanSMs);
+  return da::v2_decode_workspace_bytes(plan);
 }
 
 int diffattn_v1_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -429,7 +430,6 @@ int diffattn_v1_decode_window(const void* q, const void* k_cache, const void* v_
                               const float* lambda, int apply_norm, const float* norm_weight,
                               float norm_eps, float lambda_init, void* workspace,
                               size_t workspace_bytes, int* dev_status, void* stream) {
-  (void)dev_status;  // the kernels used here never wait on asynchronous copies
   if (!q || !k_cache || !v_cache || !out || !lambda) return DA_ERR_INVALID_ARG;
   if (window < 0) return DA_ERR_INVALID_ARG;
   if (!dtype_ok(dtype)) return DA_ERR_INVALID_ARG;
@@ -446,14 +446,24 @@ int diffattn_v1_decode_window(const void* q, const void* k_cache, const void* v_
   const int span = (window > 0 && window < max_len) ? window : max_len;
 
   if (dtype == DA_BF16 && v1_decode_fast(d_qk, d_v)) {
-    da::V1DecodePlan plan = da::plan_v1_decode(batch, n_heads, span, kPlanSMs);
-    const size_t need = da::v1_decode_workspace_bytes(plan);
+    // Each head's K row is [branch 1 | branch 2] (64 + 64) and its V row is
+    // 128 wide, so the split-KV tensor-core kernel of V2 serves it with the
+    // head as a KV head and its two branches as a pair of query heads.
+    da::V2DecodePlan plan = da::plan_v2_decode(batch, n_heads, span, kPlanSMs);
+    const size_t need = da::v2_decode_workspace_bytes(plan);
     if (!workspace || workspace_bytes < need) return DA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return DA_ERR_ALIGNMENT;
-    return cuda_status(da::launch_v1_decode(q, k_cache, v_cache, cache_lens, max_len, window, out,
-                                            batch, n_heads, lambda, apply_norm ? 1 : 0,
-                                            norm_weight, norm_eps, post_scale, plan, workspace,
-                                            st));
+    const int sms = num_sms();
+    if (sms < 1) return DA_ERR_CUDA;
+    plan.grid = plan.n_items < sms ? plan.n_items : sms;
+    CUtensorMap tk, tv;
+    if (make_tmap_4d(&tk, k_cache, 128, n_heads, max_len, batch, 64, 1, 64, 1) ||
+        make_tmap_4d(&tv, v_cache, 128, n_heads, max_len, batch, 64, 1, 64, 1))
+      return DA_ERR_CUDA;
+    return cuda_status(da::launch_v1_decode_tc(tk, tv, q, cache_lens, max_len, window, out,
+                                               batch, n_heads, lambda, apply_norm ? 1 : 0,
+                                               norm_weight, norm_eps, post_scale, plan, workspace,
+                                               dev_status, st));
   }
 
   GenericProblem P{};

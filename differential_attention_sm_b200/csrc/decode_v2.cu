@@ -46,7 +46,8 @@ constexpr int kSmemBytes =
     1024 + kStages * kStageBytes + kRedOBytes + kRedMLBytes + 2 * kStages * 8 + 16;
 
 struct Params {
-  const __nv_bfloat16* q;  // [B, Hq, 128]
+  const __nv_bfloat16* q;  // V2: [B, Hq, 128]; V1 form: [B, Hkv, 128] (branch halves)
+  int v1;                  // V1 form: each KV head is one V1 head, seen as a pair of heads
   const int* lens;
   int max_len;
   int window;  // > 0: the query sees only the last `window` valid entries
@@ -139,15 +140,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     item_coords(p, item, b, g, t0, t1);
 
     // Q^T fragments (B operand, k = feature, n = head), 8 k-steps of 16.
+    // V1 form: head 0 of the pair is the query's first 64 features with zeros
+    // above, head 1 zeros below and the last 64, so that one K row of 128
+    // gives both branches' logits.
     uint32_t qf[8][2];
     {
       const bool valid = gq < p.group;
       const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          p.q + ((size_t)b * p.Hq + (size_t)g * p.group + (valid ? gq : 0)) * kD);
+          p.v1 ? p.q + ((size_t)b * p.Hkv + g) * kD
+               : p.q + ((size_t)b * p.Hq + (size_t)g * p.group + (valid ? gq : 0)) * kD);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        qf[ks][0] = valid ? __ldg(qrow + ks * 8 + qq) : 0u;
-        qf[ks][1] = valid ? __ldg(qrow + ks * 8 + 4 + qq) : 0u;
+        const bool use = valid && (!p.v1 || (gq == (ks >> 2)));
+        qf[ks][0] = use ? __ldg(qrow + ks * 8 + qq) : 0u;
+        qf[ks][1] = use ? __ldg(qrow + ks * 8 + 4 + qq) : 0u;
       }
     }
     float o[8][4];
@@ -328,6 +334,56 @@ __global__ void v2_decode_combine_kernel(const float* __restrict__ part_o,
   out[((size_t)b * Hp + pair) * kD + c] = __float2bfloat16_rn(r);
 }
 
+// V1 form: one block per (batch, head), 128 threads = channels.  Merges the
+// splits of the head's two branches, forms o = O1/l1 - lambda * O2/l2 and,
+// with the norm, y = o / sqrt(mean(o^2) + eps) * g * (1 - lambda_init).
+__global__ void v1_decode_combine_tc_kernel(const float* __restrict__ part_o,
+                                            const float* __restrict__ part_ml,
+                                            const float* __restrict__ lambda,
+                                            __nv_bfloat16* __restrict__ out, int H, int n_split,
+                                            int apply_norm, const float* __restrict__ gain,
+                                            float eps, float post_scale) {
+  __shared__ float red[kD / 32];
+  const int bh = blockIdx.x;
+  const int h = bh % H;
+  const int c = threadIdx.x;
+  float Ma = -INFINITY, Mb = -INFINITY;
+  for (int s = 0; s < n_split; ++s) {
+    const float* ml = part_ml + ((size_t)bh * n_split + s) * kHeads * 2;
+    Ma = fmaxf(Ma, ml[0]);
+    Mb = fmaxf(Mb, ml[2]);
+  }
+  float La = 0.f, Lb = 0.f, Oa = 0.f, Ob = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    const size_t it = (size_t)bh * n_split + s;
+    const float* ml = part_ml + it * kHeads * 2;
+    const float* po = part_o + it * kHeads * kD;
+    if (ml[0] != -INFINITY) {
+      const float f = ex2(ml[0] - Ma);
+      La = fmaf(ml[1], f, La);
+      Oa = fmaf(po[c], f, Oa);
+    }
+    if (ml[2] != -INFINITY) {
+      const float f = ex2(ml[2] - Mb);
+      Lb = fmaf(ml[3], f, Lb);
+      Ob = fmaf(po[kD + c], f, Ob);
+    }
+  }
+  float o = Oa / La - lambda[h] * (Ob / Lb);
+  if (apply_norm) {
+    float ss = o * o;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if ((c & 31) == 0) red[c >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kD / 32; ++w) tot += red[w];
+    o = o * (post_scale / sqrtf(tot * (1.0f / kD) + eps)) * (gain ? gain[c] : 1.f);
+  }
+  out[(size_t)bh * kD + c] = __float2bfloat16_rn(o);
+}
+
 }  // namespace
 
 V2DecodePlan plan_v2_decode(int batch, int n_kv_heads, int max_len, int num_sms) {
@@ -389,6 +445,7 @@ cudaError_t launch_v2_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, c
                              cudaStream_t stream) {
   Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.v1 = 0;
   p.lens = lens;
   p.max_len = max_len;
   p.window = window;
@@ -411,6 +468,40 @@ cudaError_t launch_v2_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, c
   v2_decode_combine_kernel<<<batch * n_kv_heads, (p.group / 2) * kD, 0, stream>>>(
       p.part_o, p.part_ml, lambda, static_cast<__nv_bfloat16*>(out), n_kv_heads, p.group,
       plan.n_split);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_v1_decode_tc(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
+                                const int* lens, int max_len, int window, void* out, int batch,
+                                int n_heads, const float* lambda, int apply_norm,
+                                const float* norm_weight, float eps, float post_scale,
+                                const V2DecodePlan& plan, void* workspace, int* dev_status,
+                                cudaStream_t stream) {
+  Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.v1 = 1;
+  p.lens = lens;
+  p.max_len = max_len;
+  p.window = window;
+  p.Hq = 2 * n_heads;
+  p.Hkv = n_heads;
+  p.group = 2;
+  p.split_len = plan.split_len;
+  p.n_split = plan.n_split;
+  p.n_items = plan.n_items;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(64.0));  // one branch is 64 wide
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = p.part_o + (size_t)plan.n_items * kHeads * kD;
+  p.dev_status = dev_status;
+  cudaError_t e = cudaFuncSetAttribute(v2_decode_split_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  v2_decode_split_kernel<<<plan.grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_v, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  v1_decode_combine_tc_kernel<<<batch * n_heads, kD, 0, stream>>>(
+      p.part_o, p.part_ml, lambda, static_cast<__nv_bfloat16*>(out), n_heads, plan.n_split,
+      apply_norm, norm_weight, eps, post_scale);
   return cudaGetLastError();
 }
 

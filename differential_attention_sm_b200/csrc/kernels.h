@@ -60,6 +60,17 @@ cudaError_t launch_v2_decode(const CUtensorMap& tm_k, const CUtensorMap& tm_v, c
                              const V2DecodePlan& plan,
                              void* workspace, int* dev_status, cudaStream_t stream);
 
+// V1 decode (bf16, d_qk 64, d_v 128) on the same split kernel: each head is a
+// KV head whose two branches are a pair (query features split by halves);
+// the combine applies -lambda, the per-head norm and the post scale.  The
+// workspace is v2_decode_workspace_bytes of plan_v2_decode(batch, n_heads, ...).
+cudaError_t launch_v1_decode_tc(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
+                                const int* lens, int max_len, int window, void* out, int batch,
+                                int n_heads, const float* lambda, int apply_norm,
+                                const float* norm_weight, float eps, float post_scale,
+                                const V2DecodePlan& plan, void* workspace, int* dev_status,
+                                cudaStream_t stream);
+
 // ---- V1 split-KV decode (bf16, d_qk 64, d_v 128) --------------------------
 struct V1DecodePlan {
   int n_split, split_len, n_items;
