@@ -71,19 +71,6 @@ cudaError_t launch_v1_decode_tc(const CUtensorMap& tm_k, const CUtensorMap& tm_v
                                 const V2DecodePlan& plan, void* workspace, int* dev_status,
                                 cudaStream_t stream);
 
-// ---- V1 split-KV decode (bf16, d_qk 64, d_v 128) --------------------------
-struct V1DecodePlan {
-  int n_split, split_len, n_items;
-};
-V1DecodePlan plan_v1_decode(int batch, int n_heads, int max_len, int num_sms);
-size_t v1_decode_workspace_bytes(const V1DecodePlan& plan);
-cudaError_t launch_v1_decode(const void* q, const void* k_cache, const void* v_cache,
-                             const int* lens, int max_len, int window, void* out, int batch,
-                             int n_heads, const float* lambda, int apply_norm,
-                             const float* norm_weight,
-                             float eps, float post_scale, const V1DecodePlan& plan,
-                             void* workspace, cudaStream_t stream);
-
 // 4-D bf16 tensor map (128-byte swizzle, zero fill) over a dense
 // [d3][d2][d1][d0] array; returns a da_status.  Implemented in api.cu.
 int make_tmap_bf16_4d(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,

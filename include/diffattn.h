@@ -212,7 +212,9 @@ DA_API size_t diffattn_v1_decode_workspace_size(int batch, int n_heads, int d_qk
  * v_cache : device [batch, max_len, n_heads, d_v]
  * out     : device [batch, n_heads, d_v]
  * Other arguments as for diffattn_v1_fwd and diffattn_v2_decode.
- * Supported: bf16 d_qk = 64, d_v = 128 on the split-KV kernel; other
+ * Supported: bf16 d_qk = 64, d_v = 128 on the TMA-fed split-KV kernel of
+ * diffattn_v2_decode, where a head's two branches are a pair of query heads
+ * (branch 1 scores on features 0..d_qk-1, branch 2 on the rest); other
  * widths (and fp32) with d_qk <= 128, d_v <= 256 on the CUDA-core kernel. */
 DA_API int diffattn_v1_decode(const void* q, const void* k_cache, const void* v_cache,
                        const int* cache_lens, int max_len, void* out, da_dtype dtype,
