@@ -20,20 +20,24 @@
 // maxima and normalisers differ; the subtraction happens in the epilogue:
 //     o = O1 / l1 - lambda * O2 / l2   (then, V1 only, RMS norm * g * (1 - lambda_init)).
 //
-// Warp roles (416 threads):
+// Warp roles (V2: 13 warps; V1: 12, with one score issuer for both branches):
 //   warps 0-3  softmax for branch 1 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax for branch 2
 //   warp  8    TMA producer (Q per tile; K and V tiles through 4-stage rings;
 //              requests the next tile)
 //   warp  9    issues branch 1's score MMAs (Q1.K^T); owns the tensor memory
-//   warp 10    issues branch 2's score MMAs (Q2.K^T)
-//   warp 11    issues branch 1's P1.V MMAs
-//   warp 12    issues branch 2's P2.V MMAs
+//   warp 10    issues branch 2's score MMAs (Q2.K^T)           (V2 only)
+//   then       one warp per branch issuing its P_r.V MMAs
+// V1 gives both branches' score MMAs (64-wide, 4 k-steps each) to warp 9:
+// with 12 warps no sub-partition holds more than three, so the softmax
+// threads get 168 registers instead of the 128 that four warps leave, and
+// the V1 softmax runs without the spills and re-loads the cap forced.  V2's
+// score products are twice as long and keep an issuer per branch.
 // tcgen05.mma issue runs at the tensor pipe's pace and every commit and
-// barrier poll costs the issuing thread time, so each of the four MMA
-// streams has its own thread: P_r(j).V goes out as soon as P_r(j) is ready,
-// and S_r(j+2) as soon as that P.V has freed its buffer, without either
-// waiting behind the other's bookkeeping.
+// barrier poll costs the issuing thread time, so the P.V streams have a
+// thread each: P_r(j).V goes out as soon as P_r(j) is ready, and S_r(j+2)
+// as soon as that P.V has freed its buffer, without waiting behind the
+// other stream's bookkeeping.
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
 // Causal masking is applied only on the tiles that cross the diagonal (and
@@ -73,7 +77,9 @@ namespace {
 
 constexpr int kBM = 128;                   // query rows per CTA
 constexpr int kBN = 64;                    // keys per KV tile
-constexpr int kThreads = 416;
+// score-MMA issuer warps and threads per CTA, by form
+__host__ __device__ constexpr int score_issuers(int form) { return form == 1 ? 1 : 2; }
+__host__ __device__ constexpr int cta_threads(int form) { return (11 + score_issuers(form)) * 32; }
 constexpr int kQBox = kBM * 64 * 2;        // TMA box of Q: 128 rows x 64 bf16 = 16 KB
 constexpr int kQTile = 2 * kQBox;          // one 128 x 128 query tile
 constexpr int kKVBox = kBN * 64 * 2;       // TMA box of K/V: 64 rows x 64 bf16 = 8 KB
@@ -102,9 +108,11 @@ struct Barriers {
   int abort_flag;
 };
 
-// Arrivals that release a tile-number buffer: the two score issuers, the two
+// Arrivals that release a tile-number buffer: the score issuer(s), the two
 // P.V issuers and the eight softmax warps.
-constexpr uint32_t kTileReaders = 12;
+__host__ __device__ constexpr uint32_t tile_readers(int form) {
+  return 10u + (uint32_t)score_issuers(form);
+}
 
 struct Params {
   int form;
@@ -263,7 +271,7 @@ __device__ __forceinline__ int read_tile(Barriers* bars, int tc, int* dev_status
 // kWindow: sliding-window masking compiled in (p.window > 0) or out.
 // kSave: also write the training saves p.lse and p.obr.
 template <int kForm, bool kWindow, bool kSave>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(cta_threads(kForm), 1)
     diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -305,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(&bars->t_full[u], 1);
-      mbar_init(&bars->t_empty[u], kTileReaders);
+      mbar_init(&bars->t_empty[u], tile_readers(kForm));
     }
     mbar_init(&bars->clc_full, 1);
     bars->abort_flag = 0;
@@ -384,10 +392,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 9 || warp == 10) {
-    // ------------- score MMA issuer of branch r = warp - 9: S_r(j) = Q_r . K(j)^T -------------
+  } else if (warp >= 9 && warp < 9 + score_issuers(kForm)) {
+    // ------ score MMA issuer: S_r(j) = Q_r . K(j)^T for branch r = warp - 9 (V2),
+    // ------ or for both branches (V1)
     if (lane == 0) {
-      const int r = warp - 9;
+      const int r0 = score_issuers(kForm) == 1 ? 0 : warp - 9;
+      const int r1 = score_issuers(kForm) == 1 ? 2 : r0 + 1;
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const int nk = kForm == 1 ? 4 : 8;  // 16-wide k-steps of Q.K^T
@@ -401,35 +411,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < T.n_kv; ++j, ++J) {
           const int s = J % kStages;
           if (!mbar_wait(&bars->k_full[s], (J / kStages) & 1u, p.dev_status, &failed)) break;
-          // buffer J % 2 last held P_r(J-2): its P.V must have completed
-          if (J >= 2 && !mbar_wait(&bars->o_done[r][J & 1], ((J - 2) >> 1) & 1u, p.dev_status,
-                                   &failed))
-            break;
-          tc_fence_after();
           const uint32_t kt = k_addr + s * kKVTile;
-          for (int kk = 0; kk < nk; ++kk) {
-            uint32_t a, bb;
-            if (kForm == 1) {  // branch r = columns [64 r, 64 r + 64)
-              a = q_addr + r * kQBox + kk * 32;
-              bb = kt + r * kKVBox + kk * 32;
-            } else {            // branch r = query head 2p + r, full 128 columns
-              a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
-              bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
+          for (int r = r0; r < r1; ++r) {
+            // buffer J % 2 last held P_r(J-2): its P.V must have completed
+            if (J >= 2 && !mbar_wait(&bars->o_done[r][J & 1], ((J - 2) >> 1) & 1u,
+                                     p.dev_status, &failed))
+              break;
+            tc_fence_after();
+            for (int kk = 0; kk < nk; ++kk) {
+              uint32_t a, bb;
+              if (kForm == 1) {  // branch r = columns [64 r, 64 r + 64)
+                a = q_addr + r * kQBox + kk * 32;
+                bb = kt + r * kKVBox + kk * 32;
+              } else {            // branch r = query head 2p + r, full 128 columns
+                a = q_addr + r * kQTile + (kk >> 2) * kQBox + (kk & 3) * 32;
+                bb = kt + (kk >> 2) * kKVBox + (kk & 3) * 32;
+              }
+              tc_mma_ss(tmem + s_col(r, J & 1), smem_desc_sw128(a, 16, 1024),
+                        smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
             }
-            tc_mma_ss(tmem + s_col(r, J & 1), smem_desc_sw128(a, 16, 1024),
-                      smem_desc_sw128(bb, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+            tc_commit(&bars->s_full[r][J & 1]);
+            tc_commit(&bars->k_empty[s]);  // one of the two releases of this K stage
           }
-          tc_commit(&bars->s_full[r][J & 1]);
-          tc_commit(&bars->k_empty[s]);
+          if (failed) break;
         }
         if (failed) break;
-        tc_commit(&bars->q_empty);  // Q free once this branch's score MMAs are done
+        // Q free once both branches' score MMAs are done (one release each)
+        for (int r = r0; r < r1; ++r) tc_commit(&bars->q_empty);
       }
     }
-  } else if (warp == 11 || warp == 12) {
-    // ------------- P.V MMA issuer of branch r = warp - 11: O_r += P_r(j) . V(j) -------------
+  } else if (warp == 9 + score_issuers(kForm) || warp == 10 + score_issuers(kForm)) {
+    // ------- P.V MMA issuer of branch r: O_r += P_r(j) . V(j) -------
     if (lane == 0) {
-      const int r = warp - 11;
+      const int r = warp - 9 - score_issuers(kForm);
       const uint32_t v_addr = smem_u32(sV);
       const uint32_t pcol0 = tmem + s_col(r, 0);
       const uint32_t ocol = tmem + (r == 0 ? kColO1 : kColO2);
@@ -829,7 +843,7 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   const long long grid = (long long)p.n_qtiles * bh_count;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   p.n_tiles = (int)grid;
-  kern<<<(unsigned)grid, kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
+  kern<<<(unsigned)grid, cta_threads(a.form), smem, stream>>>(tm_q, tm_k, tm_v, p);
   return cudaGetLastError();
 }
 
