@@ -15,17 +15,18 @@
 //
 // Two kernels:
 //   * dq kernel, one CTA per 128 query rows of a head (V1) or head pair
-//     (V2), walking 64-key tiles like the forward: per branch, S_r and dP_r
-//     into tensor memory (two SS MMAs), dS_r written as bf16 by the
-//     softmax-backward warps, then dQ_r += dS_r K_r in tensor memory.  V1
+//     (V2), walking 64-key tiles like the forward: per branch, S_r into
+//     tensor memory (SS MMA); one dP = do_1 V^T for both branches, since
+//     do_2 = -lambda do_1 makes dP_2 = -lambda dP_1; dS_r written as bf16 by
+//     the softmax-backward warps, then dQ_r += dS_r K_r in tensor memory.  V1
 //     writes dS_r back over S_r (TS MMA); V2, whose tensor memory has no
 //     second S buffer, writes it to swizzled shared memory (SS MMA) so that
 //     S_r(j+1) only waits for S_r(j) to be loaded.  The softmax-backward
-//     warps form P as soon as S_r has landed and wait for dP_r only after
+//     warps form P as soon as S_r has landed and wait for dP only after
 //     that.  Warps: 0-15 softmax backward (thread = query row; two
 //     warpgroups per branch, one per half of the tile's 64 key columns),
-//     16 TMA producer, 17-20 the S_r and dP_r issuers (one thread per product
-//     stream, as in the forward), 21 / 22 dQ issuers.
+//     16 TMA producer, 17 / 19 the S_1 / S_2 issuers and 18 the dP issuer
+//     (one thread per product stream, as in the forward), 20 / 21 dQ issuers.
 //   * dkdv kernel, one CTA per 128 keys of a head (V1) or KV head (V2),
 //     walking 64-query tiles (and, for V2, every pair that reads the KV
 //     head): S^T = K_r Q_r^T and dP^T = V do_r^T (SS), P^T and dS^T written
@@ -64,6 +65,7 @@ struct BwdParams {
   float scale;       // 1 / sqrt(d)
   const float* lse;  // [B][units][2][npad]: p = 2^(s * scale_log2 - lse)
   const float* Dv;   // [B][units][2][npad]: D_r = do_r . O_r
+  const float* lambda;  // [units]: do_2 = -lambda do_1, so dP_2 = -lambda dP_1
   float* dq;         // like q
   float* dk;         // like k
   float* dv;         // like v
@@ -75,9 +77,9 @@ struct BwdParams {
 
 // ===================================================================== dQ
 // warps 0-15: softmax backward (branch r = (warp >> 2) & 1, key-column half
-// h = warp >> 3); 16 producer; 17-20 the S_r and dP_r issuers (17 owns tensor
-// memory); 21 / 22 the dQ_1 / dQ_2 issuers
-constexpr int kDqThreads = 736;
+// h = warp >> 3); 16 producer; 17 / 19 the S_1 / S_2 issuers and 18 the dP
+// issuer (17 owns tensor memory); 20 / 21 the dQ_1 / dQ_2 issuers
+constexpr int kDqThreads = 704;
 constexpr int kDqProducer = 16;
 constexpr int kDqStages = 2;
 
@@ -86,7 +88,7 @@ struct DqBarriers {
   uint64_t k_full[kDqStages], k_empty[kDqStages];
   uint64_t v_full[kDqStages], v_empty[kDqStages];
   uint64_t s_full[2][2];   // [branch][S buffer]: S_r landed
-  uint64_t dp_full[2];     // [branch]: dP_r landed
+  uint64_t dp_full[2];     // [0]: dP_1 landed (dP_2 = -lambda dP_1; [1] unused)
   uint64_t ds_full[2][2];  // [branch][column half]: dS_r written back (and dP_r read)
   uint64_t dq_done[2][2];  // [branch][S buffer]: the dQ product of a tile has read its dS
   uint64_t s_free[2];      // [branch], V2: the softmax backward has loaded S_r
@@ -106,8 +108,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sdO = sQ + kQBytes;                     // 2 branches x 128 x 128
-  uint8_t* sK = sdO + 2 * kTile128;                // stages x 64 x 128
+  uint8_t* sdO = sQ + kQBytes;                     // do_1: 128 x 128
+  uint8_t* sK = sdO + kTile128;                    // stages x 64 x 128
   uint8_t* sV = sK + kDqStages * kTile64;
   // V2: dS_r (128 queries x 64 keys bf16, 128-byte swizzle, K-major) per branch
   uint8_t* sDS = sV + kDqStages * kTile64;
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 4);  // both branches' S and dQ products read K
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 2);
+      mbar_init(&bars->v_empty[s], 1);  // the one dP product reads V
     }
     for (int r = 0; r < 2; ++r) {
       mbar_init(&bars->s_full[r][0], 1);
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, kQBytes + 2 * kTile128);
+      mbar_arrive_expect_tx(&bars->q_full, kQBytes + kTile128);
       if (kForm == 1) {
         tma_load_4d(sQ, &tm_q, &bars->q_full, 0, hh, q0, b);
         tma_load_4d(sQ + kBox128, &tm_q, &bars->q_full, 64, hh, q0, b);
@@ -181,10 +183,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           tma_load_4d(sQ + r * kTile128 + kBox128, &tm_q, &bars->q_full, 64, 2 * hh + r, q0, b);
         }
       }
-      for (int r = 0; r < 2; ++r) {
-        tma_load_4d(sdO + r * kTile128, &tm_do, &bars->q_full, 0, 2 * hh + r, q0, b);
-        tma_load_4d(sdO + r * kTile128 + kBox128, &tm_do, &bars->q_full, 64, 2 * hh + r, q0, b);
-      }
+      tma_load_4d(sdO, &tm_do, &bars->q_full, 0, 2 * hh, q0, b);
+      tma_load_4d(sdO + kBox128, &tm_do, &bars->q_full, 64, 2 * hh, q0, b);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kDqStages;
         const uint32_t ph = (uint32_t)(j / kDqStages) & 1u;
@@ -199,10 +199,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tma_load_4d(sV + s * kTile64 + kBox64, &tm_v, &bars->v_full[s], 64, kvh, row, b);
       }
     }
-  } else if (warp >= kDqProducer + 1 && warp <= kDqProducer + 4) {
-    if (lane == 0) {  // ---- S_r issuer (kind 0) or dP_r issuer (kind 1): warp 17 + 2r + kind
-      const int r = (warp - kDqProducer - 1) >> 1, kind = (warp - kDqProducer - 1) & 1;
-      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO) + r * kTile128;
+  } else if (warp >= kDqProducer + 1 && warp <= kDqProducer + 3) {
+    // ---- S_r issuer (kind 0, warp 17 + 2r) or the dP issuer (kind 1, warp 18):
+    // dP_2 = -lambda dP_1, so only branch 1's dP product is computed
+    const int r = (warp - kDqProducer - 1) >> 1, kind = (warp - kDqProducer - 1) & 1;
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO);
       constexpr uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       if (mbar_wait(&bars->q_full, 0, p.dev_status, &failed)) {
         for (int j = 0; j < n_kv; ++j) {
@@ -221,9 +223,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           if (kForm == 2 && kind == 0 && j >= 1 &&
               !mbar_wait(&bars->s_free[r], (uint32_t)(j - 1) & 1u, p.dev_status, &failed))
             break;
+          // dP's buffer is free once both branches' softmax backward has read dP(j-1)
           if (kind == 1 && j > 0 &&
-              !(mbar_wait(&bars->ds_full[r][0], (uint32_t)(j - 1) & 1u, p.dev_status, &failed) &&
-                mbar_wait(&bars->ds_full[r][1], (uint32_t)(j - 1) & 1u, p.dev_status, &failed)))
+              !(mbar_wait(&bars->ds_full[0][0], (uint32_t)(j - 1) & 1u, p.dev_status, &failed) &&
+                mbar_wait(&bars->ds_full[0][1], (uint32_t)(j - 1) & 1u, p.dev_status, &failed) &&
+                mbar_wait(&bars->ds_full[1][0], (uint32_t)(j - 1) & 1u, p.dev_status, &failed) &&
+                mbar_wait(&bars->ds_full[1][1], (uint32_t)(j - 1) & 1u, p.dev_status, &failed)))
             break;
           tc_fence_after();
           if (kind == 0) {
@@ -247,18 +252,18 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t a = do_addr + (kk >> 2) * kBox128 + (kk & 3) * 32;
               const uint32_t bb = vt + (kk >> 2) * kBox64 + (kk & 3) * 32;
-              tc_mma_ss(tmem + colP(r), smem_desc_sw128(a, 16, 1024),
+              tc_mma_ss(tmem + colP(0), smem_desc_sw128(a, 16, 1024),
                         smem_desc_sw128(bb, 16, 1024), idS, kk > 0 ? 1u : 0u);
             }
-            tc_commit(&bars->dp_full[r]);
+            tc_commit(&bars->dp_full[0]);
             tc_commit(&bars->v_empty[s]);
           }
         }
       }
     }
-  } else if (warp == kDqProducer + 5 || warp == kDqProducer + 6) {
-    if (lane == 0) {  // ------------------------------------ dQ_r issuer, r = warp - 21
-      const int r = warp - kDqProducer - 5;
+  } else if (warp == kDqProducer + 4 || warp == kDqProducer + 5) {
+    if (lane == 0) {  // ------------------------------------ dQ_r issuer, r = warp - 20
+      const int r = warp - kDqProducer - 4;
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, false, true);
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % kDqStages;
@@ -305,6 +310,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const float Dr = qrow < p.seqlen ? p.Dv[vrow] : 0.f;
     const float sc = p.scale_log2;
     const uint64_t sc2 = f2pack(sc, sc), nl2 = f2pack(-lse, -lse), nd2 = f2pack(-Dr, -Dr);
+    const float mr = r == 0 ? 1.f : -p.lambda[hh];  // dP_r = mr dP_1
+    const uint64_t mr2 = f2pack(mr, mr);
     // Two passes per tile: P = 2^(s sc - lse) as soon as S_r has landed (the
     // dP_r product may still be in flight), then dS = P (dP - D) from the same
     // P, kept in registers as bf16 pairs, written back over S_r.
@@ -343,7 +350,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           pp[e] = pack_bf16(p0, p1);
         }
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full[r], (uint32_t)j & 1u, p.dev_status,
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->dp_full[0], (uint32_t)j & 1u, p.dev_status,
                                              &failed))) {
         failed = true;
         break;
@@ -360,15 +367,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       tc_fence_after();
       {
         uint32_t dp[32], pk[16];
-        tmem_ld32(tmem + lane_off + colP(r) + 32 * h, dp);
+        tmem_ld32(tmem + lane_off + colP(0) + 32 * h, dp);
         tc_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const uint32_t pb = pp[e];
           float ds0, ds1;
           f2unpack(fma2(f2pack(bf16lo(pb), bf16hi(pb)),
-                        add2(f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
-                             nd2),
+                        fma2(f2pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                             mr2, nd2),
                         0ull),
                    ds0, ds1);
           pk[e] = pack_bf16(ds0, ds1);
@@ -1027,6 +1034,7 @@ cudaError_t launch_bwd_from_saves(const FusedBwdArgs& a, const void* saves, cuda
   p.scale = (float)(1.0 / std::sqrt(d));
   p.lse = lse;
   p.Dv = Dv;
+  p.lambda = a.fwd.lambda;
   p.dq = a.dq;
   p.dk = a.dk;
   p.dv = a.dv;
@@ -1039,7 +1047,7 @@ cudaError_t launch_bwd_from_saves(const FusedBwdArgs& a, const void* saves, cuda
   // dQ
   {
     const int qbytes = a.fwd.form == 1 ? kTile128 : 2 * kTile128;
-    const int smem = 1024 + qbytes + 2 * kTile128 + 2 * kDqStages * kTile64 +
+    const int smem = 1024 + qbytes + kTile128 + 2 * kDqStages * kTile64 +
                      (a.fwd.form == 2 ? 2 * kBox128 : 0) + (int)sizeof(DqBarriers) + 64;
     decltype(&diffattn_bwd_dq_kernel<1, false>) k =
         a.fwd.form == 1 ? (win ? diffattn_bwd_dq_kernel<1, true> : diffattn_bwd_dq_kernel<1, false>)
