@@ -594,11 +594,10 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
                                      sc2, nu2);
             float x0, x1, p0, p1;
             f2unpack(x2, x0, x1);
-            // Share of exponentials on the polynomial: V1's shorter Q.K^T leaves
-            // the softmax the critical path, so it offloads more: three pairs in
-            // sixteen, spread over the row, against one in eight for V2 (both
-            // shares and positions measured).
-            if (kForm == 1 ? (e == 2 || e == 7 || e == 12) : (e & 7) == 7) {
+            // Share of exponentials on the polynomial (both shares and positions
+            // measured): one pair in sixteen for V1, whose softmax has 168
+            // registers at 12 warps, one in eight for V2 at 13 warps.
+            if (kForm == 1 ? e == 3 : (e & 7) == 7) {
               exp2_poly2(x0, x1, p0, p1);
             } else {
               p0 = ex2(x0);
