@@ -38,6 +38,9 @@
 // thread each: P_r(j).V goes out as soon as P_r(j) is ready, and S_r(j+2)
 // as soon as that P.V has freed its buffer, without waiting behind the
 // other stream's bookkeeping.
+// The V1 epilogue writes each softmax warp's 32 output rows through a 4 KB
+// shared-memory block and one TMA tensor store (V2's shared memory has no
+// room for the 32 KB; it stores from registers).
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
 // Causal masking is applied only on the tiles that cross the diagonal (and
@@ -77,6 +80,9 @@ namespace {
 
 constexpr int kBM = 128;                   // query rows per CTA
 constexpr int kBN = 64;                    // keys per KV tile
+// Output staged through shared memory (V1 without training saves: V2's
+// shared memory has no room for the 32 KB)
+__host__ __device__ constexpr bool stage_out(int form, bool save) { return form == 1 && !save; }
 // score-MMA issuer warps and threads per CTA, by form
 __host__ __device__ constexpr int score_issuers(int form) { return form == 1 ? 1 : 2; }
 __host__ __device__ constexpr int cta_threads(int form) { return (11 + score_issuers(form)) * 32; }
@@ -274,7 +280,8 @@ template <int kForm, bool kWindow, bool kSave>
 __global__ void __launch_bounds__(cta_threads(kForm), 1)
     diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
-                               const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                               const __grid_constant__ CUtensorMap tm_v,
+                               const __grid_constant__ CUtensorMap tm_o, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -285,6 +292,11 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
   Barriers* bars = reinterpret_cast<Barriers*>(sV + kStages * kKVTile);
   float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [tile parity][2][128]
   float* x_ss = x_inv_l + 4 * kBM;                       // [tile parity][2][128]
+  // output staging (V1 without saves): per softmax warp, its 32 rows x 64 bf16
+  // (128-byte rows, the 16-byte chunks of row t at positions c ^ (t & 7));
+  // 1024-byte aligned, as the 128-byte swizzle of the TMA box requires
+  uint8_t* x_out = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(x_ss + 4 * kBM) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -701,7 +713,42 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
         const float tot = ssq[row] + ssq[kBM + row];
         mul = p.post_scale / sqrtf(tot * (1.0f / 128.0f) + p.eps);
       }
-      if (qrow < p.seqlen && !stop && !failed) {
+      if constexpr (stage_out(kForm, kSave)) {
+        // V1: the warp's 32 rows leave by one TMA tensor store from its
+        // staging block (128-byte swizzled, the layout of the output map's
+        // box).  Stored directly, each thread's 16-byte stores (rows 4 KB
+        // apart) would still be draining when the next tile's first P is
+        // released, and that release waits for them; the bulk store is
+        // outside that ordering.  Rows past the sequence end are clipped by
+        // the map.
+        uint8_t* wst = x_out + warp * 4096;
+        if (lane == 0) bulk_wait_read();  // the previous tile's store has read the block
+        __syncwarp();
+#pragma unroll
+        for (int v8 = 0; v8 < 8; ++v8) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = v8 * 8 + e;
+            const float gm = (p.apply_norm && p.norm_weight) ? __ldg(p.norm_weight + 64 * r + c)
+                                                             : 1.f;
+            y[e] = o[c] * mul * gm;
+          }
+          uint4 w;
+          w.x = pack_bf16(y[0], y[1]);
+          w.y = pack_bf16(y[2], y[3]);
+          w.z = pack_bf16(y[4], y[5]);
+          w.w = pack_bf16(y[6], y[7]);
+          *reinterpret_cast<uint4*>(wst + lane * 128 + ((v8 ^ (lane & 7)) << 4)) = w;
+        }
+        fence_proxy_async_smem();  // visible to the tensor-memory-access unit
+        __syncwarp();
+        const bool write = __all_sync(0xffffffffu, !failed) && !stop;
+        if (lane == 0 && write) {
+          tma_store_4d(&tm_o, wst, 64 * r, T.hh, T.q0 + sub * 32, T.b);
+          bulk_commit();
+        }
+      } else if (qrow < p.seqlen && !stop && !failed) {
         __nv_bfloat16* dst =
             p.out + (((size_t)T.b * p.seqlen + qrow) * p.heads + T.hh) * 128 + 64 * r;
 #pragma unroll
@@ -727,6 +774,7 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
   }
 
   // ---- teardown: every role reaches this point, then TMEM is released ----
+  if (stage_out(kForm, kSave) && warp < 8 && lane == 0) bulk_wait_all();
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -823,7 +871,8 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.dev_status = a.dev_status;
   const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
   const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +
-                   8 * kBM * (int)sizeof(float) + 64;
+                   8 * kBM * (int)sizeof(float) +
+                   (stage_out(a.form, a.lse && a.obr) ? 8 * 4096 + 1024 : 0) + 64;
   const bool win = a.window > 0;
   decltype(&diffattn_prefill_tc_kernel<1, false, false>) kern;
   if (a.lse && a.obr)  // training forward
@@ -842,7 +891,14 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   const long long grid = (long long)p.n_qtiles * bh_count;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   p.n_tiles = (int)grid;
-  kern<<<(unsigned)grid, cta_threads(a.form), smem, stream>>>(tm_q, tm_k, tm_v, p);
+  // output [B][N][heads][128] in boxes of 64 columns x 32 rows, for the
+  // instantiations that store through shared memory (unused by the others)
+  CUtensorMap tm_o = tm_q;
+  if (stage_out(a.form, a.lse && a.obr) &&
+      make_tmap_bf16_4d(&tm_o, a.out, 128, (uint64_t)a.heads, (uint64_t)a.seqlen,
+                        (uint64_t)a.batch, 64, 1, 32, 1) != 0)
+    return cudaErrorInvalidValue;
+  kern<<<(unsigned)grid, cta_threads(a.form), smem, stream>>>(tm_q, tm_k, tm_v, tm_o, p);
   return cudaGetLastError();
 }
 

@@ -247,6 +247,28 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const void* desc, uint64_
       : "memory");
 }
 
+// Tiled bulk store shared -> global, tracked by bulk groups.  Coordinates
+// must be non-negative; the tensor map clips what lies past its bounds.
+__device__ __forceinline__ void tma_store_4d(const void* desc, const void* src, int c0, int c1,
+                                             int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::
+          "l"(desc),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// This thread's bulk stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// This thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // warp-level MMA helpers (m16n8k16 bf16 -> fp32), ldmatrix, movmatrix
 // ---------------------------------------------------------------------------
