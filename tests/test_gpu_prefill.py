@@ -93,6 +93,30 @@ def test_v1_bf16_small(B, Bn, N, H, causal):
     assert_bf16_close(out.reshape(-1, dv), ref, False, "v1 bf16 N=%d" % N)
 
 
+@pytest.mark.parametrize("offset_bytes", [16, 32])
+def test_v1_bf16_output_offset(B, offset_bytes):
+    """The output may start at any 16-byte boundary: the V1 kernel writes it by
+    TMA tensor stores, whose map takes the caller's base as given.  Rows past
+    the ragged end must not be written, nor anything around the output."""
+    Bn, N, H, d, dv = 2, 300, 3, 64, 128
+    x = I.v1_inputs(Bn, N, H, d, dv, seed=31, dtype=torch.bfloat16)
+    lam = torch.tensor([0.4, -0.6, 1.3], dtype=torch.float32)
+    n = Bn * N * H * dv
+    pad = offset_bytes // 2
+    buf = torch.full((n + 2 * pad + 64,), -7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[pad:pad + n].view(Bn, N, H, dv)
+    assert out.data_ptr() % 16 == 0
+    st = status_word()
+    B.diffattn_v1_fwd(cuda(x["q"]), cuda(x["k"]), cuda(x["v"]), cuda(lam), causal=True,
+                      apply_norm=True, lambda_init=0.3, out=out, dev_status=st)
+    assert_status_ok(st)
+    torch.cuda.synchronize()
+    assert (buf[:pad] == -7.0).all() and (buf[pad + n:] == -7.0).all(), "write outside the output"
+    ref = O.v1_rows(x["q"], x["k"], x["v"], lam.double().numpy(), np.arange(Bn * N * H),
+                    causal=True, apply_norm=True, lambda_init_value=0.3)
+    assert_bf16_close(out.reshape(-1, dv), ref, False, "v1 bf16 output at +%d bytes" % offset_bytes)
+
+
 def test_v1_bf16_no_norm_and_gain(B):
     Bn, N, H, d, dv = 1, 257, 2, 64, 128
     x = I.v1_inputs(Bn, N, H, d, dv, seed=7, dtype=torch.bfloat16)
