@@ -87,6 +87,19 @@ int make_tmap_bf16_4d(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d
                       uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
   return make_tmap_4d(tm, base, d0, d1, d2, d3, b0, b1, b2, b3);
 }
+int make_tmap_f32_4d(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return DA_ERR_CUDA;
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0 * 4, d0 * d1 * 4, d0 * d1 * d2 * 4};
+  cuuint32_t box[4] = {b0, b1, b2, b3};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DA_OK : DA_ERR_CUDA;
+}
 }  // namespace da
 
 extern "C" {

@@ -75,6 +75,9 @@ cudaError_t launch_v1_decode_tc(const CUtensorMap& tm_k, const CUtensorMap& tm_v
 // [d3][d2][d1][d0] array; returns a da_status.  Implemented in api.cu.
 int make_tmap_bf16_4d(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                       uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3);
+// The same over fp32 elements, without swizzle (boxes of 32-byte rows).
+int make_tmap_f32_4d(CUtensorMap* tm, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3);
 
 // ---- tcgen05 prefill (bf16) -----------------------------------------------
 // Form 1 (V1): Q/K rows are 128 wide (two 64-wide branches), V 128 wide,

@@ -38,9 +38,10 @@
 // thread each: P_r(j).V goes out as soon as P_r(j) is ready, and S_r(j+2)
 // as soon as that P.V has freed its buffer, without waiting behind the
 // other stream's bookkeeping.
-// The V1 epilogue writes each softmax warp's 32 output rows through a 4 KB
-// shared-memory block and one TMA tensor store (V2's shared memory has no
-// room for the 32 KB; it stores from registers).
+// The V1 epilogue writes each softmax warp's 32 output rows (and in the
+// training forward its saved fp32 branch outputs, 8 columns at a time)
+// through a 4 KB shared-memory block and TMA tensor stores (V2's shared
+// memory has no room for the 32 KB; it stores from registers).
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
 // Causal masking is applied only on the tiles that cross the diagonal (and
@@ -81,9 +82,10 @@ namespace {
 
 constexpr int kBM = 128;                   // query rows per CTA
 constexpr int kBN = 64;                    // keys per KV tile
-// Output staged through shared memory (V1 without training saves: V2's
-// shared memory has no room for the 32 KB)
-__host__ __device__ constexpr bool stage_out(int form, bool save) { return form == 1 && !save; }
+// Output (and, for the training forward, the saved branch outputs) staged
+// through shared memory and written by TMA stores: V1 only, V2's shared
+// memory has no room for the 32 KB
+__host__ __device__ constexpr bool stage_out(int form, bool save) { return form == 1; }
 // score-MMA issuer warps and threads per CTA, by form
 __host__ __device__ constexpr int score_issuers(int form) { return form == 1 ? 1 : 2; }
 __host__ __device__ constexpr int cta_threads(int form) { return (11 + score_issuers(form)) * 32; }
@@ -282,7 +284,8 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
     diffattn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v,
-                               const __grid_constant__ CUtensorMap tm_o, const Params p) {
+                               const __grid_constant__ CUtensorMap tm_o,
+                               const __grid_constant__ CUtensorMap tm_obr, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -293,7 +296,7 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
   Barriers* bars = reinterpret_cast<Barriers*>(sV + kStages * kKVTile);
   float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [tile parity][2][128]
   float* x_ss = x_inv_l + 4 * kBM;                       // [tile parity][2][128]
-  // output staging (V1 without saves): per softmax warp, its 32 rows x 64 bf16
+  // output staging (V1): per softmax warp, its 32 rows x 64 bf16
   // (128-byte rows, the 16-byte chunks of row t at positions c ^ (t & 7));
   // 1024-byte aligned, as the 128-byte swizzle of the TMA box requires
   uint8_t* x_out = reinterpret_cast<uint8_t*>(
@@ -685,7 +688,40 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
 #pragma unroll
           for (int e = 0; e < kEC; ++e)
             o[ch * kEC + e] = __uint_as_float(a[e]) * inv1 - __uint_as_float(c2[e]) * inv2;
-          if (kSave && qrow < p.seqlen) {  // normalised branch outputs, fp32
+          if constexpr (kSave && stage_out(kForm, kSave)) {
+            // normalised branch outputs, fp32, by TMA stores: this chunk's 8
+            // columns of O_1/l_1 and of O_2/l_2 for the warp's 32 rows (1 KB
+            // each) go through one half of the warp's staging block, the
+            // halves alternating; a half is reused once the store of two
+            // chunks ago has read it
+            uint8_t* half = x_out + warp * 4096 + (ch & 1) * 2048;
+            if (lane == 0) {
+              if (ch == 0) bulk_wait_read(); else bulk_wait_read_1();
+            }
+            __syncwarp();
+            float* s1 = reinterpret_cast<float*>(half) + lane * kEC;
+            float* s2 = reinterpret_cast<float*>(half + 1024) + lane * kEC;
+#pragma unroll
+            for (int v4 = 0; v4 < kEC / 4; ++v4) {
+              *reinterpret_cast<float4*>(s1 + 4 * v4) =
+                  make_float4(__uint_as_float(a[4 * v4]) * inv1, __uint_as_float(a[4 * v4 + 1]) * inv1,
+                              __uint_as_float(a[4 * v4 + 2]) * inv1,
+                              __uint_as_float(a[4 * v4 + 3]) * inv1);
+              *reinterpret_cast<float4*>(s2 + 4 * v4) = make_float4(
+                  __uint_as_float(c2[4 * v4]) * inv2_raw, __uint_as_float(c2[4 * v4 + 1]) * inv2_raw,
+                  __uint_as_float(c2[4 * v4 + 2]) * inv2_raw,
+                  __uint_as_float(c2[4 * v4 + 3]) * inv2_raw);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            const bool wr = __all_sync(0xffffffffu, !failed) && !stop;
+            if (lane == 0 && wr) {
+              tma_store_4d(&tm_obr, half, 64 * r + kEC * ch, T.hh, T.q0 + sub * 32, T.b);
+              tma_store_4d(&tm_obr, half + 1024, 128 + 64 * r + kEC * ch, T.hh, T.q0 + sub * 32,
+                           T.b);
+              bulk_commit();
+            }
+          } else if (kSave && qrow < p.seqlen) {  // normalised branch outputs, fp32
             float* ob = p.obr + (((size_t)T.b * p.seqlen + qrow) * p.heads + T.hh) * 256 +
                         64 * r + kEC * ch;
 #pragma unroll
@@ -902,7 +938,13 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
       make_tmap_bf16_4d(&tm_o, a.out, 128, (uint64_t)a.heads, (uint64_t)a.seqlen,
                         (uint64_t)a.batch, 64, 1, 32, 1) != 0)
     return cudaErrorInvalidValue;
-  kern<<<(unsigned)grid, cta_threads(a.form), smem, stream>>>(tm_q, tm_k, tm_v, tm_o, p);
+  // training saves O_r / l_r [B][N][heads][256] fp32 in boxes of 8 columns x 32 rows
+  CUtensorMap tm_obr = tm_q;
+  if (a.lse && a.obr && stage_out(a.form, true) &&
+      make_tmap_f32_4d(&tm_obr, a.obr, 256, (uint64_t)a.heads, (uint64_t)a.seqlen,
+                       (uint64_t)a.batch, 8, 1, 32, 1) != 0)
+    return cudaErrorInvalidValue;
+  kern<<<(unsigned)grid, cta_threads(a.form), smem, stream>>>(tm_q, tm_k, tm_v, tm_o, tm_obr, p);
   return cudaGetLastError();
 }
 
