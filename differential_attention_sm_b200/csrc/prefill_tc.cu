@@ -40,8 +40,9 @@
 // other stream's bookkeeping.
 // The V1 epilogue writes each softmax warp's 32 output rows (and in the
 // training forward its saved fp32 branch outputs, 8 columns at a time)
-// through a 4 KB shared-memory block and TMA tensor stores (V2's shared
-// memory has no room for the 32 KB; it stores from registers).
+// through a 4 KB shared-memory block and TMA tensor stores; so does the V2
+// training forward (with three K/V ring slots to make room), while V2
+// inference stores from registers.
 // Softmax keeps a per-row reference maximum and only rescales O (in tensor
 // memory) when a new row maximum exceeds it by more than 2^8, so P <= 256.
 // Causal masking is applied only on the tiles that cross the diagonal (and
@@ -83,9 +84,10 @@ namespace {
 constexpr int kBM = 128;                   // query rows per CTA
 constexpr int kBN = 64;                    // keys per KV tile
 // Output (and, for the training forward, the saved branch outputs) staged
-// through shared memory and written by TMA stores: V1 only, V2's shared
-// memory has no room for the 32 KB
-__host__ __device__ constexpr bool stage_out(int form, bool save) { return form == 1; }
+// through shared memory and written by TMA stores: V1, and the V2 training
+// forward, which makes room for the 32 KB with a three-slot K/V ring (V2
+// inference keeps four slots and stores from registers)
+__host__ __device__ constexpr bool stage_out(int form, bool save) { return form == 1 || save; }
 // score-MMA issuer warps and threads per CTA, by form
 __host__ __device__ constexpr int score_issuers(int form) { return form == 1 ? 1 : 2; }
 __host__ __device__ constexpr int cta_threads(int form) { return (11 + score_issuers(form)) * 32; }
@@ -93,7 +95,8 @@ constexpr int kQBox = kBM * 64 * 2;        // TMA box of Q: 128 rows x 64 bf16 =
 constexpr int kQTile = 2 * kQBox;          // one 128 x 128 query tile
 constexpr int kKVBox = kBN * 64 * 2;       // TMA box of K/V: 64 rows x 64 bf16 = 8 KB
 constexpr int kKVTile = 2 * kKVBox;        // one 64 x 128 key or value tile
-constexpr int kStages = 4;
+constexpr int kStages = 4;  // K/V ring slots (barriers are sized for this many)
+__host__ __device__ constexpr int kv_stages(int form, bool save) { return form == 2 && save ? 3 : 4; }
 constexpr uint32_t kColS1 = 0, kColS2 = 128, kColO1 = 256, kColO2 = 384;
 constexpr float kLazyTau = 8.0f;           // log2 units: rescale only when max grows by > 2^8
 
@@ -291,9 +294,10 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t qbytes = kForm == 1 ? kQTile : 2 * kQTile;
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + qbytes;                         // kStages x kKVTile
-  uint8_t* sV = sK + kStages * kKVTile;                // kStages x kKVTile
-  Barriers* bars = reinterpret_cast<Barriers*>(sV + kStages * kKVTile);
+  constexpr int kSt = kv_stages(kForm, kSave);
+  uint8_t* sK = smem + qbytes;
+  uint8_t* sV = sK + kSt * kKVTile;
+  Barriers* bars = reinterpret_cast<Barriers*>(sV + kSt * kKVTile);
   float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [tile parity][2][128]
   float* x_ss = x_inv_l + 4 * kBM;                       // [tile parity][2][128]
   // output staging (V1): per softmax warp, its 32 rows x 64 bf16
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 2);        // released by both branches' score MMAs
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 2);   // released by both branches' MMAs
       mbar_init(&bars->v_full[s], 1);
@@ -382,8 +386,8 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
           tma_load_4d(sQ + 3 * kQBox, &tm_q, &bars->q_full, 64, 2 * T.hh + 1, T.q0, T.b);
         }
         for (int j = 0; j < T.n_kv; ++j, ++J) {
-          const int s = J % kStages;
-          const uint32_t ph = (J / kStages) & 1u;
+          const int s = J % kSt;
+          const uint32_t ph = (J / kSt) & 1u;
           const int key = (T.kv0 + j) * kBN;
           if (!mbar_wait(&bars->k_empty[s], ph ^ 1u, p.dev_status, &failed)) break;
           mbar_arrive_expect_tx(&bars->k_full[s], kKVTile);
@@ -425,8 +429,8 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
         const Tile T = tile_at(p, id, kForm, kWindow);
         if (!mbar_wait(&bars->q_full, (uint32_t)tc & 1u, p.dev_status, &failed)) break;
         for (int j = 0; j < T.n_kv; ++j, ++J) {
-          const int s = J % kStages;
-          if (!mbar_wait(&bars->k_full[s], (J / kStages) & 1u, p.dev_status, &failed)) break;
+          const int s = J % kSt;
+          if (!mbar_wait(&bars->k_full[s], (J / kSt) & 1u, p.dev_status, &failed)) break;
           const uint32_t kt = k_addr + s * kKVTile;
           for (int r = r0; r < r1; ++r) {
             // buffer J % 2 last held P_r(J-2): its P.V must have completed
@@ -470,8 +474,8 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
         if (id < 0) break;
         const Tile T = tile_at(p, id, kForm, kWindow);
         for (int j = 0; j < T.n_kv; ++j, ++J) {
-          const int s = J % kStages;
-          if (!mbar_wait(&bars->v_full[s], (J / kStages) & 1u, p.dev_status, &failed)) break;
+          const int s = J % kSt;
+          if (!mbar_wait(&bars->v_full[s], (J / kSt) & 1u, p.dev_status, &failed)) break;
           // the first P.V of a tile overwrites O: the previous tile's
           // epilogue must have read it out
           if (j == 0 && tc > 0 &&
@@ -910,7 +914,8 @@ cudaError_t launch_prefill_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   p.obr = static_cast<float*>(a.obr);
   p.dev_status = a.dev_status;
   const int qbytes = a.form == 1 ? kQTile : 2 * kQTile;
-  const int smem = 1024 + qbytes + 2 * kStages * kKVTile + (int)sizeof(Barriers) +
+  const int smem = 1024 + qbytes + 2 * kv_stages(a.form, a.lse && a.obr) * kKVTile +
+                   (int)sizeof(Barriers) +
                    8 * kBM * (int)sizeof(float) +
                    (stage_out(a.form, a.lse && a.obr) ? 8 * 4096 + 1024 : 0) + 64;
   const bool win = a.window > 0;
