@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
   Barriers* bars = reinterpret_cast<Barriers*>(sV + kSt * kKVTile);
   float* x_inv_l = reinterpret_cast<float*>(bars + 1);  // [tile parity][2][128]
   float* x_ss = x_inv_l + 4 * kBM;                       // [tile parity][2][128]
-  // output staging (V1): per softmax warp, its 32 rows x 64 bf16
+  // output staging (V1; V2 training forward): per softmax warp, its 32 rows x 64 bf16
   // (128-byte rows, the 16-byte chunks of row t at positions c ^ (t & 7));
   // 1024-byte aligned, as the 128-byte swizzle of the TMA box requires
   uint8_t* x_out = reinterpret_cast<uint8_t*>(
@@ -755,9 +755,9 @@ __global__ void __launch_bounds__(cta_threads(kForm), 1)
         mul = p.post_scale / sqrtf(tot * (1.0f / 128.0f) + p.eps);
       }
       if constexpr (stage_out(kForm, kSave)) {
-        // V1: the warp's 32 rows leave by one TMA tensor store from its
-        // staging block (128-byte swizzled, the layout of the output map's
-        // box).  Stored directly, each thread's 16-byte stores (rows 4 KB
+        // V1, and the V2 training forward: the warp's 32 rows leave by one
+        // TMA tensor store from its staging block (128-byte swizzled, the
+        // layout of the output map's box).  Stored directly, each thread's 16-byte stores (rows 4 KB
         // apart) would still be draining when the next tile's first P is
         // released, and that release waits for them; the bulk store is
         // outside that ordering.  Rows past the sequence end are clipped by
