@@ -17,6 +17,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import sys
@@ -84,11 +85,21 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
 
 
+def code_without_comments(text: str) -> str:
+    """Source text with // comments, /* */ comments and blank lines removed
+    (string literals in these files hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def kernel_source_hash():
+    """Hash of the prefill kernel's code (comments excluded: they do not change
+    the kernel), which a recorded traffic figure must match to be reported."""
     h = hashlib.sha256()
     for rel in ("prefill_tc.cu", "ptx.cuh"):
-        with open(os.path.join(ROOT, "differential_attention_sm_b200", "csrc", rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "differential_attention_sm_b200", "csrc", rel)) as f:
+            h.update(code_without_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 
