@@ -42,3 +42,15 @@ def test_oracle_samplers_run_and_count_work():
                                          np.arange(P)),
         (d["k_cache"], d["v_cache"]), 3, bench.v2_decode_bytes(1, 50, 2, 16, 4), 4)
     assert runs(2) == 2 * bench.v2_decode_bytes(1, 50, 2, 16, 4)
+
+
+def test_kernel_hash_ignores_comments_only():
+    """The hash that keys the recorded DRAM traffic changes with the code and
+    not with comments or blank lines."""
+    code = "int a = 1;  // one\n/* block\n comment */\nint b = a + 2;\n\n"
+    same = "// header\nint a = 1;\n\nint b = a + 2;  /* two */\n"
+    other = "int a = 1;\nint b = a + 3;\n"
+    strip = bench.code_without_comments
+    assert strip(code) == strip(same) == "int a = 1;\nint b = a + 2;"
+    assert strip(other) != strip(code)
+    assert len(bench.kernel_source_hash()) == 16
