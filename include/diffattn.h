@@ -32,9 +32,10 @@
  *    library calls no other library that keeps state.  Global state: for
  *    the bf16 tensor-core prefill (diffattn_v1_fwd / diffattn_v2_prefill
  *    and their window, training and projection variants), 64 tile counters
- *    per device in a statically allocated array.  The host gives each such launch the next
- *    counter in turn, fixed when the launch is enqueued (or captured into a
- *    CUDA graph, whose every replay then uses that counter).  On the device
+ *    per device in a statically allocated array.  The host gives each such
+ *    launch the next counter in turn, fixed when the launch is enqueued (or
+ *    captured into a CUDA graph, whose every replay then uses that
+ *    counter).  On the device
  *    a launch claims its counter when it is free, hands out one tile per
  *    ticket and frees it when its last tile is taken.  A launch that finds
  *    its counter held by another launch still in flight (two graph
