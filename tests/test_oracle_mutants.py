@@ -11,7 +11,8 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-# (text in the oracle, its mutated form, what the mistake is)
+# (text in the oracle, its mutated form, what the mistake is[, file under oracle/
+# when it is not the C source])
 MUTANTS = [
     ("double wj = a1[j] - lambda * a2[j];", "double wj = a1[j] + lambda * a2[j];", "lambda sign"),
     ("1.0 / sqrt((double)d)", "1.0 / sqrt((double)(2 * d))", "scale over the full head width"),
@@ -47,16 +48,38 @@ MUTANTS = [
      "        for (int c = 0; c < dv; ++c) dvj[c] += a1[j] * dout[c];", "backward: dV from map 1 only"),
     ("            dlk2[h * dim + c] = -e2 * (double)lq2[h * dim + c];",
      "            dlk2[h * dim + c] = -e2 * (double)lk2[h * dim + c];", "backward: lambda vector swap"),
+    ("dot2 += (double)lq2[(size_t)h * dim + c] * (double)lk2[(size_t)h * dim + c];",
+     "dot2 += (double)lq2[(size_t)h * dim + c] * (double)lk1[(size_t)h * dim + c];",
+     "lambda: second product with the first key vector"),
+    ("diff_attention_row(qa, qa + d, kb, kb, tok_kv, vb, tok_kv, len - first, d, d,",
+     "diff_attention_row(qa, qa, kb, kb, tok_kv, vb, tok_kv, len - first, d, d,",
+     "V2 decode: both branches from the pair's first head"),
+    ("int p = (int)(r % P), b = (int)(r / P), g = (2 * p) / group;",
+     "int p = (int)(r % P), b = (int)(r / P), g = p / group;", "V2 decode: GQA head mapping"),
+    ("diff_attention_row(qr, qr + d, kb, kb + d, tok_k, vb, tok_v, len - first, d, dv,",
+     "diff_attention_row(qr, qr + d, kb, kb, tok_k, vb, tok_v, len - first, d, dv,",
+     "V1 decode: branch-2 key half"),
+    ("lambda[h], a1, a2, NULL, o);\n        if (apply_norm) head_rms_norm(",
+     "lambda[h], a1, a2, NULL, o);\n        if (0) head_rms_norm(", "V1 decode: norm skipped"),
+    ("const int64_t qb = qa + d;", "const int64_t qb = qa;",
+     "V2 backward: both branches from the pair's first head"),
+    ("const int g = (2 * p) / group;", "const int g = p / group;", "V2 backward: GQA head mapping"),
+    # the output projection is numpy arithmetic in oracle.py
+    ("return o.reshape(t.size, P * d) @ w", "return o.reshape(t.size, P * d) @ w.T",
+     "output projection: O_W transposed", "oracle.py"),
+    ("return o.reshape(t.size, P * d) @ w",
+     "return o.reshape(t.size, P, d).transpose(0, 2, 1).reshape(t.size, P * d) @ w",
+     "output projection: channel-major flattening of the pair rows", "oracle.py"),
 ]
 
 
-def _run_mutant(tmp_root, n, before, after):
-    src = open(os.path.join(ROOT, "oracle", "diffattn_oracle.c")).read()
+def _run_mutant(tmp_root, n, before, after, fname="diffattn_oracle.c"):
+    src = open(os.path.join(ROOT, "oracle", fname)).read()
     assert before in src, before
     d = os.path.join(tmp_root, "m%d" % n)
     shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(d, "oracle"),
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
-    with open(os.path.join(d, "oracle", "diffattn_oracle.c"), "w") as f:
+    with open(os.path.join(d, "oracle", fname), "w") as f:
         f.write(src.replace(before, after, 1))
     os.makedirs(os.path.join(d, "tests"))
     for name in ("conftest.py", "test_oracle_pins.py"):
@@ -73,6 +96,6 @@ def _run_mutant(tmp_root, n, before, after):
 def test_pins_reject_every_planted_mistake(tmp_path):
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         rcs = list(ex.map(lambda a: _run_mutant(str(tmp_path), *a),
-                          [(n, b, a) for n, (b, a, _) in enumerate(MUTANTS)]))
+                          [(n, m[0], m[1], *m[3:]) for n, m in enumerate(MUTANTS)]))
     missed = [MUTANTS[n][2] for n, rc in enumerate(rcs) if rc == 0]
     assert not missed, "pins did not notice: %s" % missed
