@@ -64,6 +64,15 @@ MUTANTS = [
     ("const int64_t qb = qa + d;", "const int64_t qb = qa;",
      "V2 backward: both branches from the pair's first head"),
     ("const int g = (2 * p) / group;", "const int g = p / group;", "V2 backward: GQA head mapping"),
+    ("dkj[c] += ds * (double)qr[c];", "dkj[c] += ds * (double)kj[c];",
+     "backward: dK from the key instead of the query"),
+    ("double *dqr = r == 0 ? dq1 : dq2;", "double *dqr = r == 0 ? dq1 : dq1;",
+     "backward: branch-2 dQ into branch 1's half"),
+    ("dnorm_weight[c] += (double)dy[c] * o[c] * cpost / r;",
+     "dnorm_weight[c] += (double)dy[c] * o[c] / r;", "backward: gain gradient without (1 - lambda_init)"),
+    ("const int64_t first = window_start(n_keys, window);\n                const int64_t tq",
+     "const int64_t first = window_start(n_keys, 0);\n                const int64_t tq",
+     "V1 backward: window ignored"),
     # the output projection is numpy arithmetic in oracle.py
     ("return o.reshape(t.size, P * d) @ w", "return o.reshape(t.size, P * d) @ w.T",
      "output projection: O_W transposed", "oracle.py"),
