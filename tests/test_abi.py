@@ -117,6 +117,31 @@ def test_decode_workspace_and_validation(lib):
     assert g(*args) == b.DA_ERR_ALIGNMENT
 
 
+def test_noalloc_host_validation(lib):
+    """diffattn_v2_decode_noalloc refuses bad arguments, and sizes whose
+    partial results do not fit its fixed 8 MiB scratch, before touching the
+    device."""
+    from differential_attention_sm_b200 import binding as b
+    f = lib.diffattn_v2_decode_noalloc
+    #        q  k  v  lens  L    out batch Hq Hkv lam status stream
+    args = [A, A, A, None, 200, A, 252, 16, 8, A, None, None]
+    bad = list(args)
+    bad[0] = None
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(args)
+    bad[8] = 16                                   # a group of one query head
+    assert f(*bad) == b.DA_ERR_INVALID_ARG
+    bad = list(args)
+    bad[7], bad[8] = 32, 2                        # a group of 16
+    assert f(*bad) == b.DA_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[5] = U
+    assert f(*bad) == b.DA_ERR_ALIGNMENT
+    # 2017 units (batch x KV heads), one more than the scratch holds
+    assert f(A, A, A, None, 200, A, 2017, 2, 1, A, None, None) == b.DA_ERR_UNSUPPORTED
+    assert f(A, A, A, None, 64, A, 4096, 64, 8, A, None, None) == b.DA_ERR_UNSUPPORTED
+
+
 def test_lambda_from_params_validation(lib):
     from differential_attention_sm_b200 import binding as b
     f = lib.lambda_from_params
