@@ -73,6 +73,12 @@ MUTANTS = [
     ("const int64_t first = window_start(n_keys, window);\n                const int64_t tq",
      "const int64_t first = window_start(n_keys, 0);\n                const int64_t tq",
      "V1 backward: window ignored"),
+    ("    for (int64_t j = 0; j < n; ++j) x[j] /= s;", "    (void)s;",
+     "softmax not normalised"),
+    ("double inv_rms = 1.0 / sqrt(ss / (double)dv + eps);",
+     "double inv_rms = 1.0 / (sqrt(ss / (double)dv) + eps);", "RMS norm: epsilon outside the root"),
+    ("return 0.8 - 0.6 * exp(-0.3 * (double)(layer - 1));",
+     "return 0.8 - 0.6 * exp(-0.03 * (double)(layer - 1));", "lambda_init decay rate"),
     # the output projection is numpy arithmetic in oracle.py
     ("return o.reshape(t.size, P * d) @ w", "return o.reshape(t.size, P * d) @ w.T",
      "output projection: O_W transposed", "oracle.py"),
